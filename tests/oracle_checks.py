@@ -1,0 +1,364 @@
+"""Pins for the CPU oracle: each check asserts something the pages or the
+mathematics fix, independently of the oracle's own code.
+
+The checks are plain functions so that `test_oracle_pins.py` runs them on the
+oracle as written and `test_oracle_mutants.py` runs them on oracles with a
+planted mistake, which at least one check must catch.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+from oracle import attention as oatt
+from oracle import blocks as oblk
+
+
+# ------------------------------------------------------------ block arithmetic
+
+def check_seven_token_prompt(g):
+    """Step 3 example: 7 tokens, 4 per block, logical 0 and 1 -> physical 7 and 1."""
+    ex = g["seven_token_prompt"]
+    bs = ex["block_size"]
+    bm = oblk.BlockManager(num_blocks=8, block_size=bs)
+    first = ex["physical_blocks_of_logical_0_1"]
+    rest = [b for b in range(8) if b not in first]
+    bm.set_free_order(first + rest)
+    s = bm.new_sequence()
+    slots, cows = bm.add_tokens(s, ex["prompt_tokens"])
+    assert bm.tables[s] == first
+    assert cows == []
+    # tokens 0..3 in block 7 (slots 28..31), tokens 4..6 in block 1 (slots 4..6)
+    assert slots == [7 * 4 + i for i in range(4)] + [1 * 4 + i for i in range(3)]
+    # the last slot of block 1 waits for the next generated token: no new block
+    nxt, cow = bm.append_slot(s)
+    assert (nxt, cow) == (1 * 4 + 3, None)
+    assert bm.tables[s] == first
+    # the 9th token finds the tail full and takes the next free block
+    ninth, _ = bm.append_slot(s)
+    assert bm.tables[s] == first + [rest[0]]
+    assert ninth == rest[0] * 4
+
+
+def check_600_tokens(g):
+    ex = g["reserve_4096_use_600"]
+    assert oblk.blocks_for(ex["used_tokens"], ex["block_size"]) == ex["blocks"]
+    used = 100.0 * ex["used_tokens"] / ex["reserved_tokens"]
+    assert round(used) == ex["used_percent_about"]
+    assert round(100.0 - used) == ex["idle_percent_about"]
+
+
+def check_llama3_per_token(g):
+    ex = g["llama3_8b_per_token"]
+    per_token = oblk.kv_bytes_per_token(ex["layers"], ex["kv_heads"], ex["head_size"], 2)
+    assert per_token == ex["bytes_per_token"] == 128 * 1024
+    assert per_token * ex["max_positions"] == ex["bytes_per_full_reservation"] == 1 << 30
+    used = 100.0 * ex["request_tokens"] / ex["max_positions"]
+    assert round(used, 1) == ex["used_percent"]
+    assert round(100.0 - used, 1) == ex["wasted_percent"]
+
+
+def check_700_tokens(g):
+    ex = g["request_700_in_blocks"]
+    bs = ex["block_size"]
+    assert oblk.blocks_for(ex["tokens"], bs) == ex["blocks"]
+    slots = oblk.allocated_slots(ex["tokens"], bs)
+    assert slots == ex["slots"]
+    assert slots - ex["tokens"] == ex["idle_slots"]
+    assert round(100.0 * (slots - ex["tokens"]) / slots, 2) == ex["idle_percent"]
+
+
+def check_worked_example(g):
+    ex = g["worked_example"]
+    lens = ex["lengths"]
+    bs = ex["block_size"]
+    total = sum(lens)
+    assert total == ex["total_tokens"]
+    slab = len(lens) * g["llama3_8b_per_token"]["max_positions"]
+    assert slab == ex["slab_slots"]
+    assert round(100.0 * total / slab, 1) == ex["slab_used_percent"]
+    paged = sum(oblk.allocated_slots(n, bs) for n in lens)
+    assert paged == ex["paged_slots"]
+    assert round(100.0 * total / paged, 1) == ex["paged_used_percent"]
+
+
+def check_capacity(g):
+    """Slabs fit 59 requests in 64e9 B; blocks fit about 367.
+
+    The page's 367 follows from the batch's average ALLOCATED footprint,
+    10,640 / 8 = 1,330 slots per request; its quoted average of about 1,322
+    tokens is the filled count (10,578 / 8) and would give 369.
+    """
+    ex = g["worked_example"]
+    per_token = oblk.kv_bytes_per_token(32, 8, 128, 2)
+    budget = ex["cache_budget_bytes"]
+    slab_bytes = g["llama3_8b_per_token"]["max_positions"] * per_token
+    slabs = oblk.requests_that_fit(budget, slab_bytes)
+    assert slabs == ex["slab_requests"]
+    bs = ex["block_size"]
+    lens = ex["lengths"]
+    assert round(sum(lens) / len(lens)) == ex["average_length_about"]
+    avg_alloc = sum(oblk.allocated_slots(n, bs) for n in lens) / len(lens)
+    paged = oblk.requests_that_fit(budget, avg_alloc * per_token)
+    assert paged == ex["paged_requests_about"]
+    assert round(paged / slabs, 1) == ex["gain_times"]
+    # the filled-token reading lands two requests higher
+    assert oblk.requests_that_fit(budget, (sum(lens) / len(lens)) * per_token) == 369
+
+
+def check_worked_example_block_manager(g):
+    """The block manager holds the worked example in 665 blocks; one decode step
+    appends a token to every request: only the 128-token request (tail exactly
+    full) takes a new block, giving 666 blocks and 10,656 slots for 10,586 tokens."""
+    ex = g["worked_example"]
+    bs = ex["block_size"]
+    lens = ex["lengths"]
+    bm = oblk.BlockManager(num_blocks=700, block_size=bs)
+    seqs = []
+    for n in lens:
+        s = bm.new_sequence()
+        bm.add_tokens(s, n)
+        seqs.append(s)
+    held = sum(len(bm.tables[s]) for s in seqs)
+    assert held * bs == ex["paged_slots"]
+    assert bm.num_free() == 700 - held
+    before = {s: len(bm.tables[s]) for s in seqs}
+    for s in seqs:
+        bm.append_slot(s)
+    grew = [lens[i] for i, s in enumerate(seqs) if len(bm.tables[s]) > before[s]]
+    assert grew == [128]
+    assert sum(bm.lengths[s] for s in seqs) == ex["total_tokens"] + len(lens)
+    assert sum(len(bm.tables[s]) for s in seqs) == held + 1
+    assert (held + 1) * bs == 10_656
+    for s in seqs:
+        bm.free_sequence(s)
+    assert bm.num_free() == 700
+
+
+def check_sharing_and_copy_on_write():
+    """Fork shares every block (count + 1); the first write into a shared,
+    partly filled tail copies that one block only; counts return to zero."""
+    bm = oblk.BlockManager(num_blocks=16, block_size=4)
+    p = bm.new_sequence()
+    bm.add_tokens(p, 6)                       # blocks [0, 1], block 1 half full
+    c = bm.fork(p)
+    assert bm.tables[c] == bm.tables[p] == [0, 1]
+    assert bm.refcount[0] == bm.refcount[1] == 2
+    slot, cow = bm.append_slot(c)             # child writes into the shared tail
+    assert cow == (1, 2)                      # only the tail block is copied
+    assert bm.tables[c] == [0, 2] and bm.tables[p] == [0, 1]
+    assert slot == 2 * 4 + 2
+    assert bm.refcount[0] == 2 and bm.refcount[1] == 1 and bm.refcount[2] == 1
+    slot, cow = bm.append_slot(p)             # parent is now the only holder
+    assert cow is None and slot == 1 * 4 + 2
+    bm.free_sequence(c)
+    bm.free_sequence(p)
+    assert bm.num_free() == 16 and all(r == 0 for r in bm.refcount)
+
+
+def check_exhaustion_leaves_state():
+    bm = oblk.BlockManager(num_blocks=2, block_size=4)
+    s = bm.new_sequence()
+    bm.add_tokens(s, 8)
+    free_before, table_before = bm.num_free(), list(bm.tables[s])
+    try:
+        bm.add_tokens(s, 1)
+    except oblk.OutOfBlocks:
+        pass
+    else:
+        raise AssertionError("expected OutOfBlocks")
+    assert bm.num_free() == free_before and bm.tables[s] == table_before
+    assert bm.lengths[s] == 8
+
+
+# ------------------------------------------------------------------ attention
+
+def _contiguous_case(seed, lengths, hq, hkv, d, bs, num_blocks):
+    """Random contiguous K/V per sequence, stored through an explicit random placement."""
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(num_blocks)
+    k_cache = rng.standard_normal((num_blocks, bs, hkv, d))
+    v_cache = rng.standard_normal((num_blocks, bs, hkv, d))
+    max_blocks = max(-(-n // bs) for n in lengths)
+    tables = np.zeros((len(lengths), max_blocks), dtype=np.int64)
+    used = 0
+    for s, n in enumerate(lengths):
+        nb = -(-n // bs)
+        tables[s, :nb] = perm[used:used + nb]
+        used += nb
+    q = rng.standard_normal((len(lengths), hq, d))
+    return q, k_cache, v_cache, tables
+
+
+def _brute_force_decode(q, k_cache, v_cache, tables, lengths, scale, bs):
+    """Python loops and math.exp: walk the block table block by block."""
+    num_seqs, hq, d = q.shape
+    hkv = k_cache.shape[2]
+    out = np.zeros((num_seqs, hq, d))
+    for s in range(num_seqs):
+        n = int(lengths[s])
+        for j in range(hq):
+            h = j * hkv // hq
+            keys, vals = [], []
+            for lb in range(-(-n // bs)):
+                phys = int(tables[s][lb])
+                for off in range(bs):
+                    if lb * bs + off < n:
+                        keys.append(k_cache[phys][off][h])
+                        vals.append(v_cache[phys][off][h])
+            if not keys:
+                continue
+            xs = [scale * sum(float(q[s, j, i]) * float(k[i]) for i in range(d)) for k in keys]
+            top = max(xs)
+            es = [math.exp(x - top) for x in xs]
+            z = sum(es)
+            for i in range(d):
+                out[s, j, i] = sum(e * float(v[i]) for e, v in zip(es, vals)) / z
+    return out
+
+
+def check_brute_force_tiny():
+    lengths = [1, 4, 5, 9, 0]
+    bs, hq, hkv, d = 4, 4, 2, 4
+    q, kc, vc, tables = _contiguous_case(11, lengths, hq, hkv, d, bs, 12)
+    ref = _brute_force_decode(q, kc, vc, tables, lengths, 0.5, bs)
+    got = oatt.decode(q, kc, vc, tables, lengths, 0.5, bs)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def check_sdpa_identity_table():
+    """Identity table + contiguous cache equals torch's float64 SDPA with the
+    KV heads repeated G times (query head j -> KV head j // G)."""
+    import torch
+
+    rng = np.random.default_rng(7)
+    hq, hkv, d, bs, n = 8, 2, 16, 8, 37
+    nb = -(-n // bs)
+    kc = rng.standard_normal((nb, bs, hkv, d))
+    vc = rng.standard_normal((nb, bs, hkv, d))
+    q = rng.standard_normal((1, hq, d))
+    scale = 0.3
+    got = oatt.decode(q, kc, vc, np.arange(nb)[None, :], [n], scale, bs)
+    keys = torch.from_numpy(kc.reshape(nb * bs, hkv, d)[:n]).permute(1, 0, 2)   # [hkv, n, d]
+    vals = torch.from_numpy(vc.reshape(nb * bs, hkv, d)[:n]).permute(1, 0, 2)
+    keys = keys.repeat_interleave(hq // hkv, dim=0)
+    vals = vals.repeat_interleave(hq // hkv, dim=0)
+    qt = torch.from_numpy(q[0]).unsqueeze(1)                                      # [hq, 1, d]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, keys, vals, scale=scale)
+    assert np.max(np.abs(got[0] - ref[:, 0, :].numpy())) < 1e-12
+
+
+def check_closed_forms():
+    rng = np.random.default_rng(3)
+    hq, hkv, d, bs = 4, 2, 8, 4
+    # one cached token: the output is that token's value row, exactly
+    kc = rng.standard_normal((3, bs, hkv, d))
+    vc = rng.standard_normal((3, bs, hkv, d))
+    q = rng.standard_normal((1, hq, d))
+    out = oatt.decode(q, kc, vc, np.array([[2]]), [1], 0.7, bs)
+    for j in range(hq):
+        assert np.array_equal(out[0, j], vc[2, 0, j // 2])
+    # q = 0: uniform weights, the output is the mean of the value rows
+    table = np.array([[1, 0, 2]])
+    n = 10
+    out = oatt.decode(np.zeros((1, hq, d)), kc, vc, table, [n], 0.7, bs)
+    rows = np.concatenate([vc[1], vc[0], vc[2]])[:n]
+    for j in range(hq):
+        assert np.allclose(out[0, j], rows[:, j // 2].mean(axis=0), rtol=0, atol=1e-14)
+    # all keys equal: also uniform weights
+    kc_eq = np.broadcast_to(rng.standard_normal((1, 1, hkv, d)), kc.shape).copy()
+    out = oatt.decode(q, kc_eq, vc, table, [n], 0.7, bs)
+    for j in range(hq):
+        assert np.allclose(out[0, j], rows[:, j // 2].mean(axis=0), rtol=0, atol=1e-13)
+    # one dominant score (q parallel to key t, large): output is that value row
+    keys = np.concatenate([kc[1], kc[0], kc[2]])[:n]
+    t = 6
+    qd = np.zeros((1, hq, d))
+    for j in range(hq):
+        qd[0, j] = 40.0 * keys[t, j // 2] / np.linalg.norm(keys[t, j // 2])
+    out = oatt.decode(qd, kc, vc, table, [n], 1.0, bs)
+    for j in range(hq):
+        assert np.allclose(out[0, j], rows[t, j // 2], rtol=0, atol=1e-6)
+
+
+def check_placement_and_sharing_invariance():
+    """Output depends only on the logical token sequence: a different physical
+    placement, or prefix blocks shared instead of duplicated, gives the
+    identical float64 result."""
+    rng = np.random.default_rng(5)
+    hq, hkv, d, bs = 4, 2, 8, 4
+    n_prefix, n_a, n_b = 12, 3, 6          # prefix of 3 full blocks, then private tails
+    prefix_k = rng.standard_normal((n_prefix, hkv, d))
+    prefix_v = rng.standard_normal((n_prefix, hkv, d))
+    tail = {s: (rng.standard_normal((m, hkv, d)), rng.standard_normal((m, hkv, d)))
+            for s, m in ((0, n_a), (1, n_b))}
+    q = rng.standard_normal((2, hq, d))
+
+    def store(order, share):
+        nb = 16
+        kc = np.full((nb, bs, hkv, d), np.nan)
+        vc = np.full((nb, bs, hkv, d), np.nan)
+        free = list(order)
+        tables = np.zeros((2, 5), dtype=np.int64)
+        shared = [free.pop(0) for _ in range(3)] if share else None
+        for s in (0, 1):
+            kt = np.concatenate([prefix_k, tail[s][0]])
+            vt = np.concatenate([prefix_v, tail[s][1]])
+            nblk = -(-len(kt) // bs)
+            ids = list(shared) + [free.pop(0) for _ in range(nblk - 3)] if share else \
+                [free.pop(0) for _ in range(nblk)]
+            for t in range(len(kt)):
+                kc[ids[t // bs], t % bs] = kt[t]
+                vc[ids[t // bs], t % bs] = vt[t]
+            tables[s, :nblk] = ids
+        return kc, vc, tables
+
+    lens = [n_prefix + n_a, n_prefix + n_b]
+    base = oatt.decode(q, *store(range(16), False), lens, 0.4, bs)
+    for order in (rng.permutation(16), rng.permutation(16)):
+        assert np.array_equal(base, oatt.decode(q, *store(order, False), lens, 0.4, bs))
+        assert np.array_equal(base, oatt.decode(q, *store(order, True), lens, 0.4, bs))
+
+
+def check_append_and_copy_roundtrip():
+    rng = np.random.default_rng(9)
+    nb, bs, hkv, d = 6, 4, 2, 3
+    kc = rng.standard_normal((nb, bs, hkv, d))
+    vc = rng.standard_normal((nb, bs, hkv, d))
+    k_new = rng.standard_normal((4, hkv, d))
+    v_new = rng.standard_normal((4, hkv, d))
+    slots = np.array([5 * 4 + 1, -1, 0, 2 * 4 + 3])
+    k2, v2 = oatt.kv_append(kc, vc, k_new, v_new, slots, bs)
+    for i, slot in enumerate(slots):
+        if slot >= 0:
+            assert np.array_equal(k2[slot // bs, slot % bs], k_new[i])
+            assert np.array_equal(v2[slot // bs, slot % bs], v_new[i])
+    touched = {(int(x) // bs, int(x) % bs) for x in slots if x >= 0}
+    for b in range(nb):
+        for o in range(bs):
+            if (b, o) not in touched:
+                assert np.array_equal(k2[b, o], kc[b, o]) and np.array_equal(v2[b, o], vc[b, o])
+    # gather through a table returns exactly what was appended
+    table = np.array([5])
+    got = oatt.gather_context(k2, table, 2, bs)
+    assert np.array_equal(got[1], k_new[0])
+    k3, v3 = oatt.copy_blocks(k2, v2, np.array([[5, 1], [0, 4]]))
+    assert np.array_equal(k3[1], k2[5]) and np.array_equal(v3[4], v2[0])
+    for b in (0, 2, 3, 5):
+        assert np.array_equal(k3[b], k2[b]) and np.array_equal(v3[b], v2[b])
+
+
+BLOCK_CHECKS = [
+    check_seven_token_prompt, check_600_tokens, check_llama3_per_token, check_700_tokens,
+    check_worked_example, check_capacity, check_worked_example_block_manager,
+]
+PLAIN_BLOCK_CHECKS = [check_sharing_and_copy_on_write, check_exhaustion_leaves_state]
+ATTENTION_CHECKS = [
+    check_brute_force_tiny, check_sdpa_identity_table, check_closed_forms,
+    check_placement_and_sharing_invariance, check_append_and_copy_roundtrip,
+]
+
+assert oracle is not None

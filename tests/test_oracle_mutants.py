@@ -1,0 +1,82 @@
+"""Each planted mistake in the CPU oracle must fail at least one pin.
+
+The mistakes are planted in the oracle on the CPU (monkeypatch), never in the
+CUDA library. A mutant that every pin accepts would mean the pins cannot see
+that kind of error.
+"""
+
+import numpy as np
+import pytest
+
+import oracle_checks as oc
+from oracle import attention as oatt
+from oracle import blocks as oblk
+
+
+def _fails_some_check(golden):
+    failed = []
+    for check in oc.BLOCK_CHECKS:
+        try:
+            check(golden)
+        except Exception:  # noqa: BLE001 - any failure counts as caught
+            failed.append(check.__name__)
+    for check in oc.PLAIN_BLOCK_CHECKS + oc.ATTENTION_CHECKS:
+        try:
+            check()
+        except Exception:  # noqa: BLE001
+            failed.append(check.__name__)
+    return failed
+
+
+def _softmax_no_scale(q_vec, keys, values, scale):
+    x = np.asarray(keys, np.float64) @ np.asarray(q_vec, np.float64)
+    w = np.exp(x - x.max())
+    return (w / w.sum()) @ np.asarray(values, np.float64)
+
+
+def _softmax_unnormalised(q_vec, keys, values, scale):
+    x = scale * (np.asarray(keys, np.float64) @ np.asarray(q_vec, np.float64))
+    return np.exp(x - x.max()) @ np.asarray(values, np.float64)
+
+
+def _softmax_keys_as_values(q_vec, keys, values, scale):
+    x = scale * (np.asarray(keys, np.float64) @ np.asarray(q_vec, np.float64))
+    w = np.exp(x - x.max())
+    return (w / w.sum()) @ np.asarray(keys, np.float64)
+
+
+def _softmax_drop_last(q_vec, keys, values, scale):
+    keys, values = np.asarray(keys, np.float64), np.asarray(values, np.float64)
+    if len(keys) > 1:
+        keys, values = keys[:-1], values[:-1]
+    x = scale * (keys @ np.asarray(q_vec, np.float64))
+    w = np.exp(x - x.max())
+    return (w / w.sum()) @ values
+
+
+MUTANTS = {
+    "gqa_heads_interleaved": (oatt, "kv_head_of", lambda j, g: j % g),
+    "gqa_always_head0": (oatt, "kv_head_of", lambda j, g: 0),
+    "offset_off_by_one": (oblk, "logical_position", lambda t, bs: (t // bs, (t + 1) % bs)),
+    "block_index_swapped": (oblk, "logical_position", lambda t, bs: (t % bs, t // bs)),
+    "blocks_floor": (oblk, "blocks_for", lambda n, bs: n // bs),
+    "blocks_one_extra": (oblk, "blocks_for", lambda n, bs: n // bs + 1),
+    "kv_bytes_no_v": (oblk, "kv_bytes_per_token", lambda L, h, d, e: L * h * d * e),
+    "scale_dropped": (oatt, "softmax_attention", _softmax_no_scale),
+    "softmax_not_normalised": (oatt, "softmax_attention", _softmax_unnormalised),
+    "keys_used_as_values": (oatt, "softmax_attention", _softmax_keys_as_values),
+    "last_token_dropped": (oatt, "softmax_attention", _softmax_drop_last),
+    "slot_without_block_size": (oblk, "slot_of",
+                                lambda table, t, bs: int(table[t // bs]) + t % bs),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, golden, monkeypatch):
+    module, attr, bad = MUTANTS[name]
+    monkeypatch.setattr(module, attr, bad)
+    assert _fails_some_check(golden), f"mutant {name} passed every pin"
+
+
+def test_unmutated_oracle_passes_every_check(golden):
+    assert _fails_some_check(golden) == []
