@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of a batch: pa_kv_append of each sequence's new
+token, then pa_decode over every sequence's whole cached context (split-K
+partitions merged by a second kernel when a sequence spans more than one).
+Default workload: one Llama-3-8B-shaped layer (32/8 heads, head_dim 128, bf16,
+block 16) holding the eight requests of the pages' worked example
+(128, 700, 1500, 300, 2900, 50, 4100, 900 cached tokens), physical blocks a
+seeded random permutation of a 2048-block pool.
+
+Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the
+launching stream; the L2 is flushed (a 2 x L2 write) between steps, outside
+the events. Under torchrun each rank runs its own replica (replicas only:
+sequences never exchange data) and the time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference   # the float64 CPU oracle as the reference arm
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (fraction of HBM peak) and attended tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default="llama3_8b_layer",
+                    choices=["llama3_8b_layer", "large_batch", "shared_prefix", "long_context"])
+    ap.add_argument("--block-size", type=int, default=16, help="long_context only")
+    ap.add_argument("--partition-size", type=int, default=-1,
+                    help="tokens per split-K partition (-1: tuned default, 0: library choice)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def make_workload(name: str, block_size: int):
+    from workloads import configs
+
+    if name == "long_context":
+        return configs.long_context(block_size)
+    if name == "large_batch":
+        return configs.large_batch(steps=1)
+    return configs.ALL[name]()
+
+
+# Partition sizes measured best per workload (tokens); -1 on the command line picks these.
+TUNED_PARTITION = {"llama3_8b_layer": 0, "large_batch": 0, "shared_prefix": 0,
+                   "long_context": 512}
+
+
+def kv_bytes(wl) -> int:
+    """K and V bytes the decode step reads: every attended token, every KV head."""
+    return sum(n + 1 for n in wl.context_lens) * wl.num_kv_heads * 2 * wl.head_dim * wl.elem_bytes
+
+
+# ------------------------------------------------------------------ GPU setup
+
+def build_on_gpu(wl, device):
+    """Prefill every sequence through the library, then prepare one decode step."""
+    import torch
+
+    from paged_kv_cache_345_b200.cache import PagedKVCache
+    from workloads import synth
+
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    bs = wl.block_size
+    max_blocks = max(-(-(n + 1) // bs) for n in wl.context_lens)
+    cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.dtype, device,
+                         max_blocks_per_seq=max_blocks,
+                         free_order=synth.block_permutation(wl.num_blocks, wl.placement_seed))
+    ghosts = [cache.add_sequence() for _ in wl.ghost_lens]
+    if ghosts:
+        cache.bm.append_slots(ghosts, list(wl.ghost_lens))
+        for i in range(0, len(ghosts), 2):
+            cache.free(ghosts[i])
+
+    def rows(seq_index, n):
+        k, v = synth.kv_rows(wl.value_seed, seq_index, n, wl.num_kv_heads, wl.head_dim)
+        return (torch.from_numpy(k).to(device=device, dtype=tdt),
+                torch.from_numpy(v).to(device=device, dtype=tdt))
+
+    start = 0
+    if wl.shared_prefix:
+        parent = cache.add_sequence()
+        pk, pv = rows(100_000, wl.shared_prefix)
+        cache.write([parent], [wl.shared_prefix], pk, pv)
+        seqs = [parent] + [cache.fork(parent) for _ in range(wl.num_seqs - 1)]
+        start = wl.shared_prefix
+    else:
+        seqs = [cache.add_sequence() for _ in range(wl.num_seqs)]
+    cow_pairs = 0
+    for s, n in enumerate(wl.context_lens):     # one sequence at a time bounds host memory
+        if n - start > 0:
+            k, v = rows(s, n - start)
+            slots, cows = cache.bm.append_slots([seqs[s]], [n - start])
+            cow_pairs += len(cows)
+            if len(cows):
+                from paged_kv_cache_345_b200 import pa_copy_blocks
+                pa_copy_blocks(cache.k_cache, cache.v_cache, torch.from_numpy(cows).to(device))
+            from paged_kv_cache_345_b200 import pa_kv_append
+            pa_kv_append(k, v, torch.from_numpy(slots).to(device), cache.k_cache, cache.v_cache)
+    torch.cuda.synchronize(device)
+
+    # the decode step: one new token per sequence, appended then attended
+    new_k, new_v = synth.new_token_kv(wl.value_seed, 0, wl.num_seqs, wl.num_kv_heads, wl.head_dim)
+    q = synth.queries(wl.value_seed, 0, wl.num_seqs, wl.num_heads, wl.head_dim)
+    slots, cows = cache.bm.append_slots(seqs, [1] * len(seqs))
+    assert len(cows) == 0
+    tables, lens = cache.bm.block_tables(seqs, max_blocks)
+    host = {
+        "q": torch.from_numpy(q).to(tdt).pin_memory(),
+        "k_new": torch.from_numpy(new_k).to(tdt).pin_memory(),
+        "v_new": torch.from_numpy(new_v).to(tdt).pin_memory(),
+        "slots": torch.from_numpy(slots).pin_memory(),
+        "tables": torch.from_numpy(tables).pin_memory(),
+        "lens": torch.from_numpy(lens).pin_memory(),
+    }
+    dev = {k: v.to(device) for k, v in host.items()}
+    return cache, seqs, host, dev, int(lens.max()), cow_pairs
+
+
+class StepCalls:
+    """The C-ABI calls of one decode step with their arguments marshalled once."""
+
+    def __init__(self, cache, dev, max_len, scale, partition_size, stream):
+        import torch
+
+        import paged_kv_cache_345_b200 as pa
+
+        self.lib = pa._lib
+        s, hq, d = dev["q"].shape
+        nb, bs, hkv, _ = cache.k_cache.shape
+        dt = pa.PA_BF16 if cache.k_cache.dtype == torch.bfloat16 else pa.PA_F32
+        self.partition_size = partition_size or pa.pa_decode_partition_size(s, hkv, max_len)
+        ws_bytes = pa.pa_decode_workspace_bytes(s, hq, hkv, d, max_len, self.partition_size)
+        self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev["q"].device)
+        self.out = torch.empty_like(dev["q"])
+        self.num_partitions = -(-max_len // self.partition_size)
+        st = ctypes.c_void_p(stream.cuda_stream)
+        p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        self.append_args = (p(dev["k_new"]), p(dev["v_new"]), p(dev["slots"]), s,
+                            p(cache.k_cache), p(cache.v_cache), nb, bs, hkv, d, dt, st)
+        self.decode_args = (p(self.out), p(dev["q"]), p(cache.k_cache), p(cache.v_cache),
+                            p(dev["tables"]), p(dev["lens"]), s, hq, hkv, d, bs, nb,
+                            dev["tables"].shape[1], max_len, scale, self.partition_size,
+                            p(self.workspace), self.workspace.numel(), dt, st)
+        self.launches_per_step = 2 + (1 if self.num_partitions > 1 else 0)
+
+    def append(self):
+        st = self.lib.pa_kv_append(*self.append_args)
+        if st:
+            raise RuntimeError(f"pa_kv_append: {self.lib.pa_last_error().decode()}")
+
+    def decode(self):
+        st = self.lib.pa_decode(*self.decode_args)
+        if st:
+            raise RuntimeError(f"pa_decode: {self.lib.pa_last_error().decode()}")
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# -------------------------------------------------------------- CPU baseline
+
+def oracle_inputs(wl):
+    """The oracle's own cache (float64) built by its own block manager from the
+    same seeded rows and free order; never read back from the GPU."""
+    from oracle import attention as oatt
+    from oracle import blocks as oblk
+    from workloads import synth
+
+    def stored(x):
+        return synth.round_to_bf16(x) if wl.dtype == "bf16" else x
+
+    ob = oblk.BlockManager(wl.num_blocks, wl.block_size)
+    ob.set_free_order(synth.block_permutation(wl.num_blocks, wl.placement_seed).tolist())
+    kc = np.zeros((wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim))
+    vc = np.zeros_like(kc)
+    new_k, new_v = synth.new_token_kv(wl.value_seed, 0, wl.num_seqs, wl.num_kv_heads, wl.head_dim)
+    seqs = []
+    for s, n in enumerate(wl.context_lens):
+        sid = ob.new_sequence()
+        seqs.append(sid)
+        k, v = synth.kv_rows(wl.value_seed, s, n, wl.num_kv_heads, wl.head_dim)
+        k = np.concatenate([stored(k), stored(new_k[s:s + 1])])
+        v = np.concatenate([stored(v), stored(new_v[s:s + 1])])
+        slots, _ = ob.add_tokens(sid, n + 1)
+        kc, vc = oatt.kv_append(kc, vc, k, v, slots, wl.block_size)
+    mb = max(len(ob.tables[s]) for s in seqs)
+    tables = np.zeros((len(seqs), mb), dtype=np.int64)
+    for i, s in enumerate(seqs):
+        tables[i, :len(ob.tables[s])] = ob.tables[s]
+    q = stored(synth.queries(wl.value_seed, 0, wl.num_seqs, wl.num_heads, wl.head_dim))
+    return q, kc, vc, tables, [ob.lengths[s] for s in seqs]
+
+
+def cpu_oracle_run(wl, budget_s: float, min_steps: int = 1, max_steps: int | None = None):
+    """Time the oracle's decode step on the host cores: whole steps, repeated
+    until `budget_s` is spent (at least min_steps, at most max_steps)."""
+    from oracle import attention as oatt
+
+    if wl.shared_prefix or wl.ghost_lens or sum(wl.context_lens) > 200_000:
+        raise ValueError("the CPU oracle leg runs the single-layer worked-example workload")
+    q, kc, vc, tables, lens = oracle_inputs(wl)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while len(times) < min_steps or (time.perf_counter() < t_end and
+                                     (max_steps is None or len(times) < max_steps)):
+        t0 = time.perf_counter()
+        oatt.decode(q, kc, vc, tables, lens, wl.scale, wl.block_size)
+        times.append(time.perf_counter() - t0)
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        blas = 1
+    return times, max(1, min(cores, blas))
+
+
+# --------------------------------------------------------------------- arms
+
+def run_reference(args, wl, rank):
+    """The reference arm: the float64 CPU oracle, as it stands, on the same workload."""
+    if rank != 0:
+        return
+    bytes_step = kv_bytes(wl)
+    _, _ = cpu_oracle_run(wl, 0.0, min_steps=max(1, args.warmup), max_steps=max(1, args.warmup))
+    times, cores = cpu_oracle_run(wl, 0.0, min_steps=args.steps, max_steps=args.steps)
+    total = sum(times)
+    value = bytes_step * len(times) / total / 1e9
+    sample = f"{len(times)} whole decode steps of the {wl.num_seqs}-sequence batch"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": wl.num_seqs,
+                   "context_lens": list(wl.context_lens), "block_size": wl.block_size},
+        "attended_tokens_per_s": sum(n + 1 for n in wl.context_lens) * len(times) / total,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def load_traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (matching source hash), else None."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"{kernel_key}.traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "paged_kv_cache_345_b200", "csrc", "pa_decode.cuh")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if vals.get("source_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_b200(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_345_b200 as pa
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device)
+    stream = torch.cuda.current_stream(device)
+
+    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device)
+    ps = TUNED_PARTITION[wl.name.split("_bs")[0]] if args.partition_size < 0 else args.partition_size
+    calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream)
+    bytes_step = kv_bytes(wl)
+    tokens_step = sum(n + 1 for n in wl.context_lens)
+
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(device)
+
+    # ---- device-resident steps
+    for _ in range(args.warmup):
+        flush.zero_()
+        calls.append()
+        calls.decode()
+    torch.cuda.synchronize(device)
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        calls.append()
+        ev[i][1].record(stream)
+        calls.decode()
+        ev[i][2].record(stream)
+    barrier()
+    wall = time.perf_counter() - t_wall
+    clk = clocks.stop()
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    decode_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+
+    # ---- end to end: pinned host inputs -> device -> kernels -> host output
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(calls.out.shape, dtype=calls.out.dtype).pin_memory()
+        names = ("q", "k_new", "v_new", "slots", "tables", "lens")
+        h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step():
+            for k in names:
+                dev[k].copy_(host[k], non_blocking=True)
+            calls.append()
+            calls.decode()
+            out_host.copy_(calls.out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            e2e_step()
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            ee[i][0].record(stream)
+            e2e_step()
+            ee[i][1].record(stream)
+        barrier()
+        e2e_ms = sum(ee[i][0].elapsed_time(ee[i][1]) for i in range(args.steps))
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": bytes_step * args.steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.steps}
+
+    # ---- roofline of pa_decode (decode kernel + split-K merge kernel)
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        peak, peak_src = float(json.load(open(peaks_path))["hbm_gbs"]), "measured"
+    else:
+        peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+    dec_s = statistics.mean(decode_ms) * 1e-3
+    achieved = bytes_step / dec_s / 1e9
+    traffic = load_traffic(f"pa_decode_{wl.name}")
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            times, cores = cpu_oracle_run(wl, args.cpu_budget_s)
+            cpu = {"value": bytes_step * len(times) / sum(times) / 1e9, "unit": "GB/s",
+                   "cores": cores, "kind": "oracle",
+                   "sample": f"{len(times)} whole decode steps of the {wl.num_seqs}-sequence "
+                             f"batch in {sum(times):.1f} s (float64 NumPy)"}
+        except ValueError as exc:
+            cpu = {"value": None, "unit": "GB/s", "cores": 0, "kind": "oracle",
+                   "sample": f"not run: {exc}"}
+
+    value = bytes_step * args.steps * world / (total_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+                   "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
+                   "partition_size": calls.partition_size,
+                   "num_partitions": calls.num_partitions, "copy_on_write_pairs": cow_pairs,
+                   "l2": f"flushed between steps ({flush.numel() >> 20} MiB write, outside the "
+                         "timed events)",
+                   "parallelism": f"replicas x{world}"},
+        "attended_tokens_per_s": tokens_step * args.steps * world / (total_ms * 1e-3),
+        "us_per_step": 1e3 * total_ms / args.steps,
+        "us_per_decode_call": 1e3 * statistics.mean(decode_ms),
+        "decode_call_us_p10_p50_p90": [1e3 * float(np.percentile(decode_ms, p))
+                                       for p in (10, 50, 90)],
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "pa_decode (decode kernel + split-K merge kernel)",
+                     "peak_source": f"{peak_src} hbm_gbs"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": calls.launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3 and args.impl == "b200":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    rank, world, local_rank = dist_env()
+    wl = make_workload(args.workload, args.block_size)
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    run_b200(args, wl, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

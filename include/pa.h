@@ -1,0 +1,269 @@
+/*
+ * pa.h — C ABI of the paged KV-cache decode path (B200, sm_100a).
+ *
+ * The method: the KV cache of every sequence lives in fixed-size physical
+ * blocks from a shared pool; a per-sequence block table maps the sequence's
+ * logical blocks (token t is in logical block t / block_size at offset
+ * t % block_size) to physical block ids, and attention reads the cache
+ * through that table without first copying it into contiguous memory.
+ *   Sources: "Paged Attention" (klaylearn.com glossary), definition;
+ *   "PagedAttention — AI Glossary" (modelrefs.com), How it works 1-5;
+ *   "What is paged attention in vLLM, and why does it matter?"
+ *   (interview.clozo.ai), Steps 1-4 and "Trade-offs and edge cases".
+ *
+ * Conventions shared by every call below.
+ *   Memory. Every pointer is owned by the caller. "device" pointers are CUDA
+ *   global-memory addresses on the current device; "host" pointers are CPU
+ *   memory. The kernels allocate no device memory: scratch space for the
+ *   split-K pass is a caller-provided workspace sized by
+ *   pa_decode_workspace_bytes.
+ *   Streams. Kernel calls are asynchronous on `stream` (a cudaStream_t; NULL
+ *   is the legacy default stream) and never synchronise the host.
+ *   Cache layout. k_cache and v_cache are each
+ *   [num_blocks][block_size][num_kv_heads][head_dim], row-major, dense, in the
+ *   element type `dtype`. The flat slot of (physical block b, offset o) is
+ *   b * block_size + o, i.e. row `slot` of the cache viewed as
+ *   [num_blocks * block_size][num_kv_heads][head_dim].
+ *   Alignment. Cache, query, output, new-token and workspace pointers must be
+ *   16-byte aligned; index arrays naturally aligned.
+ *   Errors. Arguments are checked on the host before anything is launched;
+ *   a failed check returns PA_ERR_INVALID or PA_ERR_UNSUPPORTED and launches
+ *   nothing. A failed launch returns PA_ERR_CUDA. pa_last_error() gives a
+ *   one-line reason for the last failure on the calling thread. Indices that
+ *   live in device memory (slots, block ids, context lengths, copy pairs) are
+ *   checked inside the kernels: a bad one is skipped, never dereferenced, and
+ *   sets a bit of the device error word read by pa_device_errors().
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* pa_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,      /* bad argument; nothing launched, no state changed   */
+  PA_ERR_UNSUPPORTED = 2,  /* valid but not built: dtype, head_dim or group size */
+  PA_ERR_CUDA = 3,         /* a CUDA runtime call failed                          */
+  PA_ERR_NO_BLOCKS = 4,    /* the free pool cannot supply the blocks asked for    */
+  PA_ERR_DEVICE_CHECK = 5  /* a kernel found a bad device-side index              */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word (pa_device_errors). */
+#define PA_DEVERR_SLOT 0x1u       /* pa_kv_append: slot >= num_blocks * block_size       */
+#define PA_DEVERR_BLOCK_ID 0x2u   /* pa_decode: table entry outside [0, num_blocks)       */
+#define PA_DEVERR_CONTEXT 0x4u    /* pa_decode: context_lens[s] < 0, > max_context_len,
+                                     or > max_blocks_per_seq * block_size                 */
+#define PA_DEVERR_COPY_PAIR 0x8u  /* pa_copy_blocks: src or dst outside [0, num_blocks)  */
+#define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up               */
+
+/* ------------------------------------------------------------------ cache writes */
+
+/*
+ * pa_kv_append — write new tokens' K and V rows into their cache slots.
+ * "Paged Attention" (klaylearn.com glossary), definition: during prefill blocks
+ * are filled as prompt tokens produce K and V; during decode a new token is
+ * appended into the current tail block. "What is paged attention in vLLM...",
+ * Step 4: each decoding step writes the new token's keys and values into the
+ * last block.
+ *
+ *   k_new, v_new   device, [num_tokens][num_kv_heads][head_dim], dtype.
+ *   slot_mapping   device, int64 [num_tokens]: flat slot of each row; a
+ *                  negative slot skips the row (padding). Slots must be
+ *                  distinct; slot >= num_blocks * block_size sets
+ *                  PA_DEVERR_SLOT and skips the row.
+ *   k_cache, v_cache  device, written in place.
+ * Rows are copied bit for bit. num_tokens == 0 is a no-op. Prefill and decode
+ * use the same call (num_tokens = prompt tokens, or one per sequence).
+ * Requires num_kv_heads * head_dim * element size to be a multiple of 16.
+ */
+int pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                 int num_tokens, void* k_cache, void* v_cache, int num_blocks, int block_size,
+                 int num_kv_heads, int head_dim, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks — copy-on-write of shared blocks: for each pair,
+ * block dst := block src, in both caches, bit for bit.
+ * "PagedAttention — AI Glossary", How it works 5: when a shared sequence
+ * diverges only the block being written is copied; "What is paged attention in
+ * vLLM...", "Trade-offs and edge cases", third point.
+ *
+ *   block_mapping  device, int64 [num_pairs][2] = (src, dst). Sources and
+ *                  destinations must be disjoint sets (the copies of one call
+ *                  run concurrently). An id outside [0, num_blocks) sets
+ *                  PA_DEVERR_COPY_PAIR and the pair is skipped.
+ * num_pairs == 0 is a no-op.
+ */
+int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int num_pairs,
+                   int num_blocks, int block_size, int num_kv_heads, int head_dim,
+                   pa_dtype dtype, pa_stream_t stream);
+
+/* --------------------------------------------------------------- decode attention */
+
+/*
+ * pa_decode_partition_size — the partition length (tokens) pa_decode uses when
+ * passed partition_size = 0. Chosen from the grid size alone (sequences, KV
+ * heads, max_context_len), never from block_size or placement, so results do
+ * not depend on either. Always a multiple of 16.
+ */
+int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len);
+
+/*
+ * pa_decode_workspace_bytes — bytes of workspace pa_decode needs for these
+ * sizes (0 when no sequence can span more than one partition).
+ * partition_size = 0 means the automatic choice.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int partition_size);
+
+/*
+ * pa_decode — one decode query per sequence attends over its whole cached
+ * context, reading K and V through the block table.
+ * "Paged Attention" (klaylearn.com glossary), definition: the kernel computes
+ * each token's logical block and offset, looks up the physical block and loads
+ * the K/V from it. "PagedAttention — AI Glossary", Example: the attention
+ * mathematics is unchanged, so for sequence s and query head j (KV head
+ * h = j / (num_heads / num_kv_heads)):
+ *     x_t = scale * dot(q[s][j], K_s[t][h]),  t < context_lens[s]
+ *     out[s][j] = sum_t softmax(x)_t * V_s[t][h]
+ * with K_s[t] the cache row in block block_tables[s][t / block_size] at offset
+ * t % block_size. Accumulation is float32.
+ *
+ *   out            device, [num_seqs][num_heads][head_dim], dtype (bf16 output
+ *                  is rounded to nearest even from the float32 result).
+ *   q              device, [num_seqs][num_heads][head_dim], dtype.
+ *   k_cache, v_cache  device, read only.
+ *   block_tables   device, int32 [num_seqs][max_blocks_per_seq]; only the first
+ *                  ceil(context_lens[s] / block_size) entries of a row are read.
+ *   context_lens   device, int32 [num_seqs]: tokens to attend (after the
+ *                  step's append). 0 gives an all-zero output row.
+ *   max_context_len  host upper bound of context_lens (sizes the grid without a
+ *                  device read); <= max_blocks_per_seq * block_size.
+ *   partition_size tokens per split-K partition, a multiple of 16, or 0 for
+ *                  pa_decode_partition_size(). A sequence longer than one
+ *                  partition is split; partial results (max, sum, unnormalised
+ *                  output) go to the workspace and a second kernel combines
+ *                  them with a log-sum-exp rescale.
+ *   workspace      device scratch of at least pa_decode_workspace_bytes(...)
+ *                  bytes (may be NULL when that is 0). Contents on entry are
+ *                  ignored; calls sharing one workspace must not overlap.
+ * Supported: dtype PA_F32 or PA_BF16; head_dim 64 or 128; num_heads /
+ * num_kv_heads in {1, 2, 4, 8}; block_size a power of two in [1, 256].
+ * The result for a sequence depends only on its logical tokens and on
+ * partition_size: physical placement and block_size do not change a bit of it.
+ */
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
+              void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_device_errors — synchronise `stream`, return the device error word
+ * (PA_DEVERR_* bits set by kernels since the last call) in *flags and clear
+ * it. Returns PA_ERR_DEVICE_CHECK if any bit was set, PA_OK otherwise. The
+ * word is per device and shared by all streams.
+ */
+int pa_device_errors(pa_stream_t stream, unsigned int* flags);
+
+/* One-line reason for the last non-OK return on this thread ("" if none). */
+const char* pa_last_error(void);
+/* Static name of a pa_status value. */
+const char* pa_status_string(int status);
+
+/* ---------------------------------------------------------- host block allocator */
+/*
+ * The pool of physical blocks: a free list (LIFO stack of ids) and a
+ * reference count per block. "What is paged attention in vLLM...", Step 3:
+ * the block manager keeps the table beside a pool of free blocks and a
+ * reference count per block; Step 4: blocks return to the free pool when the
+ * request ends. Host memory only; not thread safe (one owner thread).
+ */
+typedef struct pa_alloc pa_alloc;
+
+/* New pool of num_blocks free blocks; the first allocations return 0, 1, 2, ...
+ * NULL if num_blocks <= 0 or on allocation failure. */
+pa_alloc* pa_alloc_create(int num_blocks);
+void pa_alloc_destroy(pa_alloc* a);
+/* Pop a free block into *out_id with count 1; PA_ERR_NO_BLOCKS if none. */
+int pa_alloc_block(pa_alloc* a, int32_t* out_id);
+/* Add a reference to an allocated block; PA_ERR_INVALID if out of range or free. */
+int pa_incref(pa_alloc* a, int32_t id);
+/* Drop a reference; at zero the block goes back on the free list.
+ * PA_ERR_INVALID if out of range or already free. */
+int pa_decref(pa_alloc* a, int32_t id);
+/* Reference count of a block, or -1 if id is out of range. */
+int pa_refcount(const pa_alloc* a, int32_t id);
+int pa_num_free(const pa_alloc* a);
+int pa_num_blocks(const pa_alloc* a);
+/* Make the next allocations return ids[0], ids[1], ... ; ids must list every
+ * free block exactly once (n == pa_num_free), else PA_ERR_INVALID. */
+int pa_alloc_set_free_order(pa_alloc* a, const int32_t* ids, int n);
+
+/* ---------------------------------------------------------- host block manager */
+/*
+ * Sequences over a pool: per-sequence block tables, allocation on demand,
+ * sharing by fork, copy-on-write. Host memory only; not thread safe.
+ *   "What is paged attention in vLLM...", Step 4: a new physical block is
+ *   allocated only when the last one is full.
+ *   "PagedAttention — AI Glossary", How it works 4-5: sequences sharing a
+ *   prefix point at the same reference-counted blocks; a shared block is
+ *   copied when one sharer writes into it.
+ */
+typedef struct pa_bm pa_bm;
+
+/* New manager owning a fresh pool (pa_alloc_create(num_blocks)). block_size > 0. */
+pa_bm* pa_bm_create(int num_blocks, int block_size);
+void pa_bm_destroy(pa_bm* bm);
+/* The manager's pool, for the pa_alloc_* calls (owned by the manager). */
+pa_alloc* pa_bm_allocator(pa_bm* bm);
+int pa_bm_block_size(const pa_bm* bm);
+/* New empty sequence; its id is written to *seq_id. */
+int pa_bm_add_seq(pa_bm* bm, int32_t* seq_id);
+/* New sequence sharing every block of `parent` (each count + 1) and its length. */
+int pa_bm_fork(pa_bm* bm, int32_t parent, int32_t* child);
+/* Drop the sequence's references (blocks at count 0 return to the free list);
+ * the id becomes invalid. */
+int pa_bm_free_seq(pa_bm* bm, int32_t seq_id);
+/* Tokens in the sequence, or -1 for an unknown id. */
+int pa_bm_seq_len(const pa_bm* bm, int32_t seq_id);
+/* Blocks in the sequence's table, or -1 for an unknown id. */
+int pa_bm_seq_num_blocks(const pa_bm* bm, int32_t seq_id);
+/*
+ * pa_bm_append_slots — reserve slots for counts[i] new tokens of sequence
+ * seq_ids[i], for i < n, in that order (ids distinct). Writes the flat slot
+ * of every new token to slot_mapping (host, int64, sum(counts) entries, in
+ * order). When a sequence's first new token falls in a shared, partly filled
+ * tail block, a fresh block replaces it in that sequence's table and the pair
+ * (old, fresh) is written to cow_pairs (host, int64 [cow_capacity][2]); the
+ * caller must run pa_copy_blocks on those pairs before writing the tokens.
+ * *num_cow receives the number of pairs. All or nothing: if the pool lacks
+ * the blocks, or cow_capacity is too small, returns PA_ERR_NO_BLOCKS /
+ * PA_ERR_INVALID and changes nothing.
+ */
+int pa_bm_append_slots(pa_bm* bm, const int32_t* seq_ids, const int32_t* counts, int n,
+                       int64_t* slot_mapping, int64_t* cow_pairs, int cow_capacity,
+                       int* num_cow);
+/*
+ * pa_bm_block_tables — write the block tables of seq_ids[0..n) as rows of
+ * `tables` (host, int32 [n][max_blocks_per_seq], unused entries set to 0)
+ * and their lengths to context_lens (host, int32 [n]; may be NULL).
+ * PA_ERR_INVALID if a sequence holds more than max_blocks_per_seq blocks.
+ */
+int pa_bm_block_tables(const pa_bm* bm, const int32_t* seq_ids, int n, int32_t* tables,
+                       int max_blocks_per_seq, int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,333 @@
+"""Paged KV cache decode path for B200 (sm_100a): Python binding of libpa.so.
+
+This module only marshals arguments: it turns torch tensors and numpy arrays
+into pointers and sizes and calls the C ABI declared in include/pa.h. Every
+step of the hot path runs in the library's CUDA kernels or its C++ block
+manager. There is no CPU fallback: importing this package fails if libpa.so
+has not been built (python -m paged_kv_cache_345_b200.build).
+
+Entry points (same names as the C ABI):
+  pa_kv_append     write new tokens' K/V rows into their slots
+  pa_copy_blocks   copy-on-write of shared blocks
+  pa_decode        paged decode attention (split-K over partitions)
+  BlockManager     host free list + reference counts + block tables
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+__all__ = [
+    "PagedAttentionError", "PA_OK", "PA_ERR_INVALID", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
+    "PA_ERR_NO_BLOCKS", "PA_ERR_DEVICE_CHECK", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID",
+    "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
+    "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
+    "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
+]
+
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
+    range(6)
+PA_F32, PA_BF16 = 0, 1
+PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = \
+    0x1, 0x2, 0x4, 0x8, 0x10
+
+lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+if not os.path.exists(lib_path):
+    raise ImportError(
+        f"{lib_path} is missing: build the CUDA library first "
+        "(python -m paged_kv_cache_345_b200.build). There is no CPU fallback.")
+_lib = ctypes.CDLL(lib_path)
+
+_vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, \
+    ctypes.c_size_t
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def _sig(name, restype, *argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = list(argtypes)
+    return fn
+
+
+_sig("pa_kv_append", _i32, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
+_sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
+_sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
+_sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
+_sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+     _i32, _f32, _i32, _vp, _sz, _i32, _vp)
+_sig("pa_device_errors", _i32, _vp, ctypes.POINTER(ctypes.c_uint))
+_sig("pa_last_error", ctypes.c_char_p)
+_sig("pa_status_string", ctypes.c_char_p, _i32)
+_sig("pa_alloc_create", _vp, _i32)
+_sig("pa_alloc_destroy", None, _vp)
+_sig("pa_alloc_block", _i32, _vp, _i32p)
+_sig("pa_incref", _i32, _vp, ctypes.c_int32)
+_sig("pa_decref", _i32, _vp, ctypes.c_int32)
+_sig("pa_refcount", _i32, _vp, ctypes.c_int32)
+_sig("pa_num_free", _i32, _vp)
+_sig("pa_num_blocks", _i32, _vp)
+_sig("pa_alloc_set_free_order", _i32, _vp, _i32p, _i32)
+_sig("pa_bm_create", _vp, _i32, _i32)
+_sig("pa_bm_destroy", None, _vp)
+_sig("pa_bm_allocator", _vp, _vp)
+_sig("pa_bm_block_size", _i32, _vp)
+_sig("pa_bm_add_seq", _i32, _vp, _i32p)
+_sig("pa_bm_fork", _i32, _vp, ctypes.c_int32, _i32p)
+_sig("pa_bm_free_seq", _i32, _vp, ctypes.c_int32)
+_sig("pa_bm_seq_len", _i32, _vp, ctypes.c_int32)
+_sig("pa_bm_seq_num_blocks", _i32, _vp, ctypes.c_int32)
+_sig("pa_bm_append_slots", _i32, _vp, _i32p, _i32p, _i32, _i64p, _i64p, _i32,
+     ctypes.POINTER(ctypes.c_int))
+_sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
+
+EXPORTED = (
+    "pa_kv_append", "pa_copy_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
+    "pa_decode", "pa_device_errors", "pa_last_error", "pa_status_string", "pa_alloc_create",
+    "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
+    "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
+    "pa_bm_allocator", "pa_bm_block_size", "pa_bm_add_seq", "pa_bm_fork", "pa_bm_free_seq",
+    "pa_bm_seq_len", "pa_bm_seq_num_blocks", "pa_bm_append_slots", "pa_bm_block_tables",
+)
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        name = _lib.pa_status_string(status).decode()
+        super().__init__(f"{name}: {message}")
+
+
+def _check(status: int) -> None:
+    if status != PA_OK:
+        raise PagedAttentionError(status, _lib.pa_last_error().decode())
+
+
+# ------------------------------------------------------------ tensor helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.float32:
+        return PA_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev_ptr(t, name, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------- kernels
+
+def pa_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """Write row i of k_new/v_new [N, Hkv, d] at flat slot slot_mapping[i] (int64) of the caches."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    if tuple(k_new.shape[1:]) != (hkv, d) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be [N, num_kv_heads, head_dim] matching the cache")
+    if v_cache.shape != k_cache.shape or slot_mapping.shape != (k_new.shape[0],):
+        raise ValueError("cache or slot_mapping shape mismatch")
+    dt = k_cache.dtype
+    _check(_lib.pa_kv_append(
+        _dev_ptr(k_new, "k_new", dt), _dev_ptr(v_new, "v_new", dt),
+        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", dt), nb, bs, hkv, d,
+        _dtype_code(k_cache), _stream(stream, k_cache.device)))
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
+    """block dst := block src for each row (src, dst) of block_mapping [n, 2] (int64, device)."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be [num_pairs, 2]")
+    _check(_lib.pa_copy_blocks(
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", k_cache.dtype),
+        _dev_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], nb, bs,
+        hkv, d, _dtype_code(k_cache), _stream(stream, k_cache.device)))
+
+
+def pa_decode_partition_size(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:
+    return int(_lib.pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len))
+
+
+def pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                              partition_size=0) -> int:
+    return int(_lib.pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                              max_context_len, partition_size))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+              scale: float, partition_size: int = 0, workspace=None, stream=None) -> None:
+    """Paged decode attention; see pa_decode in include/pa.h.
+
+    out, q: [S, Hq, d]; caches: [num_blocks, bs, Hkv, d]; block_tables: int32
+    [S, max_blocks_per_seq]; context_lens: int32 [S]; workspace: a uint8 CUDA
+    tensor of at least pa_decode_workspace_bytes(...) bytes, or None when that is 0.
+    """
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    s, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    dt = k_cache.dtype
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode(
+        _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
+        block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,
+        ws_bytes, _dtype_code(k_cache), _stream(stream, q.device)))
+
+
+def pa_device_errors(stream=None) -> int:
+    """Synchronise, read and clear the device error word; returns its PA_DEVERR_* bits."""
+    torch = _torch()
+    flags = ctypes.c_uint(0)
+    st = _lib.pa_device_errors(_stream(stream, torch.cuda.current_device()), ctypes.byref(flags))
+    if st not in (PA_OK, PA_ERR_DEVICE_CHECK):
+        _check(st)
+    return int(flags.value)
+
+
+# ------------------------------------------------------------- host allocator
+
+def _i32_array(x):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+    return a, a.ctypes.data_as(_i32p)
+
+
+class Allocator:
+    """Free list + reference counts of a block pool (pa_alloc_*).
+
+    Allocator(n) owns a new pool; BlockManager.allocator returns a view of the
+    manager's pool that keeps the manager alive.
+    """
+
+    def __init__(self, num_blocks: int = 0, _handle=None, _owner=None):
+        self._owner = _owner
+        if _handle is not None:
+            self._h = _handle
+            self._own = False
+        else:
+            self._h = _lib.pa_alloc_create(num_blocks)
+            if not self._h:
+                raise PagedAttentionError(PA_ERR_INVALID, _lib.pa_last_error().decode())
+            self._own = True
+
+    def __del__(self):
+        if getattr(self, "_own", False) and self._h:
+            _lib.pa_alloc_destroy(self._h)
+            self._h = None
+
+    def alloc(self) -> int:
+        out = ctypes.c_int32()
+        _check(_lib.pa_alloc_block(self._h, ctypes.byref(out)))
+        return out.value
+
+    def incref(self, block: int) -> None:
+        _check(_lib.pa_incref(self._h, block))
+
+    def decref(self, block: int) -> None:
+        _check(_lib.pa_decref(self._h, block))
+
+    def refcount(self, block: int) -> int:
+        return int(_lib.pa_refcount(self._h, block))
+
+    def num_free(self) -> int:
+        return int(_lib.pa_num_free(self._h))
+
+    def num_blocks(self) -> int:
+        return int(_lib.pa_num_blocks(self._h))
+
+    def set_free_order(self, ids) -> None:
+        a, p = _i32_array(ids)
+        _check(_lib.pa_alloc_set_free_order(self._h, p, a.size))
+
+
+class BlockManager:
+    """Sequences over a block pool (pa_bm_*): tables, on-demand blocks, fork, copy-on-write."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self._h = _lib.pa_bm_create(num_blocks, block_size)
+        if not self._h:
+            raise PagedAttentionError(PA_ERR_INVALID, _lib.pa_last_error().decode())
+        self.block_size = block_size
+
+    @property
+    def allocator(self) -> Allocator:
+        return Allocator(_handle=_lib.pa_bm_allocator(self._h), _owner=self)
+
+    def __del__(self):
+        if getattr(self, "_h", None):
+            _lib.pa_bm_destroy(self._h)
+            self._h = None
+
+    def add_seq(self) -> int:
+        out = ctypes.c_int32()
+        _check(_lib.pa_bm_add_seq(self._h, ctypes.byref(out)))
+        return out.value
+
+    def fork(self, parent: int) -> int:
+        out = ctypes.c_int32()
+        _check(_lib.pa_bm_fork(self._h, parent, ctypes.byref(out)))
+        return out.value
+
+    def free_seq(self, seq: int) -> None:
+        _check(_lib.pa_bm_free_seq(self._h, seq))
+
+    def seq_len(self, seq: int) -> int:
+        return int(_lib.pa_bm_seq_len(self._h, seq))
+
+    def seq_num_blocks(self, seq: int) -> int:
+        return int(_lib.pa_bm_seq_num_blocks(self._h, seq))
+
+    def append_slots(self, seq_ids, counts):
+        """Reserve slots; returns (slot_mapping int64 [sum(counts)], cow_pairs int64 [k, 2])."""
+        ids, pids = _i32_array(seq_ids)
+        cnt, pcnt = _i32_array(counts)
+        if ids.shape != cnt.shape:
+            raise ValueError("seq_ids and counts differ in length")
+        slots = np.empty(int(cnt.sum()), dtype=np.int64)
+        cows = np.empty((max(ids.size, 1), 2), dtype=np.int64)
+        ncow = ctypes.c_int(0)
+        _check(_lib.pa_bm_append_slots(self._h, pids, pcnt, ids.size,
+                                       slots.ctypes.data_as(_i64p), cows.ctypes.data_as(_i64p),
+                                       cows.shape[0], ctypes.byref(ncow)))
+        return slots, cows[:ncow.value].copy()
+
+    def block_tables(self, seq_ids, max_blocks_per_seq: int):
+        """(tables int32 [n, max_blocks_per_seq], context_lens int32 [n]) for the sequences."""
+        ids, pids = _i32_array(seq_ids)
+        tables = np.empty((ids.size, max_blocks_per_seq), dtype=np.int32)
+        lens = np.empty(ids.size, dtype=np.int32)
+        _check(_lib.pa_bm_block_tables(self._h, pids, ids.size, tables.ctypes.data_as(_i32p),
+                                       max_blocks_per_seq, lens.ctypes.data_as(_i32p)))
+        return tables, lens

@@ -1,0 +1,107 @@
+"""PagedKVCache: one layer's paged K/V cache driven through the C ABI.
+
+Holds the device caches [num_blocks, block_size, Hkv, d], the native block
+manager (free list, reference counts, tables) and a reusable decode
+workspace. Each method marshals arguments and calls libpa.so:
+
+  write(seq_ids, counts, k_rows, v_rows)  reserve slots (native), copy shared
+      tail blocks first when needed (pa_copy_blocks), then scatter the rows
+      (pa_kv_append). Serves both prefill (many tokens) and decode (one token).
+  decode(q, seq_ids)  block tables to the device, then pa_decode.
+  decode_step(q, k_new, v_new, seq_ids)  write one token per sequence, then decode.
+
+"Paged Attention" (klaylearn.com glossary), definition: prefill allocates and
+fills blocks, decode appends into the tail block or triggers an allocation,
+finished requests return their blocks to the free list.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_partition_size,
+               pa_decode_workspace_bytes, pa_kv_append)
+
+_TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
+                 dtype="bf16", device="cuda", max_blocks_per_seq: int | None = None,
+                 free_order=None, stream=None):
+        self.dtype = _TORCH_DTYPES.get(dtype, dtype)
+        self.device = torch.device(device)
+        self.block_size = block_size
+        self.num_blocks = num_blocks
+        self.num_kv_heads = num_kv_heads
+        self.head_dim = head_dim
+        self.max_blocks_per_seq = max_blocks_per_seq or num_blocks
+        shape = (num_blocks, block_size, num_kv_heads, head_dim)
+        self.k_cache = torch.zeros(shape, dtype=self.dtype, device=self.device)
+        self.v_cache = torch.zeros(shape, dtype=self.dtype, device=self.device)
+        self.bm = BlockManager(num_blocks, block_size)
+        if free_order is not None:
+            self.bm.allocator.set_free_order(free_order)
+        self.stream = stream
+        self._workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    # ------------------------------------------------------------ sequences
+    def add_sequence(self) -> int:
+        return self.bm.add_seq()
+
+    def fork(self, seq: int) -> int:
+        return self.bm.fork(seq)
+
+    def free(self, seq: int) -> None:
+        self.bm.free_seq(seq)
+
+    def context_len(self, seq: int) -> int:
+        return self.bm.seq_len(seq)
+
+    # --------------------------------------------------------------- writes
+    def _to_device(self, a: np.ndarray):
+        return torch.from_numpy(np.ascontiguousarray(a)).pin_memory().to(self.device,
+                                                                          non_blocking=True)
+
+    def write(self, seq_ids, counts, k_rows, v_rows):
+        """Append counts[i] tokens to seq_ids[i]; k_rows/v_rows are [sum(counts), Hkv, d]
+        device tensors in sequence order. Returns the host slot mapping."""
+        slots, cows = self.bm.append_slots(seq_ids, counts)
+        if len(cows):
+            pa_copy_blocks(self.k_cache, self.v_cache, self._to_device(cows), stream=self.stream)
+        if len(slots):
+            pa_kv_append(k_rows, v_rows, self._to_device(slots), self.k_cache, self.v_cache,
+                         stream=self.stream)
+        return slots
+
+    # --------------------------------------------------------------- decode
+    def tables(self, seq_ids, max_blocks_per_seq: int | None = None):
+        """(block_tables, context_lens) of the sequences, as device int32 tensors."""
+        mbps = max_blocks_per_seq or max(1, max(self.bm.seq_num_blocks(s) for s in seq_ids))
+        tables, lens = self.bm.block_tables(seq_ids, mbps)
+        return self._to_device(tables), self._to_device(lens), int(lens.max(initial=0))
+
+    def workspace(self, num_seqs, num_heads, max_context_len, partition_size=0):
+        need = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_dim,
+                                         max_context_len, partition_size)
+        if need > self._workspace.numel():
+            self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self._workspace if need > 0 else None
+
+    def decode(self, q, seq_ids, scale: float | None = None, partition_size: int = 0, out=None):
+        num_seqs, num_heads, _ = q.shape
+        block_tables, context_lens, max_len = self.tables(seq_ids)
+        if partition_size == 0:
+            partition_size = pa_decode_partition_size(num_seqs, self.num_kv_heads, max_len)
+        out = torch.empty_like(q) if out is None else out
+        scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+        pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, max_len, scale,
+                  partition_size, self.workspace(num_seqs, num_heads, max_len, partition_size),
+                  stream=self.stream)
+        return out
+
+    def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
+                    out=None):
+        self.write(seq_ids, [1] * len(seq_ids), k_new, v_new)
+        return self.decode(q, seq_ids, scale, partition_size, out)

@@ -1,0 +1,246 @@
+// C-ABI shim: argument checks on the host, then one launch per call.
+// Nothing here touches device memory except through the launchers.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int elem_bytes(pa_dtype dt) { return dt == PA_BF16 ? 2 : 4; }
+bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16; }
+
+int cuda_fail(const char* what, cudaError_t e) {
+  return pa_fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+void pa_set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+void pa_clear_error() { g_last_error.clear(); }
+
+int pa_fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+namespace pa {
+
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int num_partitions) {
+  WorkspaceLayout w{};
+  if (num_partitions <= 1) return w;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * num_partitions;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  w.m_off = 0;
+  w.l_off = up(rows * sizeof(float));
+  w.acc_off = w.l_off + up(rows * sizeof(float));
+  w.total = w.acc_off + up(rows * head_dim * sizeof(float));
+  return w;
+}
+
+}  // namespace pa
+
+extern "C" {
+
+const char* pa_last_error(void) { return g_last_error.c_str(); }
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID: return "PA_ERR_INVALID";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_NO_BLOCKS: return "PA_ERR_NO_BLOCKS";
+    case PA_ERR_DEVICE_CHECK: return "PA_ERR_DEVICE_CHECK";
+    default: return "PA_ERR_UNKNOWN";
+  }
+}
+
+int pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                 int num_tokens, void* k_cache, void* v_cache, int num_blocks, int block_size,
+                 int num_kv_heads, int head_dim, pa_dtype dtype, pa_stream_t stream) {
+  if (num_tokens < 0) return pa_fail(PA_ERR_INVALID, "pa_kv_append: num_tokens < 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append: null pointer");
+  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_kv_append: dtype %d", dtype);
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append: sizes must be positive");
+  const int64_t row_bytes = static_cast<int64_t>(num_kv_heads) * head_dim * elem_bytes(dtype);
+  if (row_bytes % 16 != 0 || row_bytes > (1 << 30))
+    return pa_fail(PA_ERR_UNSUPPORTED,
+                   "pa_kv_append: num_kv_heads*head_dim*elem (%lld B) not a multiple of 16",
+                   static_cast<long long>(row_bytes));
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(slot_mapping, 8))
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append: misaligned pointer");
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  cudaError_t e = pa::launch_kv_append(k_new, v_new, slot_mapping, num_tokens, k_cache, v_cache,
+                                       num_slots, static_cast<int>(row_bytes),
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_kv_append launch", e);
+}
+
+int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int num_pairs,
+                   int num_blocks, int block_size, int num_kv_heads, int head_dim,
+                   pa_dtype dtype, pa_stream_t stream) {
+  if (num_pairs < 0) return pa_fail(PA_ERR_INVALID, "pa_copy_blocks: num_pairs < 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping)
+    return pa_fail(PA_ERR_INVALID, "pa_copy_blocks: null pointer");
+  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: dtype %d", dtype);
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_copy_blocks: sizes must be positive");
+  if (num_pairs > 2147483647 / 2)
+    return pa_fail(PA_ERR_INVALID, "pa_copy_blocks: too many pairs");
+  const int64_t block_bytes =
+      static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes(dtype);
+  if (block_bytes % 16 != 0)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_copy_blocks: block bytes not a multiple of 16");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8))
+    return pa_fail(PA_ERR_INVALID, "pa_copy_blocks: misaligned pointer");
+  cudaError_t e = pa::launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, num_blocks,
+                                         block_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_copy_blocks launch", e);
+}
+
+int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
+  // Aim for about eight CTAs per SM (148 SMs) if every sequence were as long
+  // as the longest, and keep partitions between 64 and 512 tokens: long
+  // enough to amortise a CTA's start-up, short enough to bound the tail.
+  const double work = static_cast<double>(max_context_len) * (num_seqs > 0 ? num_seqs : 1) *
+                      (num_kv_heads > 0 ? num_kv_heads : 1);
+  double p = std::ceil(work / (148.0 * 8.0));
+  if (p < 64) p = 64;
+  if (p > 512) p = 512;
+  const int c = pa::kChunkTokens;
+  return (static_cast<int>(p) + c - 1) / c * c;
+}
+
+static int resolve_partitions(int max_context_len, int* partition_size) {
+  if (*partition_size == 0) *partition_size = pa_decode_partition_size(1, 1, 0);
+  return max_context_len <= 0 ? 1 : (max_context_len + *partition_size - 1) / *partition_size;
+}
+
+size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int partition_size) {
+  if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      partition_size < 0)
+    return 0;
+  int ps = partition_size == 0 ? pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len)
+                               : partition_size;
+  const int np = resolve_partitions(max_context_len, &ps);
+  return pa::workspace_layout(num_seqs, num_heads, head_dim, np).total;
+}
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
+              void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode: num_seqs < 0");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: null pointer");
+  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: dtype %d", dtype);
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: num_heads %d not a multiple of num_kv_heads %d",
+                   num_heads, num_kv_heads);
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d (built: 1, 2, 4, 8)", group);
+  if (head_dim != 64 && head_dim != 128)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: head_dim %d (built: 64, 128)", head_dim);
+  if (!pow2(block_size) || block_size > 256)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: block_size %d not a power of two <= 256",
+                   block_size);
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: num_blocks and max_blocks_per_seq must be > 0");
+  if (max_context_len < 0 ||
+      static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: max_context_len %d outside [0, %lld]",
+                   max_context_len,
+                   static_cast<long long>(max_blocks_per_seq) * block_size);
+  if (!std::isfinite(scale)) return pa_fail(PA_ERR_INVALID, "pa_decode: scale not finite");
+  if (partition_size < 0 || partition_size % pa::kChunkTokens != 0 ||
+      partition_size > pa::kMaxPartitionSize)
+    return pa_fail(PA_ERR_INVALID, "pa_decode: partition_size %d not a multiple of %d in [0, %d]",
+                   partition_size, pa::kChunkTokens, pa::kMaxPartitionSize);
+  if (num_seqs > 65535) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: num_seqs > 65535");
+  if (num_kv_heads > 65535) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: num_kv_heads > 65535");
+  if (static_cast<int64_t>(num_blocks) * block_size * num_kv_heads * head_dim *
+          elem_bytes(dtype) / 16 > (int64_t(1) << 36))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: cache larger than 1 TiB");
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) ||
+      (workspace && !aligned(workspace, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
+
+  pa::DecodeShape sh{};
+  sh.num_seqs = num_seqs;
+  sh.num_heads = num_heads;
+  sh.num_kv_heads = num_kv_heads;
+  sh.head_dim = head_dim;
+  sh.block_size = block_size;
+  sh.num_blocks = num_blocks;
+  sh.max_blocks_per_seq = max_blocks_per_seq;
+  sh.max_context_len = max_context_len;
+  sh.partition_size = partition_size == 0
+                          ? pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len)
+                          : partition_size;
+  sh.num_partitions = resolve_partitions(max_context_len, &sh.partition_size);
+  sh.scale = scale;
+  sh.dtype = dtype;
+  if (sh.num_partitions > pa::kMaxPartitions)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: %d partitions > %d", sh.num_partitions,
+                   pa::kMaxPartitions);
+  const size_t need = pa::workspace_layout(num_seqs, num_heads, head_dim, sh.num_partitions).total;
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return pa_fail(PA_ERR_INVALID, "pa_decode: workspace %zu B < %zu B needed",
+                   workspace ? workspace_bytes : size_t(0), need);
+  cudaError_t e = pa::launch_decode(sh, out, q, k_cache, v_cache, block_tables, context_lens,
+                                    workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: no kernel for this shape");
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode launch", e);
+}
+
+int pa_device_errors(pa_stream_t stream, unsigned int* flags) {
+  unsigned int* word = nullptr;
+  cudaError_t e = pa::device_error_word(&word);
+  if (e != cudaSuccess) return cuda_fail("pa_device_errors: symbol", e);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int host = 0;
+  if ((e = cudaMemcpyAsync(&host, word, sizeof(host), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail("pa_device_errors: read", e);
+  if ((e = cudaMemsetAsync(word, 0, sizeof(unsigned int), st)) != cudaSuccess)
+    return cuda_fail("pa_device_errors: clear", e);
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess)
+    return cuda_fail("pa_device_errors: sync", e);
+  if (flags) *flags = host;
+  if (host != 0)
+    return pa_fail(PA_ERR_DEVICE_CHECK, "device error word 0x%x", host);
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// Internal declarations shared by the C-ABI shim, the allocator and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime_api.h>
+
+#include "pa.h"
+
+// Thread-local "last error" text behind pa_last_error().
+void pa_set_error(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+void pa_clear_error();
+// Sets the last-error text and returns `status`.
+int pa_fail(int status, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+
+namespace pa {
+
+constexpr int kChunkTokens = 16;       // tokens per pipeline stage of the decode kernel
+constexpr int kMaxPartitions = 65535;        // grid-y limit
+constexpr int kMaxPartitionSize = 1 << 20;   // tokens; keeps partition * size in int range
+
+// Sizes of one pa_decode call after validation.
+struct DecodeShape {
+  int num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks;
+  int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
+  float scale;
+  pa_dtype dtype;
+};
+
+// Byte offsets of the split-K workspace regions.
+struct WorkspaceLayout {
+  size_t m_off, l_off, acc_off, total;
+};
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int num_partitions);
+
+// Launchers (pa_kernels.cu). Return cudaSuccess or the launch error.
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                             int num_tokens, void* k_cache, void* v_cache, int64_t num_slots,
+                             int row_bytes, cudaStream_t stream);
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                               int num_pairs, int num_blocks, int64_t block_bytes,
+                               cudaStream_t stream);
+// Returns cudaErrorNotSupported when no kernel is built for the shape.
+cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, void* workspace, cudaStream_t stream);
+// Device error word of the current device (address in device memory).
+cudaError_t device_error_word(unsigned int** ptr);
+
+}  // namespace pa

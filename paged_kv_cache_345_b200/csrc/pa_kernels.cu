@@ -1,0 +1,261 @@
+// Kernels and launchers: cache append, block copy, paged decode + split-K merge.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "pa_decode.cuh"
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// Device error word: kernels OR PA_DEVERR_* bits into it; pa_device_errors
+// reads and clears it.
+__device__ unsigned int g_error_word = 0;
+
+cudaError_t device_error_word(unsigned int** ptr) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<unsigned int*> cache[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < kMaxDevices) {
+    unsigned int* c = cache[dev].load(std::memory_order_acquire);
+    if (c) {
+      *ptr = c;
+      return cudaSuccess;
+    }
+  }
+  void* addr = nullptr;
+  e = cudaGetSymbolAddress(&addr, g_error_word);
+  if (e != cudaSuccess) return e;
+  *ptr = static_cast<unsigned int*>(addr);
+  if (dev < kMaxDevices) cache[dev].store(*ptr, std::memory_order_release);
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------------ append
+
+// One warp per token row (K and V rows of all KV heads of a token are
+// contiguous both in k_new and in the cache slot): 16-byte vector copies.
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                     const int64_t* __restrict__ slot_mapping, int num_tokens,
+                     uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, int64_t num_slots,
+                     int vec_per_row, unsigned* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t tok = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       tok < num_tokens; tok += warps) {
+    const int64_t slot = __ldg(slot_mapping + tok);
+    if (slot < 0) continue;  // padding row
+    if (slot >= num_slots) {
+      if (lane == 0) atomicOr(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const uint4* ks = k_new + tok * vec_per_row;
+    const uint4* vs = v_new + tok * vec_per_row;
+    uint4* kd = k_cache + slot * vec_per_row;
+    uint4* vd = v_cache + slot * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) {
+      const uint4 a = ldg_stream(ks + v);
+      const uint4 b = ldg_stream(vs + v);
+      kd[v] = a;
+      vd[v] = b;
+    }
+  }
+}
+
+cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                             int num_tokens, void* k_cache, void* v_cache, int64_t num_slots,
+                             int row_bytes, cudaStream_t stream) {
+  unsigned* err = nullptr;
+  cudaError_t e = device_error_word(&err);
+  if (e != cudaSuccess) return e;
+  const int threads = 256, warps_per_cta = threads / 32;
+  int64_t ctas = (static_cast<int64_t>(num_tokens) + warps_per_cta - 1) / warps_per_cta;
+  if (ctas > 148 * 16) ctas = 148 * 16;
+  kv_append_kernel<<<static_cast<int>(ctas), threads, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping,
+      num_tokens, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots,
+      row_bytes / 16, err);
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------------------- copy blocks
+
+// blockIdx.x = pair, blockIdx.y = slice of the block; 16-byte vector copies.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const int64_t* __restrict__ block_mapping, int num_blocks,
+                       int64_t vec_per_block, unsigned* err) {
+  const int64_t src = __ldg(block_mapping + 2 * blockIdx.x);
+  const int64_t dst = __ldg(block_mapping + 2 * blockIdx.x + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, PA_DEVERR_COPY_PAIR);
+    return;
+  }
+  const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; v < vec_per_block;
+       v += stride) {
+    const uint4 a = ldg_stream(k_cache + src * vec_per_block + v);
+    const uint4 b = ldg_stream(v_cache + src * vec_per_block + v);
+    k_cache[dst * vec_per_block + v] = a;
+    v_cache[dst * vec_per_block + v] = b;
+  }
+}
+
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                               int num_pairs, int num_blocks, int64_t block_bytes,
+                               cudaStream_t stream) {
+  unsigned* err = nullptr;
+  cudaError_t e = device_error_word(&err);
+  if (e != cudaSuccess) return e;
+  const int64_t vec = block_bytes / 16;
+  const int threads = 256;
+  int64_t slices = (vec + threads * 4 - 1) / (threads * 4);  // ~4 vectors per thread
+  if (slices < 1) slices = 1;
+  if (slices > 65535) slices = 65535;
+  dim3 grid(num_pairs, static_cast<unsigned>(slices));
+  copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_cache),
+                                                   static_cast<uint4*>(v_cache), block_mapping,
+                                                   num_blocks, vec, err);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ decode
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 4-D view of a cache [num_blocks][block_size][num_kv_heads][head_dim]; a box is
+// `box_rows` consecutive tokens of one block for one KV head (head_dim x 1 x rows x 1).
+cudaError_t encode_cache_map(CUtensorMap* map, const void* base, const DecodeShape& sh,
+                             int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const int eb = sh.dtype == PA_BF16 ? 2 : 4;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(sh.head_dim),
+                              static_cast<cuuint64_t>(sh.num_kv_heads),
+                              static_cast<cuuint64_t>(sh.block_size),
+                              static_cast<cuuint64_t>(sh.num_blocks)};
+  const cuuint64_t row = static_cast<cuuint64_t>(sh.head_dim) * eb;
+  const cuuint64_t strides[3] = {row, row * sh.num_kv_heads,
+                                 row * sh.num_kv_heads * static_cast<cuuint64_t>(sh.block_size)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(sh.head_dim), 1u,
+                             static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, sh.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   4, const_cast<void*>(base), dims, strides, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_decode_t(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
+                            const void* v_cache, cudaStream_t stream) {
+  using Cfg = DecodeConfig<T, D, G>;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<unsigned long long> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev % kMaxDevices);
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(pa_decode_kernel<T, D, G>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  CUtensorMap kmap, vmap;
+  const int box_rows = sh.block_size < Cfg::kC ? sh.block_size : Cfg::kC;
+  if ((e = encode_cache_map(&kmap, k_cache, sh, box_rows)) != cudaSuccess) return e;
+  if ((e = encode_cache_map(&vmap, v_cache, sh, box_rows)) != cudaSuccess) return e;
+  dim3 grid(sh.num_kv_heads, sh.num_partitions, sh.num_seqs);
+  pa_decode_kernel<T, D, G><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(kmap, vmap, p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (sh.num_partitions > 1) {
+    dim3 rgrid(sh.num_heads, sh.num_seqs);
+    pa_reduce_kernel<T, D><<<rgrid, D, 0, stream>>>(p);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+template <typename T, int D>
+cudaError_t dispatch_group(const DecodeShape& sh, const DecodeParams& p, const void* kc,
+                           const void* vc, cudaStream_t st) {
+  switch (sh.num_heads / sh.num_kv_heads) {
+    case 1: return launch_decode_t<T, D, 1>(sh, p, kc, vc, st);
+    case 2: return launch_decode_t<T, D, 2>(sh, p, kc, vc, st);
+    case 4: return launch_decode_t<T, D, 4>(sh, p, kc, vc, st);
+    case 8: return launch_decode_t<T, D, 8>(sh, p, kc, vc, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+template <typename T>
+cudaError_t dispatch_dim(const DecodeShape& sh, const DecodeParams& p, const void* kc,
+                         const void* vc, cudaStream_t st) {
+  switch (sh.head_dim) {
+    case 64: return dispatch_group<T, 64>(sh, p, kc, vc, st);
+    case 128: return dispatch_group<T, 128>(sh, p, kc, vc, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
+                          const void* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, void* workspace, cudaStream_t stream) {
+  DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  const WorkspaceLayout wl =
+      workspace_layout(sh.num_seqs, sh.num_heads, sh.head_dim, sh.num_partitions);
+  if (sh.num_partitions > 1) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.ws_m = reinterpret_cast<float*>(ws + wl.m_off);
+    p.ws_l = reinterpret_cast<float*>(ws + wl.l_off);
+    p.ws_acc = reinterpret_cast<float*>(ws + wl.acc_off);
+  }
+  cudaError_t e = device_error_word(&p.err);
+  if (e != cudaSuccess) return e;
+  p.num_heads = sh.num_heads;
+  p.num_kv_heads = sh.num_kv_heads;
+  p.block_size = sh.block_size;
+  int lg = 0;
+  while ((1 << lg) < sh.block_size) ++lg;
+  p.log2_block_size = lg;
+  p.num_blocks = sh.num_blocks;
+  p.max_blocks_per_seq = sh.max_blocks_per_seq;
+  p.max_context_len = sh.max_context_len;
+  p.partition_size = sh.partition_size;
+  p.num_partitions = sh.num_partitions;
+  p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
+  if (sh.dtype == PA_BF16) return dispatch_dim<__nv_bfloat16>(sh, p, k_cache, v_cache, stream);
+  return dispatch_dim<float>(sh, p, k_cache, v_cache, stream);
+}
+
+}  // namespace pa

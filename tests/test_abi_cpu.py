@@ -1,0 +1,203 @@
+"""C-ABI library on the CPU: it loads, exports every declared symbol, rejects bad
+arguments on the host before any launch, and its block manager matches the
+oracle's bit for bit. No GPU and no kernel launch."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_345_b200 as pa
+from oracle import blocks as oblk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_functions()
+    assert len(declared) >= 25
+    lib = ctypes.CDLL(pa.lib_path)
+    missing = [name for name in declared if not hasattr(lib, name)]
+    assert missing == []
+    assert sorted(pa.EXPORTED) == declared
+
+
+def test_library_is_built_for_sm100a():
+    # the fatbin records its target; nvcc's ELF note names the SM
+    data = open(pa.lib_path, "rb").read()
+    assert b"sm_100a" in data or b"compute_100a" in data
+
+
+def test_status_strings():
+    assert pa._lib.pa_status_string(pa.PA_ERR_NO_BLOCKS) == b"PA_ERR_NO_BLOCKS"
+    assert pa._lib.pa_status_string(99) == b"PA_ERR_UNKNOWN"
+
+
+# ------------------------------------------------------ host-side validation
+# Fake, never-dereferenced pointers: each call must fail validation before any
+# CUDA call is made.
+FAKE = ctypes.c_void_p(0x10000)
+
+
+def _decode(**over):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, S=2, Hq=32, Hkv=8, D=128, bs=16,
+             nb=64, mbps=8, maxlen=100, scale=0.1, P=0, ws=None, wsb=0, dt=pa.PA_BF16)
+    a.update(over)
+    st = pa._lib.pa_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["S"], a["Hq"],
+                           a["Hkv"], a["D"], a["bs"], a["nb"], a["mbps"], a["maxlen"], a["scale"],
+                           a["P"], a["ws"], a["wsb"], a["dt"], None)
+    return st, pa._lib.pa_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(Hq=30), pa.PA_ERR_INVALID),                  # heads not a multiple of kv heads
+    (dict(Hq=24, Hkv=8), pa.PA_ERR_UNSUPPORTED),       # group 3
+    (dict(Hq=128, Hkv=8), pa.PA_ERR_UNSUPPORTED),      # group 16
+    (dict(D=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(bs=12), pa.PA_ERR_INVALID),
+    (dict(bs=512), pa.PA_ERR_INVALID),
+    (dict(maxlen=8 * 16 + 1), pa.PA_ERR_INVALID),      # beyond the table's capacity
+    (dict(maxlen=-1), pa.PA_ERR_INVALID),
+    (dict(P=100), pa.PA_ERR_INVALID),                  # not a multiple of 16
+    (dict(scale=float("nan")), pa.PA_ERR_INVALID),
+    (dict(dt=7), pa.PA_ERR_UNSUPPORTED),
+    (dict(out=None), pa.PA_ERR_INVALID),
+    (dict(q=ctypes.c_void_p(0x10008)), pa.PA_ERR_INVALID),   # misaligned
+    (dict(maxlen=128, P=16), pa.PA_ERR_INVALID),       # needs a workspace, none given
+    (dict(nb=0), pa.PA_ERR_INVALID),
+])
+def test_decode_rejects_on_host(over, status):
+    st, msg = _decode(**over)
+    assert st == status, msg
+    assert msg
+
+
+def test_decode_zero_sequences_is_a_no_op():
+    assert _decode(S=0)[0] == pa.PA_OK
+
+
+def test_append_and_copy_reject_on_host():
+    lib = pa._lib
+    assert lib.pa_kv_append(FAKE, FAKE, FAKE, -1, FAKE, FAKE, 4, 4, 2, 64, 0, None) == \
+        pa.PA_ERR_INVALID
+    assert lib.pa_kv_append(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 4, 2, 64, 0, None) == pa.PA_OK
+    assert lib.pa_kv_append(FAKE, FAKE, FAKE, 3, FAKE, FAKE, 4, 4, 1, 2, 1, None) == \
+        pa.PA_ERR_UNSUPPORTED                                         # 4-byte rows
+    assert lib.pa_kv_append(None, FAKE, FAKE, 3, FAKE, FAKE, 4, 4, 2, 64, 0, None) == \
+        pa.PA_ERR_INVALID
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 4, 4, 2, 64, 0, None) == pa.PA_OK
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, -2, 4, 4, 2, 64, 0, None) == pa.PA_ERR_INVALID
+    assert lib.pa_copy_blocks(FAKE, FAKE, ctypes.c_void_p(0x10004), 2, 4, 4, 2, 64, 0, None) == \
+        pa.PA_ERR_INVALID
+
+
+def test_partition_size_and_workspace():
+    for s, h, n in [(8, 8, 4101), (256, 8, 4096), (1, 1, 7), (16, 8, 32768), (64, 8, 3054)]:
+        p = pa.pa_decode_partition_size(s, h, n)
+        assert p % 16 == 0 and 64 <= p <= 512
+    assert pa.pa_decode_partition_size(8, 8, 4101) == 224
+    # one partition: no workspace
+    assert pa.pa_decode_workspace_bytes(2, 4, 2, 64, 34, 64) == 0
+    # 3 partitions of 16 tokens: m, l and acc regions, each 256-byte aligned
+    rows = 2 * 4 * 3
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert pa.pa_decode_workspace_bytes(2, 4, 2, 64, 34, 16) == \
+        up(rows * 4) * 2 + up(rows * 64 * 4)
+
+
+# ----------------------------------------------- block manager vs the oracle
+
+def _snapshot_native(bm, seqs):
+    tables, lens = bm.block_tables(seqs, 4096)
+    return ([list(tables[i, :bm.seq_num_blocks(s)]) for i, s in enumerate(seqs)], list(lens),
+            bm.allocator.num_free())
+
+
+def _snapshot_oracle(ob, seqs):
+    return [list(ob.tables[s]) for s in seqs], [ob.lengths[s] for s in seqs], ob.num_free()
+
+
+def test_block_manager_matches_oracle_on_random_operations():
+    rng = np.random.default_rng(12)
+    nb, bs = 300, 4
+    order = rng.permutation(nb).astype(np.int32)
+    nat = pa.BlockManager(nb, bs)
+    nat.allocator.set_free_order(order)
+    ob = oblk.BlockManager(nb, bs)
+    ob.set_free_order(order.tolist())
+    live_n, live_o = [], []
+    for step in range(400):
+        op = rng.integers(0, 10)
+        if op <= 1 or not live_n:
+            live_n.append(nat.add_seq())
+            live_o.append(ob.new_sequence())
+        elif op == 2:
+            i = rng.integers(len(live_n))
+            live_n.append(nat.fork(live_n[i]))
+            live_o.append(ob.fork(live_o[i]))
+        elif op == 3 and len(live_n) > 1:
+            i = rng.integers(len(live_n))
+            nat.free_seq(live_n.pop(i))
+            ob.free_sequence(live_o.pop(i))
+        else:
+            k = int(rng.integers(1, min(len(live_n), 6) + 1))
+            idx = rng.choice(len(live_n), size=k, replace=False)
+            counts = rng.integers(0, 9, size=k)
+            need = sum(ob.blocks_needed(live_o[i], int(c)) for i, c in zip(idx, counts))
+            if need > ob.num_free():
+                with pytest.raises(pa.PagedAttentionError) as ei:
+                    nat.append_slots([live_n[i] for i in idx], counts)
+                assert ei.value.status == pa.PA_ERR_NO_BLOCKS
+                continue
+            slots_n, cows_n = nat.append_slots([live_n[i] for i in idx], counts)
+            slots_o, cows_o = [], []
+            for i, c in zip(idx, counts):
+                sl, cw = ob.add_tokens(live_o[i], int(c))
+                slots_o += sl
+                cows_o += cw
+            assert slots_n.tolist() == slots_o
+            assert [tuple(x) for x in cows_n.tolist()] == cows_o
+        assert _snapshot_native(nat, live_n) == _snapshot_oracle(ob, live_o)
+        for b in range(0, nb, 7):
+            assert nat.allocator.refcount(b) == ob.refcount[b]
+
+
+def test_block_manager_worked_example_and_exhaustion(golden):
+    ex = golden["worked_example"]
+    bm = pa.BlockManager(700, ex["block_size"])
+    seqs = [bm.add_seq() for _ in ex["lengths"]]
+    slots, cows = bm.append_slots(seqs, ex["lengths"])
+    assert len(slots) == ex["total_tokens"] and len(cows) == 0
+    assert sum(bm.seq_num_blocks(s) for s in seqs) * ex["block_size"] == ex["paged_slots"]
+    _, _ = bm.append_slots(seqs, [1] * len(seqs))
+    assert sum(bm.seq_num_blocks(s) for s in seqs) == 666
+    free_before = bm.allocator.num_free()
+    with pytest.raises(pa.PagedAttentionError) as ei:
+        bm.append_slots(seqs[:1], [100_000])
+    assert ei.value.status == pa.PA_ERR_NO_BLOCKS
+    assert bm.allocator.num_free() == free_before and bm.seq_len(seqs[0]) == 129
+
+
+def test_allocator_rejects_bad_ids():
+    a = pa.Allocator(4)
+    b = a.alloc()
+    a.decref(b)
+    for bad in (lambda: a.decref(b), lambda: a.incref(b), lambda: a.decref(99),
+                lambda: a.set_free_order([0, 1, 2])):
+        with pytest.raises(pa.PagedAttentionError) as ei:
+            bad()
+        assert ei.value.status == pa.PA_ERR_INVALID
+    assert a.refcount(99) == -1
+    for _ in range(4):
+        a.alloc()
+    with pytest.raises(pa.PagedAttentionError) as ei:
+        a.alloc()
+    assert ei.value.status == pa.PA_ERR_NO_BLOCKS
