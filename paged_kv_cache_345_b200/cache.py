@@ -44,7 +44,7 @@ class PagedKVCache:
         if free_order is not None:
             self.bm.allocator.set_free_order(free_order)
         self.stream = stream
-        self._workspace = torch.empty(0, dtype=torch.uint8, device=self.device)
+        self._workspace = torch.zeros(0, dtype=torch.uint8, device=self.device)
 
     # ------------------------------------------------------------ sequences
     def add_sequence(self) -> int:

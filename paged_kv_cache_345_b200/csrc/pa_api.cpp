@@ -46,13 +46,15 @@ int pa_fail(int status, const char* fmt, ...) {
 
 namespace pa {
 
-WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int num_partitions) {
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int num_partitions) {
   WorkspaceLayout w{};
   if (num_partitions <= 1) return w;
   const size_t rows = static_cast<size_t>(num_seqs) * num_heads * num_partitions;
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  (void)num_kv_heads;
   w.m_off = 0;
-  w.l_off = up(rows * sizeof(float));
+  w.l_off = w.m_off + up(rows * sizeof(float));
   w.acc_off = w.l_off + up(rows * sizeof(float));
   w.total = w.acc_off + up(rows * head_dim * sizeof(float));
   return w;
@@ -125,12 +127,15 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, i
 }
 
 int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
-  // Aim for about eight CTAs per SM (148 SMs) if every sequence were as long
-  // as the longest, and keep partitions between 64 and 512 tokens: long
+  // The bf16 kernel runs one CTA per (group of up to 4 KV heads, partition,
+  // sequence), two per SM. Aim for about three CTAs per SM if every sequence
+  // were as long as the longest, with partitions of 64..512 tokens: long
   // enough to amortise a CTA's start-up, short enough to bound the tail.
+  const int groups = num_kv_heads % 4 == 0 ? num_kv_heads / 4
+                     : num_kv_heads % 2 == 0 ? num_kv_heads / 2 : num_kv_heads;
   const double work = static_cast<double>(max_context_len) * (num_seqs > 0 ? num_seqs : 1) *
-                      (num_kv_heads > 0 ? num_kv_heads : 1);
-  double p = std::ceil(work / (148.0 * 8.0));
+                      (groups > 0 ? groups : 1);
+  double p = std::ceil(work / (148.0 * 3.0));
   if (p < 64) p = 64;
   if (p > 512) p = 512;
   const int c = pa::kChunkTokens;
@@ -150,7 +155,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
   int ps = partition_size == 0 ? pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len)
                                : partition_size;
   const int np = resolve_partitions(max_context_len, &ps);
-  return pa::workspace_layout(num_seqs, num_heads, head_dim, np).total;
+  return pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, np).total;
 }
 
 int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -214,7 +219,8 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   if (sh.num_partitions > pa::kMaxPartitions)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: %d partitions > %d", sh.num_partitions,
                    pa::kMaxPartitions);
-  const size_t need = pa::workspace_layout(num_seqs, num_heads, head_dim, sh.num_partitions).total;
+  const size_t need =
+      pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, sh.num_partitions).total;
   if (need > 0 && (!workspace || workspace_bytes < need))
     return pa_fail(PA_ERR_INVALID, "pa_decode: workspace %zu B < %zu B needed",
                    workspace ? workspace_bytes : size_t(0), need);

@@ -364,30 +364,67 @@ __global__ void __launch_bounds__(DecodeConfig<T, D, G>::kThreads)
   }
 }
 
-// Split-K merge: for each (sequence, query head) with more than one partition,
+
+// Split-K merge: one CTA of 4 warps per (sequence, query head) row with more
+// than one partition:
 //   M = max_p m_p,  Lambda = sum_p l_p 2^(m_p - M),  out = sum_p 2^(m_p - M) acc_p / Lambda.
-// Partitions are summed in index order, so the result does not depend on
-// scheduling. One CTA of D threads per (query head, sequence).
+// Warp w takes partitions w, w + 4, ...; each lane owns D / 32 columns, so a
+// warp's partition rows are independent loads, all in flight together. The
+// four warps' sums are added in warp order through shared memory, so the
+// result depends only on the partials (deterministic). Launched with
+// programmatic dependent launch: it waits for the decode kernel before reading.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) pa_reduce_kernel(const DecodeParams p) {
-  const int j = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
-  int L = __ldg(p.context_lens + s);
+__global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
+  constexpr int E = D / 32;
+  __shared__ float s_max[4], s_l[4], s_acc[4][D];
+  pdl_wait();
+  const int64_t r = blockIdx.x;  // row = s * num_heads + j
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = static_cast<int>(r / p.num_heads);
+  const int L = __ldg(p.context_lens + s);
   if (L < 0 || L > p.max_context_len ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size)
     return;  // flagged and zero-filled by the decode kernel
   const int np = (L + p.partition_size - 1) / p.partition_size;
-  if (np <= 1) return;
-  const int64_t row = (static_cast<int64_t>(s) * p.num_heads + j) * p.num_partitions;
+  if (np <= 1) return;  // written directly by the decode kernel
+  const int64_t row = r * p.num_partitions;
   float M = -INFINITY;
-  for (int q = 0; q < np; ++q) M = fmaxf(M, p.ws_m[row + q]);
-  float A = 0.0f, Lsum = 0.0f;
-  for (int q = 0; q < np; ++q) {
-    const float f = exp2f(p.ws_m[row + q] - M);
-    Lsum = fmaf(f, p.ws_l[row + q], Lsum);
-    A = fmaf(f, p.ws_acc[(row + q) * D + d], A);
+  for (int q = threadIdx.x; q < np; q += 128) M = fmaxf(M, __ldcg(p.ws_m + row + q));
+#pragma unroll
+  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+  if (lane == 0) s_max[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
+  float acc[E], lw = 0.0f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+  const float* a = p.ws_acc + row * D + lane * E;
+#pragma unroll 4
+  for (int q = warp; q < np; q += 4) {
+    const float w = exp2f(__ldcg(p.ws_m + row + q) - M);
+    lw = fmaf(w, __ldcg(p.ws_l + row + q), lw);
+    if constexpr (E == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a + static_cast<int64_t>(q) * D));
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+    } else {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(a + static_cast<int64_t>(q) * D));
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+    }
   }
-  T* out = static_cast<T*>(p.out);
-  ElemTraits<T>::store(out + (static_cast<int64_t>(s) * p.num_heads + j) * D + d, A / Lsum);
+#pragma unroll
+  for (int e = 0; e < E; ++e) s_acc[warp][lane * E + e] = acc[e];
+  if (lane == 0) s_l[warp] = lw;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int d = threadIdx.x;
+    const float lsum = ((s_l[0] + s_l[1]) + s_l[2]) + s_l[3];
+    const float v = ((s_acc[0][d] + s_acc[1][d]) + s_acc[2][d]) + s_acc[3][d];
+    ElemTraits<T>::store(static_cast<T*>(p.out) + r * D + d, v / lsum);
+  }
 }
 
 }  // namespace pa

@@ -1,0 +1,343 @@
+// Paged decode attention, bfloat16 cache, tensor-core inner products (sm_100a).
+//
+// Computes the same thing as pa_decode_kernel ("Paged Attention", klaylearn.com
+// glossary, definition; "PagedAttention — AI Glossary", Example: the block
+// table changes where K/V are read from, not the attention arithmetic).
+//
+// Why tensor cores in an HBM-bound kernel: on CUDA cores every token row costs
+// 2 * G * head_dim fp32 FMAs plus cross-lane reductions, ~90 warp instructions
+// per (token, KV head), about the whole issue budget an SM has per (token, KV
+// head) at its share of HBM bandwidth. The G query heads of a GQA group
+// against 16 K rows are a small dense contraction (G x head_dim x 16): one
+// m16n8k16 MMA covers 8 x 16 x 8 of it with the group's heads as the M rows
+// (zero-padded), which leaves ~8 warp instructions per (token, KV head).
+//
+// Why whole-block TMA boxes: measured on B200, TMA boxes of one KV head's
+// 256-byte rows (16 rows per box) reach ~3 TB/s with one CTA per SM and need
+// four CTAs per SM to approach the HBM roofline; one box covering a group of
+// KV heads of a block (kilobytes contiguous per token) reaches ~7 TB/s with one.
+//
+// Layout and pipeline:
+//  * CTA = (group of HB KV heads, partition, sequence): HB consumer warps (one
+//    per KV head) + 1 producer warp.
+//  * The producer reads the block table 32 entries at a time (one coalesced
+//    load, shuffled out) and, per chunk of 16 tokens, issues one TMA box per
+//    block for K and one for V: {head_dim + 8 columns, min(block_size, 16)
+//    tokens, HB heads}. The 8 columns past head_dim lie outside the tensor and
+//    arrive as zeros, so every row lands at a padded stride of head_dim * 2 +
+//    16 bytes and ldmatrix reads of 8 consecutive rows hit 8 bank groups.
+//    The tensor map orders the dimensions (column, token, head, block), so a
+//    box lands as [head][token][row].
+//  * Stages form a ring of NS; a stage is released once all HB warps read it.
+//  * Consumer warp per chunk: S = Q K^T with m16n8k16 (A = Q rows of the
+//    group, B = K rows via ldmatrix), online softmax in base 2 on the
+//    accumulator fragments (row max / sum over the 4-lane quad), P converted to
+//    bfloat16 in registers becomes the A operand of O += P V (B = V rows via
+//    ldmatrix.trans). m, l and O stay in registers.
+//  * End: a single-partition sequence writes `out`; otherwise (m, l, O) go to
+//    the split-K workspace and pa_merge_kernel (launched right behind, with
+//    programmatic dependent launch) combines the partitions.
+//  * Chunks hold the same 16 logical tokens and are reduced in the same order
+//    whatever the block size or placement, so results are bit-identical across
+//    both.
+#pragma once
+
+#include <cmath>
+#include <cstdint>
+
+#include "pa_decode.cuh"
+#include "pa_device.cuh"
+
+namespace pa {
+
+template <int D, int G, int HB, int NS>
+struct GroupConfig {
+  static constexpr int kC = 16;                       // tokens per chunk / stage
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRS = kRowBytes + 16;          // padded row stride in shared memory
+  // One chunk of K (or V) for the group: up to 16 boxes (block_size 1) of HB
+  // rows each, every box padded to a 128-byte boundary; fewer, larger boxes
+  // (block_size 2..16+) always fit in the same space.
+  static constexpr int kTensorBytes = kC * ((HB * kRS + 127) & ~127);
+  static constexpr int kStageBytes = 2 * kTensorBytes;
+  static constexpr int kThreads = (HB + 1) * 32;
+  static constexpr int kRingBytes = NS * kStageBytes;
+  static constexpr int kBarBytes = 2 * NS * 8;
+  static constexpr int kSmemBytes = 128 + kRingBytes + kBarBytes;
+  static_assert(G >= 1 && G <= 8, "group must fit the 8 real rows of an m16 tile");
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+};
+
+// Bytes between consecutive TMA boxes of one chunk (rows_per_box tokens of HB
+// heads each), rounded up so every box starts 128-byte aligned.
+__host__ __device__ constexpr int box_stride_bytes(int hb, int rows_per_box, int rs) {
+  return (hb * rows_per_box * rs + 127) & ~127;
+}
+
+template <int D, int G, int HB, int NS>
+__global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
+    pa_decode_mma_kernel(const __grid_constant__ CUtensorMap k_map,
+                         const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
+  using Cfg = GroupConfig<D, G, HB, NS>;
+  constexpr int C = Cfg::kC, RS = Cfg::kRS, TB = Cfg::kTensorBytes;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                             ~uintptr_t(127));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);  // full[NS], empty[NS]
+
+  const int hg = blockIdx.x, part = blockIdx.y, s = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int P = p.partition_size, bs = p.block_size, lg = p.log2_block_size;
+  const int rows_per_box = bs < C ? bs : C;
+  const int box_stride = box_stride_bytes(HB, rows_per_box, RS);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(smem_u32(bars + i), 1);        // full: producer arrive + TMA bytes
+      mbar_init(smem_u32(bars + NS + i), HB);  // empty: every consumer warp releases
+    }
+    fence_barrier_init();
+  }
+  pdl_wait();  // inputs may come from the previous kernel in the stream
+  pdl_launch_dependents();
+
+  // Independent loads first so their latencies overlap: the context length,
+  // the first 32 block-table entries of this partition (producer warp) and the
+  // query fragments (consumer warps).
+  int L = __ldg(p.context_lens + s);
+  const int t0 = part * P;
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
+  int base = t0 >> lg, ent = 0;
+  if (warp == HB && base + lane < p.max_blocks_per_seq) ent = __ldg(trow + base + lane);
+  const int kvh = hg * HB + (warp < HB ? warp : 0);  // this consumer warp's KV head
+  const int qr = lane >> 2;  // fragment row: query head of the group (rows >= G are padding)
+  const int qc = lane & 3;   // fragment column pair
+  const bool real_row = qr < G;
+  const int64_t out_row = static_cast<int64_t>(s) * p.num_heads + kvh * G;
+  uint32_t qa[D / 16][2];  // Q as the A operand: rows = heads of the group, bf16 pairs
+  if (warp < HB) {
+    const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+        static_cast<const __nv_bfloat16*>(p.q) + (out_row + (real_row ? qr : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qa[ks][0] = real_row ? __ldg(qp + ks * 8 + qc) : 0u;
+      qa[ks][1] = real_row ? __ldg(qp + ks * 8 + 4 + qc) : 0u;
+    }
+  }
+
+  if (L < 0 || L > p.max_context_len ||
+      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
+    if (threadIdx.x == 0 && hg == 0 && part == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+    L = 0;
+  }
+  const int n_part_s = (L + P - 1) / P;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+
+  if (L == 0) {  // empty context: zeros for every query head of the group
+    if (part == 0) {
+      const int64_t first = static_cast<int64_t>(s) * p.num_heads + hg * HB * G;
+      for (int e = threadIdx.x; e < HB * G * D; e += blockDim.x)
+        out[first * D + e] = __float2bfloat16_rn(0.0f);
+    }
+    return;
+  }
+  if (t0 >= L) return;
+  const int t1 = min(t0 + P, L);
+  const int nchunks = (t1 - t0 + C - 1) / C;
+  __syncthreads();
+
+  if (warp == HB) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tensormap(&k_map);
+      prefetch_tensormap(&v_map);
+    }
+    const int lb_last = (t1 - 1) >> lg;
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % NS, u = c / NS;
+      if (u >= 1) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(bars + NS + st), (u - 1) & 1, p.err);
+        if (!__shfl_sync(kFullMask, ok, 0)) break;
+      }
+      const int t = t0 + c * C;
+      const int nvalid = min(C, t1 - t);
+      const int lb_lo = t >> lg, lb_hi = (t + nvalid - 1) >> lg;
+      if (lb_hi - base >= 32) {  // refill: the next 32 table entries, one per lane
+        base = lb_lo;
+        ent = (base + lane <= lb_last) ? __ldg(trow + base + lane) : 0;
+      }
+      const int nbox = lb_hi - lb_lo + 1;  // blocks holding valid tokens of this chunk
+      const int blk = __shfl_sync(kFullMask, ent, min(lane, nbox - 1) + lb_lo - base);
+      const uint32_t full_bar = smem_u32(bars + st);
+      const uint32_t kdst = smem_u32(smem + st * Cfg::kStageBytes);
+      if (lane == 0) mbar_arrive_expect_tx(full_bar, 2u * nbox * HB * rows_per_box * RS);
+      __syncwarp();
+      if (lane < nbox) {
+        // an id outside the pool is flagged; TMA reads an out-of-range box as zeros
+        if (static_cast<unsigned>(blk) >= static_cast<unsigned>(p.num_blocks))
+          atomicOr(p.err, PA_DEVERR_BLOCK_ID);
+        const int off = bs < C ? 0 : (t & (bs - 1));
+        const uint32_t d = kdst + lane * box_stride;
+        tma_load_4d(d, &k_map, 0, off, hg * HB, blk, full_bar);
+        tma_load_4d(d + TB, &v_map, 0, off, hg * HB, blk, full_bar);
+      }
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  // Operands are swapped so the 16 rows of each MMA are tokens or head_dim
+  // rows, and the GQA group is the 8-wide N side:
+  //   S^T[token][head] = K[token][:] . Q^T[:][head]         (A = K rows, B = Q^T)
+  //   O^T[d][head]    += V^T[d][token] . P^T[token][head]   (A = V^T, B = P^T)
+  // Fragment coordinates: g = lane / 4 (row), t = lane % 4 (column pair).
+  const int g = lane >> 2, t = lane & 3;
+  const float qscale = p.q_scale;
+  float o[D / 16][4];  // O^T fragments: (d = 16i + g (+8), head 2t (+1))
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+  float m[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.0f, 0.0f};  // heads 2t, 2t+1
+
+  // byte offset of (token r of the chunk, 16-byte column c) of this warp's head
+  const int head_off = warp * rows_per_box * RS;
+  const int lgb = lg < 4 ? lg : 4;  // log2(rows_per_box)
+  auto at = [&](int r, int c) -> uint32_t {
+    const int b = r >> lgb;
+    return b * box_stride + head_off + (r - (b << lgb)) * RS + c * 16;
+  };
+  const int lrow = lane & 7, lmat = lane >> 3;  // ldmatrix: row within matrix, matrix index
+  // K as A (non-transposed): matrix j = tokens (j & 1) * 8 .. +7, column chunk + (j >> 1)
+  const uint32_t k_lane = at((lmat & 1) * 8 + lrow, lmat >> 1);
+  // V^T as A (transposed load): matrix j = tokens (j >> 1) * 8 .. +7, column chunk + (j & 1)
+  const uint32_t v_lane = at((lmat >> 1) * 8 + lrow, lmat & 1);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c % NS, u = c / NS;
+    if (!mbar_wait(smem_u32(bars + st), u & 1, p.err)) {
+      mbar_wait(smem_u32(bars + st), u & 1, p.err);  // let an in-flight copy land
+      break;
+    }
+    uint8_t* stage = smem + st * Cfg::kStageBytes;
+    const uint32_t ks_u32 = smem_u32(stage), vs_u32 = ks_u32 + TB;
+    const int nvalid = min(C, t1 - (t0 + c * C));
+    if (nvalid < C) {
+      // rows past the context hold stale bits: zero this head's V rows so 0 * stale = 0
+      for (int i = lane; i < (C - nvalid) * (D / 8); i += 32) {
+        const int r = nvalid + i / (D / 8), cc = i % (D / 8);
+        *reinterpret_cast<uint4*>(stage + TB + at(r, cc)) = make_uint4(0, 0, 0, 0);
+      }
+      // order these generic-proxy writes before the next async copy into the stage
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+    }
+
+    // S^T: two accumulation chains (even / odd k-steps) for latency
+    float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a[4];
+      ldmatrix_x4(a, ks_u32 + k_lane + ks * 32);
+      mma_bf16_16816(ks & 1 ? s1 : s0, a, qa[ks][0], qa[ks][1]);
+    }
+    // x[0], x[1]: token g, heads 2t, 2t+1; x[2], x[3]: token g + 8
+    float x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = g + (i >> 1) * 8;
+      x[i] = tok < nvalid ? (s0[i] + s1[i]) * qscale : -INFINITY;
+    }
+    // per-head (column) max over the 16 tokens: over the lane's 2 rows, then over g
+    float cm0 = fmaxf(x[0], x[2]), cm1 = fmaxf(x[1], x[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      cm0 = fmaxf(cm0, __shfl_xor_sync(kFullMask, cm0, off));
+      cm1 = fmaxf(cm1, __shfl_xor_sync(kFullMask, cm1, off));
+    }
+    const float mn0 = fmaxf(m[0], cm0), mn1 = fmaxf(m[1], cm1);
+    const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    const float p0 = exp2f(x[0] - mn0), p1 = exp2f(x[1] - mn1);
+    const float p2 = exp2f(x[2] - mn0), p3 = exp2f(x[3] - mn1);
+    l_part[0] = fmaf(l_part[0], al0, p0 + p2);
+    l_part[1] = fmaf(l_part[1], al1, p1 + p3);
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      o[i][0] *= al0;
+      o[i][1] *= al1;
+      o[i][2] *= al0;
+      o[i][3] *= al1;
+    }
+    // P^T as B: (token 2t, 2t+1 (+8), head g) = transpose of the (token g, head 2t..) pairs
+    const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, vs_u32 + v_lane + dt * 32);
+      mma_bf16_16816(o[dt], a, b0, b1);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(bars + NS + st));
+  }
+
+  // softmax denominators per head: sum over the 8 row groups
+  float l0 = l_part[0], l1 = l_part[1];
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(kFullMask, l0, off);
+    l1 += __shfl_xor_sync(kFullMask, l1, off);
+  }
+  const bool h0_real = 2 * t < G, h1_real = 2 * t + 1 < G;
+
+  if (n_part_s == 1) {
+    const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
+    __nv_bfloat16* o0 = out + (out_row + 2 * t) * D + g;
+    __nv_bfloat16* o1 = o0 + D;
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      if (h0_real) {
+        o0[dt * 16] = __float2bfloat16_rn(o[dt][0] * i0);
+        o0[dt * 16 + 8] = __float2bfloat16_rn(o[dt][2] * i0);
+      }
+      if (h1_real) {
+        o1[dt * 16] = __float2bfloat16_rn(o[dt][1] * i1);
+        o1[dt * 16 + 8] = __float2bfloat16_rn(o[dt][3] * i1);
+      }
+    }
+    return;
+  }
+
+  // split-K: this partition's (m, l, O) to the workspace
+  {
+    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + part;
+    const int64_t w1 = w0 + p.num_partitions;
+    float* a0 = p.ws_acc + w0 * D + g;
+    float* a1 = p.ws_acc + w1 * D + g;
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      if (h0_real) {
+        a0[dt * 16] = o[dt][0];
+        a0[dt * 16 + 8] = o[dt][2];
+      }
+      if (h1_real) {
+        a1[dt * 16] = o[dt][1];
+        a1[dt * 16 + 8] = o[dt][3];
+      }
+    }
+    if (g == 0) {
+      if (h0_real) {
+        p.ws_m[w0] = m[0];
+        p.ws_l[w0] = l0;
+      }
+      if (h1_real) {
+        p.ws_m[w1] = m[1];
+        p.ws_l[w1] = l1;
+      }
+    }
+  }
+}
+
+}  // namespace pa

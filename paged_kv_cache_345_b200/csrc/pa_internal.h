@@ -32,7 +32,8 @@ struct DecodeShape {
 struct WorkspaceLayout {
   size_t m_off, l_off, acc_off, total;
 };
-WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int num_partitions);
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int num_partitions);
 
 // Launchers (pa_kernels.cu). Return cudaSuccess or the launch error.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,

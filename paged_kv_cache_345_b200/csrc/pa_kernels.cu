@@ -5,8 +5,10 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "pa_decode.cuh"
+#include "pa_decode_mma.cuh"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -37,6 +39,25 @@ cudaError_t device_error_word(unsigned int** ptr) {
   return cudaSuccess;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream drains; it calls pdl_wait() before reading
+// anything that kernel could have written.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------------ append
 
 // One warp per token row (K and V rows of all KV heads of a token are
@@ -46,6 +67,8 @@ __global__ void __launch_bounds__(256)
                      const int64_t* __restrict__ slot_mapping, int num_tokens,
                      uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, int64_t num_slots,
                      int vec_per_row, unsigned* err) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t tok = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -78,11 +101,10 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t
   const int threads = 256, warps_per_cta = threads / 32;
   int64_t ctas = (static_cast<int64_t>(num_tokens) + warps_per_cta - 1) / warps_per_cta;
   if (ctas > 148 * 16) ctas = 148 * 16;
-  kv_append_kernel<<<static_cast<int>(ctas), threads, 0, stream>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), slot_mapping,
-      num_tokens, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots,
-      row_bytes / 16, err);
-  return cudaGetLastError();
+  return launch_pdl(kv_append_kernel, dim3(static_cast<unsigned>(ctas)), dim3(threads), 0, stream,
+                    static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                    slot_mapping, num_tokens, static_cast<uint4*>(k_cache),
+                    static_cast<uint4*>(v_cache), num_slots, row_bytes / 16, err);
 }
 
 // -------------------------------------------------------------- copy blocks
@@ -92,6 +114,8 @@ __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                        const int64_t* __restrict__ block_mapping, int num_blocks,
                        int64_t vec_per_block, unsigned* err) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t src = __ldg(block_mapping + 2 * blockIdx.x);
   const int64_t dst = __ldg(block_mapping + 2 * blockIdx.x + 1);
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -120,10 +144,9 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* bloc
   if (slices < 1) slices = 1;
   if (slices > 65535) slices = 65535;
   dim3 grid(num_pairs, static_cast<unsigned>(slices));
-  copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_cache),
-                                                   static_cast<uint4*>(v_cache), block_mapping,
-                                                   num_blocks, vec, err);
-  return cudaGetLastError();
+  return launch_pdl(copy_blocks_kernel, grid, dim3(threads), 0, stream,
+                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping,
+                    num_blocks, vec, err);
 }
 
 // ------------------------------------------------------------------ decode
@@ -145,9 +168,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 4-D view of a cache [num_blocks][block_size][num_kv_heads][head_dim]; a box is
-// `box_rows` consecutive tokens of one block for one KV head (head_dim x 1 x rows x 1).
+// `box_rows` consecutive tokens of one block for one KV head and `box_cols`
+// columns (all of head_dim when 0): box_cols x 1 x box_rows x 1.
 cudaError_t encode_cache_map(CUtensorMap* map, const void* base, const DecodeShape& sh,
-                             int box_rows) {
+                             int box_rows, int box_cols = 0, bool swizzle128 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   const int eb = sh.dtype == PA_BF16 ? 2 : 4;
@@ -158,66 +182,121 @@ cudaError_t encode_cache_map(CUtensorMap* map, const void* base, const DecodeSha
   const cuuint64_t row = static_cast<cuuint64_t>(sh.head_dim) * eb;
   const cuuint64_t strides[3] = {row, row * sh.num_kv_heads,
                                  row * sh.num_kv_heads * static_cast<cuuint64_t>(sh.block_size)};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(sh.head_dim), 1u,
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols ? box_cols : sh.head_dim), 1u,
                              static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
   CUresult r = enc(map, sh.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                    4, const_cast<void*>(base), dims, strides, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int D, int G>
-cudaError_t launch_decode_t(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
-                            const void* v_cache, cudaStream_t stream) {
-  using Cfg = DecodeConfig<T, D, G>;
-  constexpr int kMaxDevices = 64;
-  static std::atomic<unsigned long long> configured{0};
+// Sets a kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<unsigned long long>& configured) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const unsigned long long bit = 1ull << (dev % kMaxDevices);
-  if (!(configured.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(pa_decode_kernel<T, D, G>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured.fetch_or(bit, std::memory_order_acq_rel);
-  }
+  const unsigned long long bit = 1ull << (dev % 64);
+  if (configured.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) configured.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <typename T, int D>
+cudaError_t launch_merge(const DecodeShape& sh, const DecodeParams& p, cudaStream_t stream) {
+  if (sh.num_partitions <= 1) return cudaSuccess;
+  const unsigned rows = static_cast<unsigned>(sh.num_seqs) * sh.num_heads;
+  return launch_pdl(pa_merge_kernel<T, D>, dim3(rows), dim3(128), 0, stream, p);
+}
+
+// float32 caches: CUDA-core kernel (tensor maps, exact fp32 products).
+template <int D, int G>
+cudaError_t launch_decode_f32(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
+                              const void* v_cache, cudaStream_t stream) {
+  using Cfg = DecodeConfig<float, D, G>;
+  static std::atomic<unsigned long long> configured{0};
+  cudaError_t e = ensure_smem(pa_decode_kernel<float, D, G>, Cfg::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   CUtensorMap kmap, vmap;
   const int box_rows = sh.block_size < Cfg::kC ? sh.block_size : Cfg::kC;
   if ((e = encode_cache_map(&kmap, k_cache, sh, box_rows)) != cudaSuccess) return e;
   if ((e = encode_cache_map(&vmap, v_cache, sh, box_rows)) != cudaSuccess) return e;
   dim3 grid(sh.num_kv_heads, sh.num_partitions, sh.num_seqs);
-  pa_decode_kernel<T, D, G><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(kmap, vmap, p);
+  pa_decode_kernel<float, D, G><<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(kmap, vmap, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (sh.num_partitions > 1) {
-    dim3 rgrid(sh.num_heads, sh.num_seqs);
-    pa_reduce_kernel<T, D><<<rgrid, D, 0, stream>>>(p);
-    e = cudaGetLastError();
-  }
-  return e;
+  return launch_merge<float, D>(sh, p, stream);
 }
 
-template <typename T, int D>
+// 4-D view of a cache with the dimensions ordered (column, token, head, block)
+// so that a box {head_dim + 8, rows, heads, 1} lands in shared memory as
+// [head][token][head_dim + 8]; the 8 columns past head_dim are outside the
+// tensor and arrive as zeros (row padding against bank conflicts).
+cudaError_t encode_group_map(CUtensorMap* map, const void* base, const DecodeShape& sh,
+                             int box_rows, int box_heads) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t row = static_cast<cuuint64_t>(sh.head_dim) * 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(sh.head_dim),
+                              static_cast<cuuint64_t>(sh.block_size),
+                              static_cast<cuuint64_t>(sh.num_kv_heads),
+                              static_cast<cuuint64_t>(sh.num_blocks)};
+  const cuuint64_t strides[3] = {row * sh.num_kv_heads, row,
+                                 row * sh.num_kv_heads * static_cast<cuuint64_t>(sh.block_size)};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(sh.head_dim + 8),
+                             static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>(box_heads), 1u};
+  const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// bfloat16 caches: tensor-core kernel over groups of HB KV heads.
+template <int D, int G, int HB>
+cudaError_t launch_decode_bf16_t(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
+                                 const void* v_cache, cudaStream_t stream) {
+  // stages: as many as fit ~112 KB of ring (two CTAs per SM), at most 4
+  constexpr int kStage = 2 * GroupConfig<D, G, HB, 1>::kTensorBytes;
+  constexpr int kNSfit = 114688 / kStage;
+  constexpr int NS = kNSfit < 2 ? 2 : (kNSfit > 4 ? 4 : kNSfit);
+  using Cfg = GroupConfig<D, G, HB, NS>;
+  auto kernel = pa_decode_mma_kernel<D, G, HB, NS>;
+  static std::atomic<unsigned long long> configured{0};
+  cudaError_t e = ensure_smem(kernel, Cfg::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
+  CUtensorMap kmap, vmap;
+  const int rows = sh.block_size < Cfg::kC ? sh.block_size : Cfg::kC;
+  if ((e = encode_group_map(&kmap, k_cache, sh, rows, HB)) != cudaSuccess) return e;
+  if ((e = encode_group_map(&vmap, v_cache, sh, rows, HB)) != cudaSuccess) return e;
+  dim3 grid(sh.num_kv_heads / HB, sh.num_partitions, sh.num_seqs);
+  e = launch_pdl(kernel, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, kmap, vmap, p);
+  if (e != cudaSuccess) return e;
+  return launch_merge<__nv_bfloat16, D>(sh, p, stream);
+}
+
+template <int D, int G>
+cudaError_t launch_decode_bf16(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
+                               const void* v_cache, cudaStream_t stream) {
+  if (sh.num_kv_heads % 4 == 0) return launch_decode_bf16_t<D, G, 4>(sh, p, k_cache, v_cache, stream);
+  if (sh.num_kv_heads % 2 == 0) return launch_decode_bf16_t<D, G, 2>(sh, p, k_cache, v_cache, stream);
+  return launch_decode_bf16_t<D, G, 1>(sh, p, k_cache, v_cache, stream);
+}
+
+template <int D>
 cudaError_t dispatch_group(const DecodeShape& sh, const DecodeParams& p, const void* kc,
                            const void* vc, cudaStream_t st) {
+  const bool bf = sh.dtype == PA_BF16;
   switch (sh.num_heads / sh.num_kv_heads) {
-    case 1: return launch_decode_t<T, D, 1>(sh, p, kc, vc, st);
-    case 2: return launch_decode_t<T, D, 2>(sh, p, kc, vc, st);
-    case 4: return launch_decode_t<T, D, 4>(sh, p, kc, vc, st);
-    case 8: return launch_decode_t<T, D, 8>(sh, p, kc, vc, st);
-    default: return cudaErrorNotSupported;
-  }
-}
-
-template <typename T>
-cudaError_t dispatch_dim(const DecodeShape& sh, const DecodeParams& p, const void* kc,
-                         const void* vc, cudaStream_t st) {
-  switch (sh.head_dim) {
-    case 64: return dispatch_group<T, 64>(sh, p, kc, vc, st);
-    case 128: return dispatch_group<T, 128>(sh, p, kc, vc, st);
+    case 1: return bf ? launch_decode_bf16<D, 1>(sh, p, kc, vc, st) : launch_decode_f32<D, 1>(sh, p, kc, vc, st);
+    case 2: return bf ? launch_decode_bf16<D, 2>(sh, p, kc, vc, st) : launch_decode_f32<D, 2>(sh, p, kc, vc, st);
+    case 4: return bf ? launch_decode_bf16<D, 4>(sh, p, kc, vc, st) : launch_decode_f32<D, 4>(sh, p, kc, vc, st);
+    case 8: return bf ? launch_decode_bf16<D, 8>(sh, p, kc, vc, st) : launch_decode_f32<D, 8>(sh, p, kc, vc, st);
     default: return cudaErrorNotSupported;
   }
 }
@@ -232,8 +311,8 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   p.q = q;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  const WorkspaceLayout wl =
-      workspace_layout(sh.num_seqs, sh.num_heads, sh.head_dim, sh.num_partitions);
+  const WorkspaceLayout wl = workspace_layout(sh.num_seqs, sh.num_heads, sh.num_kv_heads,
+                                              sh.head_dim, sh.num_partitions);
   if (sh.num_partitions > 1) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.ws_m = reinterpret_cast<float*>(ws + wl.m_off);
@@ -254,8 +333,11 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   p.partition_size = sh.partition_size;
   p.num_partitions = sh.num_partitions;
   p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
-  if (sh.dtype == PA_BF16) return dispatch_dim<__nv_bfloat16>(sh, p, k_cache, v_cache, stream);
-  return dispatch_dim<float>(sh, p, k_cache, v_cache, stream);
+  switch (sh.head_dim) {
+    case 64: return dispatch_group<64>(sh, p, k_cache, v_cache, stream);
+    case 128: return dispatch_group<128>(sh, p, k_cache, v_cache, stream);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 }  // namespace pa

@@ -229,7 +229,7 @@ def test_short_contexts_under_a_large_grid():
     S, Hq, D = case.q.shape
     bt, cl, _ = case.cache.tables(case.seqs, max_blocks_per_seq=1024)
     out = torch.empty_like(case.out)
-    ws = torch.empty(pa.pa_decode_workspace_bytes(S, Hq, 2, D, 16000, 16), dtype=torch.uint8,
+    ws = torch.zeros(pa.pa_decode_workspace_bytes(S, Hq, 2, D, 16000, 16), dtype=torch.uint8,
                      device="cuda")
     pa.pa_decode(out, case.out.new_tensor(case.q).to(torch.bfloat16), case.cache.k_cache,
                  case.cache.v_cache, bt, cl, 16000, case.scale, 16, ws)
