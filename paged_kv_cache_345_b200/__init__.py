@@ -4,7 +4,7 @@ This module only marshals arguments: it turns torch tensors and numpy arrays
 into pointers and sizes and calls the C ABI declared in include/pa.h. Every
 step of the hot path runs in the library's CUDA kernels or its C++ block
 manager. There is no CPU fallback: importing this package fails if libpa.so
-has not been built (python -m paged_kv_cache_345_b200.build).
+has not been built (python paged_kv_cache_345_b200/build.py).
 
 Entry points (same names as the C ABI):
   pa_kv_append     write new tokens' K/V rows into their slots
@@ -38,7 +38,7 @@ lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 if not os.path.exists(lib_path):
     raise ImportError(
         f"{lib_path} is missing: build the CUDA library first "
-        "(python -m paged_kv_cache_345_b200.build). There is no CPU fallback.")
+        "(python paged_kv_cache_345_b200/build.py). There is no CPU fallback.")
 _lib = ctypes.CDLL(lib_path)
 
 _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, \

@@ -1,6 +1,7 @@
 """Build libpa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: python -m paged_kv_cache_345_b200.build [--force] [--verbose]
+Usage: python paged_kv_cache_345_b200/build.py [--force] [--verbose]
+(run it by path: importing the package first would load the library.)
 The shared library lands next to this file; objects go to _build/ at the
 repository root. A rebuild happens only when a source or header is newer than
 the library (or with --force).
