@@ -361,8 +361,23 @@ def run_b200(args, wl, rank, world, local_rank):
     bytes_step = kv_bytes(wl)
     tokens_step = sum(n + 1 for n in wl.context_lens)
 
+    # L2 flush between steps: write a buffer larger than L2, then read another
+    # one, so the timed step starts with L2 holding clean, unrelated lines (a
+    # write alone would leave the step paying for the write-back of its dirty
+    # lines).
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
+    flush_w = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
+    flush_r = torch.ones((2 * l2 + (64 << 20)) // 4, dtype=torch.float32, device=device)
+
+    class _Flush:
+        def zero_(self):
+            flush_w.zero_()
+            flush_r.sum()
+
+        def numel(self):
+            return flush_w.numel() + flush_r.numel() * 4
+
+    flush = _Flush()
 
     def barrier():
         if world > 1:
@@ -471,7 +486,8 @@ def run_b200(args, wl, rank, world, local_rank):
                    "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
                    "partition_size": calls.partition_size,
                    "num_partitions": calls.num_partitions, "copy_on_write_pairs": cow_pairs,
-                   "l2": f"flushed between steps ({flush.numel() >> 20} MiB write, outside the "
+                   "l2": f"flushed between steps ({flush_w.numel() >> 20} MiB written, then "
+                         f"{(flush_r.numel() * 4) >> 20} MiB of another buffer read; outside the "
                          "timed events)",
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": tokens_step * args.steps * world / (total_ms * 1e-3),
