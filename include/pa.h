@@ -168,6 +168,42 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is an interface convenience of this
+ * library, not part of the method.
+ *
+ * Some callers cannot call cudaMalloc where they decode: their framework's
+ * memory manager owns the whole device pool, their serving loop must not take
+ * an allocation's implicit synchronisation, or they are plain C hosts that
+ * only receive pointers to buffers made elsewhere. pa_decode_noalloc takes the
+ * same arguments as pa_decode minus the workspace and keeps the split-K
+ * partial results in a scratch array compiled into the library:
+ *   - The array holds PA_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) on every GPU
+ *     that loads the library, until the process exits.
+ *   - A call whose pa_decode_workspace_bytes(...) exceeds that size returns
+ *     PA_ERR_INVALID before launching anything (raise partition_size, split
+ *     the batch, or use pa_decode with your own workspace).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture. Later calls do no set-up.
+ *   - Nothing here allocates: no cudaMalloc, cudaFree or allocating library
+ *     routine.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents. Nothing in it has to start at zero: each call writes every
+ *     value it reads back. Calls whose kernels overlap on the GPU (different
+ *     streams, or several host threads) race on the array and give wrong
+ *     results; serialise them.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, pa_dtype dtype, pa_stream_t stream);
+/* Size of the scratch array behind pa_decode_noalloc, in bytes. */
+size_t pa_decode_noalloc_scratch_bytes(void);
+
+/*
  * pa_device_errors — synchronise `stream`, return the device error word
  * (PA_DEVERR_* bits set by kernels since the last call) in *flags and clear
  * it. Returns PA_ERR_DEVICE_CHECK if any bit was set, PA_OK otherwise. The

@@ -60,6 +60,9 @@ _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _f32, _i32, _vp, _sz, _i32, _vp)
+_sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _f32, _i32, _i32, _vp)
+_sig("pa_decode_noalloc_scratch_bytes", _sz)
 _sig("pa_device_errors", _i32, _vp, ctypes.POINTER(ctypes.c_uint))
 _sig("pa_last_error", ctypes.c_char_p)
 _sig("pa_status_string", ctypes.c_char_p, _i32)
@@ -87,7 +90,8 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 
 EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_device_errors", "pa_last_error", "pa_status_string", "pa_alloc_create",
+    "pa_decode", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
+    "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
     "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
     "pa_bm_allocator", "pa_bm_block_size", "pa_bm_add_seq", "pa_bm_fork", "pa_bm_free_seq",
