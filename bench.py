@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--block-size", type=int, default=16, help="long_context only")
     ap.add_argument("--partition-size", type=int, default=-1,
                     help="tokens per split-K partition (-1: tuned default, 0: library choice)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -148,9 +150,12 @@ def build_on_gpu(wl, device):
 
 
 class StepCalls:
-    """The C-ABI calls of one decode step with their arguments marshalled once."""
+    """The C-ABI calls of one decode step with their arguments marshalled once.
 
-    def __init__(self, cache, dev, max_len, scale, partition_size, stream):
+    fused: the step is one pa_decode_append call (append each newest token, then
+    attend); otherwise pa_kv_append followed by pa_decode (same result)."""
+
+    def __init__(self, cache, dev, max_len, scale, partition_size, stream, fused=True):
         import torch
 
         import paged_kv_cache_345_b200 as pa
@@ -172,7 +177,12 @@ class StepCalls:
                             p(dev["tables"]), p(dev["lens"]), s, hq, hkv, d, bs, nb,
                             dev["tables"].shape[1], max_len, scale, self.partition_size,
                             p(self.workspace), self.workspace.numel(), dt, st)
-        self.launches_per_step = 2 + (1 if self.num_partitions > 1 else 0)
+        self.step_args = (p(self.out), p(dev["q"]), p(dev["k_new"]), p(dev["v_new"]),
+                          p(cache.k_cache), p(cache.v_cache), p(dev["tables"]), p(dev["lens"]),
+                          s, hq, hkv, d, bs, nb, dev["tables"].shape[1], max_len, scale,
+                          self.partition_size, p(self.workspace), self.workspace.numel(), dt, st)
+        self.fused = fused
+        self.launches_per_step = (1 if fused else 2) + (1 if self.num_partitions > 1 else 0)
 
     def append(self):
         st = self.lib.pa_kv_append(*self.append_args)
@@ -183,6 +193,15 @@ class StepCalls:
         st = self.lib.pa_decode(*self.decode_args)
         if st:
             raise RuntimeError(f"pa_decode: {self.lib.pa_last_error().decode()}")
+
+    def step(self):
+        if not self.fused:
+            self.append()
+            self.decode()
+            return
+        st = self.lib.pa_decode_append(*self.step_args)
+        if st:
+            raise RuntimeError(f"pa_decode_append: {self.lib.pa_last_error().decode()}")
 
 
 # --------------------------------------------------------------------- clocks
@@ -320,11 +339,21 @@ def run_reference(args, wl, rank):
     }), flush=True)
 
 
+def kernel_source_digest() -> str:
+    """sha256 (first 16 hex digits) over the decode kernels' sources."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_345_b200", "csrc")
+    for path in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + [os.path.join(csrc, "pa_kernels.cu")]):
+        h.update(open(path, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel_key: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source (matching source hash), else None."""
-    import hashlib
-
     path = os.path.join(ROOT, "profiles", f"{kernel_key}.traffic.txt")
     if not os.path.exists(path):
         return None
@@ -333,8 +362,7 @@ def load_traffic(kernel_key: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    src = os.path.join(ROOT, "paged_kv_cache_345_b200", "csrc", "pa_decode.cuh")
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    digest = kernel_source_digest()
     if vals.get("source_sha256_16") != digest:
         return None
     try:
@@ -357,7 +385,7 @@ def run_b200(args, wl, rank, world, local_rank):
 
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device)
     ps = TUNED_PARTITION[wl.name.split("_bs")[0]] if args.partition_size < 0 else args.partition_size
-    calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream)
+    calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused)
     bytes_step = kv_bytes(wl)
     tokens_step = sum(n + 1 for n in wl.context_lens)
 
@@ -387,12 +415,11 @@ def run_b200(args, wl, rank, world, local_rank):
     # ---- device-resident steps
     for _ in range(args.warmup):
         flush.zero_()
-        calls.append()
-        calls.decode()
+        calls.step()
     torch.cuda.synchronize(device)
     if pa.pa_device_errors() != 0:
         raise RuntimeError("device error word set during warm-up")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(local_rank)
     clocks.start()
     barrier()
@@ -400,15 +427,13 @@ def run_b200(args, wl, rank, world, local_rank):
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        calls.append()
+        calls.step()
         ev[i][1].record(stream)
-        calls.decode()
-        ev[i][2].record(stream)
     barrier()
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
-    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    decode_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    decode_ms = step_ms  # the step's kernels: (append +) decode + split-K merge
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], device=device)
@@ -421,15 +446,14 @@ def run_b200(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         out_host = torch.empty(calls.out.shape, dtype=calls.out.dtype).pin_memory()
-        names = ("q", "k_new", "v_new", "slots", "tables", "lens")
+        names = ("q", "k_new", "v_new", "tables", "lens") + (() if calls.fused else ("slots",))
         h2d = sum(host[k].numel() * host[k].element_size() for k in names)
         d2h = out_host.numel() * out_host.element_size()
 
         def e2e_step():
             for k in names:
                 dev[k].copy_(host[k], non_blocking=True)
-            calls.append()
-            calls.decode()
+            calls.step()
             out_host.copy_(calls.out, non_blocking=True)
 
         for _ in range(args.warmup):
@@ -492,12 +516,12 @@ def run_b200(args, wl, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": tokens_step * args.steps * world / (total_ms * 1e-3),
         "us_per_step": 1e3 * total_ms / args.steps,
-        "us_per_decode_call": 1e3 * statistics.mean(decode_ms),
-        "decode_call_us_p10_p50_p90": [1e3 * float(np.percentile(decode_ms, p))
-                                       for p in (10, 50, 90)],
+        "step_us_p10_p50_p90": [1e3 * float(np.percentile(decode_ms, p)) for p in (10, 50, 90)],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "pa_decode (decode kernel + split-K merge kernel)",
+                     "kernel": ("pa_decode_append (fused append + decode kernel, split-K "
+                                "merge kernel)" if calls.fused else
+                                "pa_kv_append + pa_decode (decode + split-K merge kernels)"),
                      "peak_source": f"{peak_src} hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": e2e,

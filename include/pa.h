@@ -168,6 +168,34 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_decode_append — one whole decode step in one call: append each
+ * sequence's newest token, then attend over the context including it.
+ * "What is paged attention in vLLM...", Step 4: at each decoding step the
+ * system writes the new token's keys and values into the last block;
+ * "Paged Attention" (klaylearn.com glossary), definition: decode appends into
+ * the tail block. Same result as pa_kv_append (with each new token's slot
+ * taken from the block table) followed by pa_decode, without the separate
+ * launch: the CTA that reads a sequence's last position writes it first.
+ *
+ *   k_new, v_new   device, [num_seqs][num_kv_heads][head_dim], dtype: the K
+ *                  and V rows of each sequence's newest token, which sits at
+ *                  position context_lens[s] - 1 (context_lens counts it). Its
+ *                  slot is block_tables[s][(L - 1) / block_size] * block_size
+ *                  + (L - 1) % block_size; that block must already be in the
+ *                  table and not shared (copy-on-write first, pa_copy_blocks).
+ *   k_cache, v_cache  device, the newest rows are written in place.
+ * Everything else as pa_decode. A sequence with context_lens[s] == 0 appends
+ * nothing. A table entry outside the pool sets PA_DEVERR_BLOCK_ID and the row
+ * is not written.
+ */
+int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                     void* k_cache, void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                     int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                     int max_context_len, float scale, int partition_size, void* workspace,
+                     size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The pages have no counterpart: this is an interface convenience of this
  * library, not part of the method.

@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
   pa_kv_append     write new tokens' K/V rows into their slots
   pa_copy_blocks   copy-on-write of shared blocks
   pa_decode        paged decode attention (split-K over partitions)
+  pa_decode_append one decode step: append each newest token, then attend
   BlockManager     host free list + reference counts + block tables
 """
 
@@ -24,7 +25,8 @@ __all__ = [
     "PagedAttentionError", "PA_OK", "PA_ERR_INVALID", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_NO_BLOCKS", "PA_ERR_DEVICE_CHECK", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID",
     "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
-    "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
+    "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_decode", "pa_decode_append",
+    "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
 ]
 
@@ -60,6 +62,8 @@ _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _f32, _i32, _vp, _sz, _i32, _vp)
+_sig("pa_decode_append", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i32, _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _f32, _i32, _i32, _vp)
 _sig("pa_decode_noalloc_scratch_bytes", _sz)
@@ -90,7 +94,7 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 
 EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
+    "pa_decode", "pa_decode_append", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
     "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
@@ -205,6 +209,34 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
         ws_bytes = workspace.numel() * workspace.element_size()
     _check(_lib.pa_decode(
         _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
+        block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,
+        ws_bytes, _dtype_code(k_cache), _stream(stream, q.device)))
+
+
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                     max_context_len: int, scale: float, partition_size: int = 0, workspace=None,
+                     stream=None) -> None:
+    """Append each sequence's newest token (k_new / v_new [S, Hkv, d], at position
+    context_lens[s] - 1 through the block table), then attend; see include/pa.h."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    s, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if k_new.shape != (s, hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new/v_new must be [S, num_kv_heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    dt = k_cache.dtype
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_append(
+        _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_new, "k_new", dt),
+        _dev_ptr(v_new, "v_new", dt), _dev_ptr(k_cache, "k_cache"),
         _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
         _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
         block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,

@@ -8,7 +8,10 @@ workspace. Each method marshals arguments and calls libpa.so:
       tail blocks first when needed (pa_copy_blocks), then scatter the rows
       (pa_kv_append). Serves both prefill (many tokens) and decode (one token).
   decode(q, seq_ids)  block tables to the device, then pa_decode.
-  decode_step(q, k_new, v_new, seq_ids)  write one token per sequence, then decode.
+  decode_step(q, k_new, v_new, seq_ids)  one decode step: reserve each sequence's
+      next slot (native; shared tail blocks copied first), then pa_decode_append
+      writes the new K/V rows and attends in one launch (fused=False: separate
+      pa_kv_append and pa_decode calls, same result).
 
 "Paged Attention" (klaylearn.com glossary), definition: prefill allocates and
 fills blocks, decode appends into the tail block or triggers an allocation,
@@ -20,8 +23,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_partition_size,
-               pa_decode_workspace_bytes, pa_kv_append)
+from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append,
+               pa_decode_partition_size, pa_decode_workspace_bytes, pa_kv_append)
 
 _TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
 
@@ -102,6 +105,21 @@ class PagedKVCache:
         return out
 
     def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
-                    out=None):
-        self.write(seq_ids, [1] * len(seq_ids), k_new, v_new)
-        return self.decode(q, seq_ids, scale, partition_size, out)
+                    out=None, fused: bool = True):
+        if not fused:
+            self.write(seq_ids, [1] * len(seq_ids), k_new, v_new)
+            return self.decode(q, seq_ids, scale, partition_size, out)
+        _, cows = self.bm.append_slots(seq_ids, [1] * len(seq_ids))
+        if len(cows):
+            pa_copy_blocks(self.k_cache, self.v_cache, self._to_device(cows), stream=self.stream)
+        num_seqs, num_heads, _ = q.shape
+        block_tables, context_lens, max_len = self.tables(seq_ids)
+        if partition_size == 0:
+            partition_size = pa_decode_partition_size(num_seqs, self.num_kv_heads, max_len)
+        out = torch.empty_like(q) if out is None else out
+        scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+        pa_decode_append(out, q, k_new, v_new, self.k_cache, self.v_cache, block_tables,
+                         context_lens, max_len, scale, partition_size,
+                         self.workspace(num_seqs, num_heads, max_len, partition_size),
+                         stream=self.stream)
+        return out

@@ -158,11 +158,13 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
   return pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, np).total;
 }
 
-int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-              const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
-              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-              int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
-              void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+static int decode_common(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                         int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void* workspace, size_t workspace_bytes,
+                         pa_dtype dtype, const void* k_new, const void* v_new,
+                         pa_stream_t stream) {
   if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode: num_seqs < 0");
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
@@ -225,10 +227,38 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
     return pa_fail(PA_ERR_INVALID, "pa_decode: workspace %zu B < %zu B needed",
                    workspace ? workspace_bytes : size_t(0), need);
   cudaError_t e = pa::launch_decode(sh, out, q, k_cache, v_cache, block_tables, context_lens,
-                                    workspace, reinterpret_cast<cudaStream_t>(stream));
+                                    workspace, k_new, v_new,
+                                    reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: no kernel for this shape");
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode launch", e);
+}
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+              int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
+              void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype,
+                       nullptr, nullptr, stream);
+}
+
+int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                     void* k_cache, void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                     int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                     int max_context_len, float scale, int partition_size, void* workspace,
+                     size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs > 0 && (!k_new || !v_new))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_append: null k_new or v_new");
+  if (num_seqs > 0 && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_append: misaligned k_new or v_new");
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype,
+                       k_new, v_new, stream);
 }
 
 int pa_device_errors(pa_stream_t stream, unsigned int* flags) {

@@ -33,6 +33,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "pa_device.cuh"
 
@@ -46,11 +47,39 @@ struct DecodeParams {
   float* ws_m;    // [S][Hq][NP]  running max (base-2 domain) per partition
   float* ws_l;    // [S][Hq][NP]  softmax denominator per partition
   float* ws_acc;  // [S][Hq][NP][D] unnormalised output per partition
+  // Fused append (pa_decode_append): each sequence's newest token (position
+  // context_lens[s] - 1) is written from k_new / v_new [S][Hkv][D] into the
+  // caches through the block table before it is read. Null for pa_decode.
+  const uint8_t* k_new;
+  const uint8_t* v_new;
+  uint8_t* k_cache_w;
+  uint8_t* v_cache_w;
   unsigned* err;
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks;
   int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
   float q_scale;  // scale * log2(e)
 };
+
+
+// Fused append (pa_decode_append): the producer warp of the CTA that holds a
+// sequence's newest token copies that token's K and V rows for KV heads
+// [h0, h0 + nh) from k_new / v_new into cache block `blk` at offset `off`,
+// then orders these generic-proxy writes before the TMA reads that follow.
+__device__ __forceinline__ void append_newest_rows(const DecodeParams& p, int s, int blk, int off,
+                                                   int h0, int nh, int row_bytes, int lane) {
+  const int64_t vec = static_cast<int64_t>(nh) * row_bytes / 16;
+  const int64_t src = (static_cast<int64_t>(s) * p.num_kv_heads + h0) * row_bytes;
+  const int64_t dst =
+      ((static_cast<int64_t>(blk) * p.block_size + off) * p.num_kv_heads + h0) * row_bytes;
+  for (int64_t i = lane; i < vec; i += 32) {
+    const uint4 a = ldg_stream(p.k_new + src + i * 16);
+    const uint4 b = ldg_stream(p.v_new + src + i * 16);
+    *reinterpret_cast<uint4*>(p.k_cache_w + dst + i * 16) = a;
+    *reinterpret_cast<uint4*>(p.v_cache_w + dst + i * 16) = b;
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncwarp();
+}
 
 template <typename T, int D, int G>
 struct DecodeConfig {
@@ -179,6 +208,15 @@ __global__ void __launch_bounds__(DecodeConfig<T, D, G>::kThreads)
       const uint32_t full_bar = smem_u32(bars + bi);
       const uint32_t kdst = smem_u32(smem + bi * Cfg::kStageBytes);
       const uint32_t vdst = kdst + C * ROW;
+      if (p.k_new != nullptr && c == nchunks - 1 && t1 == L) {
+        // this CTA holds the sequence's newest token: write it before reading it
+        const int tn = L - 1;
+        const int bn = __ldg(trow + (tn >> p.log2_block_size));
+        if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks))
+          append_newest_rows(p, s, bn, tn & (bs - 1), h, 1, ROW, lane);
+        else if (lane == 0)
+          atomicOr(p.err, PA_DEVERR_BLOCK_ID);
+      }
       if (lane == 0) mbar_arrive_expect_tx(full_bar, 2u * nblk * rows_per_box * ROW);
       for (int b = 0; b < nblk; ++b) {
         const int lb = lb0 + b;
@@ -368,61 +406,86 @@ __global__ void __launch_bounds__(DecodeConfig<T, D, G>::kThreads)
 // Split-K merge: one CTA of 4 warps per (sequence, query head) row with more
 // than one partition:
 //   M = max_p m_p,  Lambda = sum_p l_p 2^(m_p - M),  out = sum_p 2^(m_p - M) acc_p / Lambda.
-// Warp w takes partitions w, w + 4, ...; each lane owns D / 32 columns, so a
-// warp's partition rows are independent loads, all in flight together. The
-// four warps' sums are added in warp order through shared memory, so the
-// result depends only on the partials (deterministic). Launched with
-// programmatic dependent launch: it waits for the decode kernel before reading.
+// Warp w takes partitions w, w + 4, ... in batches of 8: a batch's maxima,
+// sums and accumulator rows (each lane owns D / 32 columns) are loaded
+// together, so a row with up to 32 partitions costs one round trip; batches
+// are folded in with an online rescale. The four warps' results are combined
+// in warp order through shared memory: the result depends only on the
+// partials (deterministic). Launched with programmatic dependent launch.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
-  constexpr int E = D / 32;
-  __shared__ float s_max[4], s_l[4], s_acc[4][D];
-  pdl_wait();
+  constexpr int E = D / 32;  // columns per lane
+  constexpr int B = 8;       // partitions per warp per batch
+  using Vec = typename std::conditional<E == 4, float4, float2>::type;
+  __shared__ float s_m[4], s_l[4], s_acc[4][D];
   const int64_t r = blockIdx.x;  // row = s * num_heads + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = static_cast<int>(r / p.num_heads);
+  // The context length is read before the dependent-launch wait: the kernel
+  // before this one is the decode kernel of the same call, which itself waited
+  // for all earlier work before letting this kernel start, and neither writes it.
   const int L = __ldg(p.context_lens + s);
   if (L < 0 || L > p.max_context_len ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size)
     return;  // flagged and zero-filled by the decode kernel
   const int np = (L + p.partition_size - 1) / p.partition_size;
   if (np <= 1) return;  // written directly by the decode kernel
+  pdl_wait();  // the partials are the decode kernel's output
   const int64_t row = r * p.num_partitions;
-  float M = -INFINITY;
-  for (int q = threadIdx.x; q < np; q += 128) M = fmaxf(M, __ldcg(p.ws_m + row + q));
-#pragma unroll
-  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
-  if (lane == 0) s_max[warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-  float acc[E], lw = 0.0f;
+  const float* a = p.ws_acc + row * D + lane * E;
+  float Mw = -INFINITY, Lw = 0.0f, acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-  const float* a = p.ws_acc + row * D + lane * E;
-#pragma unroll 4
-  for (int q = warp; q < np; q += 4) {
-    const float w = exp2f(__ldcg(p.ws_m + row + q) - M);
-    lw = fmaf(w, __ldcg(p.ws_l + row + q), lw);
-    if constexpr (E == 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(a + static_cast<int64_t>(q) * D));
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-    } else {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(a + static_cast<int64_t>(q) * D));
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
+  for (int q0 = warp; q0 < np; q0 += 4 * B) {
+    float mq[B], lq[B];
+    Vec vq[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const int q = q0 + 4 * j;
+      if (q < np) {
+        mq[j] = __ldcg(p.ws_m + row + q);
+        lq[j] = __ldcg(p.ws_l + row + q);
+        vq[j] = __ldcg(reinterpret_cast<const Vec*>(a + static_cast<int64_t>(q) * D));
+      } else {
+        mq[j] = -INFINITY;
+        lq[j] = 0.0f;
+        vq[j] = Vec{};
+      }
     }
+    float bm = Mw;
+#pragma unroll
+    for (int j = 0; j < B; ++j) bm = fmaxf(bm, mq[j]);
+    const float sc = exp2f(Mw - bm);  // 0 on the first batch (Mw = -inf, bm finite)
+    Lw *= sc;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] *= sc;
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const float w = exp2f(mq[j] - bm);  // 0 for the padding slots of a batch
+      Lw = fmaf(w, lq[j], Lw);
+      const float* v = reinterpret_cast<const float*>(&vq[j]);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+    }
+    Mw = bm;
   }
 #pragma unroll
   for (int e = 0; e < E; ++e) s_acc[warp][lane * E + e] = acc[e];
-  if (lane == 0) s_l[warp] = lw;
+  if (lane == 0) {
+    s_m[warp] = Mw;
+    s_l[warp] = Lw;
+  }
   __syncthreads();
   if (threadIdx.x < D) {
     const int d = threadIdx.x;
-    const float lsum = ((s_l[0] + s_l[1]) + s_l[2]) + s_l[3];
-    const float v = ((s_acc[0][d] + s_acc[1][d]) + s_acc[2][d]) + s_acc[3][d];
+    const float M = fmaxf(fmaxf(s_m[0], s_m[1]), fmaxf(s_m[2], s_m[3]));
+    float lsum = 0.0f, v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float f = s_m[w] == -INFINITY ? 0.0f : exp2f(s_m[w] - M);
+      lsum = fmaf(f, s_l[w], lsum);
+      v = fmaf(f, s_acc[w][d], v);
+    }
     ElemTraits<T>::store(static_cast<T*>(p.out) + r * D + d, v / lsum);
   }
 }

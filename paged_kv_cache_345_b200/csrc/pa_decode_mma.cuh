@@ -99,6 +99,10 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
     }
     fence_barrier_init();
   }
+  if (warp == HB && lane == 0) {  // descriptors are kernel parameters: fetch them early
+    prefetch_tensormap(&k_map);
+    prefetch_tensormap(&v_map);
+  }
   pdl_wait();  // inputs may come from the previous kernel in the stream
   pdl_launch_dependents();
 
@@ -149,10 +153,6 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
 
   if (warp == HB) {
     // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tensormap(&k_map);
-      prefetch_tensormap(&v_map);
-    }
     const int lb_last = (t1 - 1) >> lg;
     for (int c = 0; c < nchunks; ++c) {
       const int st = c % NS, u = c / NS;
@@ -167,6 +167,15 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
       if (lb_hi - base >= 32) {  // refill: the next 32 table entries, one per lane
         base = lb_lo;
         ent = (base + lane <= lb_last) ? __ldg(trow + base + lane) : 0;
+      }
+      if (p.k_new != nullptr && c == nchunks - 1 && t1 == L) {
+        // this CTA holds the sequence's newest token: write it before reading it
+        const int tn = L - 1;
+        const int bn = __shfl_sync(kFullMask, ent, (tn >> lg) - base);
+        if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks))
+          append_newest_rows(p, s, bn, tn & (bs - 1), hg * HB, HB, Cfg::kRowBytes, lane);
+        else if (lane == 0)
+          atomicOr(p.err, PA_DEVERR_BLOCK_ID);
       }
       const int nbox = lb_hi - lb_lo + 1;  // blocks holding valid tokens of this chunk
       const int blk = __shfl_sync(kFullMask, ent, min(lane, nbox - 1) + lb_lo - base);

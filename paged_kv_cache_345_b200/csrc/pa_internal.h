@@ -43,9 +43,11 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* bloc
                                int num_pairs, int num_blocks, int64_t block_bytes,
                                cudaStream_t stream);
 // Returns cudaErrorNotSupported when no kernel is built for the shape.
+// k_new / v_new non-null: fused append of each sequence's newest token.
 cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* block_tables,
-                          const int32_t* context_lens, void* workspace, cudaStream_t stream);
+                          const int32_t* context_lens, void* workspace, const void* k_new,
+                          const void* v_new, cudaStream_t stream);
 // Device error word of the current device (address in device memory).
 cudaError_t device_error_word(unsigned int** ptr);
 

@@ -305,9 +305,14 @@ cudaError_t dispatch_group(const DecodeShape& sh, const DecodeParams& p, const v
 
 cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* block_tables,
-                          const int32_t* context_lens, void* workspace, cudaStream_t stream) {
+                          const int32_t* context_lens, void* workspace, const void* k_new,
+                          const void* v_new, cudaStream_t stream) {
   DecodeParams p{};
   p.out = out;
+  p.k_new = static_cast<const uint8_t*>(k_new);
+  p.v_new = static_cast<const uint8_t*>(v_new);
+  p.k_cache_w = static_cast<uint8_t*>(const_cast<void*>(k_cache));
+  p.v_cache_w = static_cast<uint8_t*>(const_cast<void*>(v_cache));
   p.q = q;
   p.block_tables = block_tables;
   p.context_lens = context_lens;

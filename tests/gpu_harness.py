@@ -92,7 +92,7 @@ def stage_rows(wl, device="cuda", keep=None):
 
 
 def build_case(wl, device="cuda", free_order=None, partition_size=None, share_prefix=True,
-               staged=None, keep=None):
+               staged=None, keep=None, fused=True):
     """Prefill every sequence, then one decode step (append one token each + attend)."""
     from paged_kv_cache_345_b200.cache import PagedKVCache
 
@@ -135,7 +135,7 @@ def build_case(wl, device="cuda", free_order=None, partition_size=None, share_pr
     k_new, v_new = sk.index_select(0, last), sv.index_select(0, last)
     ps = wl.partition_size if partition_size is None else partition_size
     qd = torch.from_numpy(q).to(device=device, dtype=tdt)
-    out = cache.decode_step(qd, k_new, v_new, seqs, wl.scale, ps)
+    out = cache.decode_step(qd, k_new, v_new, seqs, wl.scale, ps, fused=fused)
     torch.cuda.synchronize()
     return Case(cache, seqs, rows_k, rows_v, q, out, wl.scale, wl.dtype)
 

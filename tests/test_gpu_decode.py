@@ -235,3 +235,18 @@ def test_short_contexts_under_a_large_grid():
                  case.cache.v_cache, bt, cl, 16000, case.scale, 16, ws)
     gh.assert_close(out.float().cpu().numpy(), gh.expected_all(case), "bf16", "large grid")
     assert pa.pa_device_errors() == 0
+
+
+@pytest.mark.parametrize("bs", [1, 4, 16, 64])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fused_step_equals_append_then_decode(bs, dtype):
+    """pa_decode_append (one launch) == pa_kv_append + pa_decode, bit for bit,
+    in the output and in the caches it wrote."""
+    wl = _custom(8, 2, 128, dtype, bs, RAGGED + (600,))
+    a = gh.build_case(wl, partition_size=48, fused=True)
+    b = gh.build_case(wl, partition_size=48, fused=False)
+    assert torch.equal(a.out, b.out)
+    assert torch.equal(a.cache.k_cache, b.cache.k_cache)
+    assert torch.equal(a.cache.v_cache, b.cache.v_cache)
+    gh.assert_close(gh.gpu_out(a), gh.expected_all(a), dtype, f"fused bs={bs}")
+    assert pa.pa_device_errors() == 0
