@@ -46,13 +46,20 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="llama3_8b_layer",
-                    choices=["llama3_8b_layer", "large_batch", "shared_prefix", "long_context"])
+                    choices=["llama3_8b_layer", "large_batch", "shared_prefix", "long_context",
+                             "swap"])
+    ap.add_argument("--placement", choices=["random", "identity"], default="random",
+                    help="physical block order: a seeded permutation (default) or identity "
+                         "(each sequence's blocks contiguous in memory)")
     ap.add_argument("--block-size", type=int, default=16, help="long_context only")
     ap.add_argument("--partition-size", type=int, default=-1,
                     help="tokens per split-K partition (-1: tuned default, 0: library choice)")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-back-to-back", action="store_true")
+    ap.add_argument("--layers", type=int, default=32,
+                    help="cache replicas of the back-to-back figure (one per model layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     return ap.parse_args()
@@ -85,7 +92,7 @@ def kv_bytes(wl) -> int:
 
 # ------------------------------------------------------------------ GPU setup
 
-def build_on_gpu(wl, device):
+def build_on_gpu(wl, device, placement="random"):
     """Prefill every sequence through the library, then prepare one decode step."""
     import torch
 
@@ -95,9 +102,10 @@ def build_on_gpu(wl, device):
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     bs = wl.block_size
     max_blocks = max(-(-(n + 1) // bs) for n in wl.context_lens)
+    order = synth.block_permutation(wl.num_blocks, wl.placement_seed) if placement == "random" \
+        else np.arange(wl.num_blocks, dtype=np.int32)
     cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.dtype, device,
-                         max_blocks_per_seq=max_blocks,
-                         free_order=synth.block_permutation(wl.num_blocks, wl.placement_seed))
+                         max_blocks_per_seq=max_blocks, free_order=order)
     ghosts = [cache.add_sequence() for _ in wl.ghost_lens]
     if ghosts:
         cache.bm.append_slots(ghosts, list(wl.ghost_lens))
@@ -381,9 +389,11 @@ def run_b200(args, wl, rank, world, local_rank):
     torch.cuda.set_device(device)
     if world > 1:
         dist.init_process_group("nccl", device_id=device)
-    stream = torch.cuda.current_stream(device)
+    # a stream of our own (CUDA graphs cannot be captured on the default stream)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
 
-    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device)
+    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device, args.placement)
     ps = TUNED_PARTITION[wl.name.split("_bs")[0]] if args.partition_size < 0 else args.partition_size
     calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused)
     bytes_step = kv_bytes(wl)
@@ -476,12 +486,58 @@ def run_b200(args, wl, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.steps}
 
+    # ---- back to back: the same step over `layers` different cache replicas
+    # (one per model layer, together far larger than L2, so no flush), all
+    # layers captured in one CUDA graph and replayed. Consecutive layers
+    # overlap launch and start-up through programmatic dependent launch.
+    b2b = None
+    if not args.no_back_to_back and world == 1:
+        reps = []
+        for _ in range(args.layers):
+            kc = cache.k_cache.clone()
+            vc = cache.v_cache.clone()
+            reps.append((kc, vc))
+        del kc, vc
+        layer_calls = []
+        for kc, vc in reps:
+            view = type("CacheView", (), {})()
+            view.k_cache, view.v_cache = kc, vc
+            layer_calls.append(StepCalls(view, dev, max_len, wl.scale, calls.partition_size,
+                                         stream, fused=calls.fused))
+        for c in layer_calls:   # warm-up, eager
+            c.step()
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for c in layer_calls:
+                c.step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(device)
+        reps_n = max(5, min(50, args.steps // args.layers))
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps_n)]
+        for i in range(reps_n):
+            gev[i][0].record(stream)
+            graph.replay()
+            gev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        per_layer_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in gev) / args.layers
+        if pa.pa_device_errors() != 0:
+            raise RuntimeError("device error word set during the back-to-back replay")
+        b2b = {"layers": args.layers, "us_per_layer": 1e3 * per_layer_ms,
+               "kv_GB_per_s": bytes_step / (per_layer_ms * 1e-3) / 1e9,
+               "how": "one CUDA graph of the step over per-layer cache replicas, no L2 flush"}
+        del graph, layer_calls, reps
+        torch.cuda.empty_cache()
+
     # ---- roofline of pa_decode (decode kernel + split-K merge kernel)
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(peaks_path):
         peak, peak_src = float(json.load(open(peaks_path))["hbm_gbs"]), "measured"
     else:
         peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+    if b2b is not None:
+        b2b["frac_of_peak"] = b2b["kv_GB_per_s"] / peak
     dec_s = statistics.mean(decode_ms) * 1e-3
     achieved = bytes_step / dec_s / 1e9
     traffic = load_traffic(f"pa_decode_{wl.name}")
@@ -525,6 +581,7 @@ def run_b200(args, wl, rank, world, local_rank):
                      "peak_source": f"{peak_src} hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "back_to_back": b2b,
         "gpu_launches": calls.launches_per_step * args.steps,
         "clocks": clk,
         "wall_s_timed_region": wall,
@@ -536,11 +593,70 @@ def run_b200(args, wl, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+def run_swap(args, rank, world, local_rank):
+    """pa_swap_blocks throughput: every block of the Llama-3-8B layer batch swapped
+    out to a page-locked host pool, then back into the device pool."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    wl = make_workload("llama3_8b_layer", 16)
+    cache, seqs, host, dev, max_len, _ = build_on_gpu(wl, device)
+    tables = host["tables"].numpy()
+    ids = sorted({int(b) for i, s in enumerate(seqs)
+                  for b in tables[i, :cache.bm.seq_num_blocks(s)]})
+    n = len(ids)
+    shape = (n,) + tuple(cache.k_cache.shape[1:])
+    host_k = torch.empty(shape, dtype=cache.k_cache.dtype).pin_memory()
+    host_v = torch.empty(shape, dtype=cache.k_cache.dtype).pin_memory()
+    out_map = torch.tensor([[b, i] for i, b in enumerate(ids)], dtype=torch.int64, device=device)
+    in_map = out_map.flip(1).contiguous()
+    block_bytes = cache.k_cache[0].numel() * cache.k_cache.element_size()
+    moved = 2 * n * block_bytes
+    res = {}
+    for name, fn in (("device_to_host", lambda: pa.pa_swap_blocks(host_k, host_v, cache.k_cache,
+                                                                  cache.v_cache, out_map)),
+                     ("host_to_device", lambda: pa.pa_swap_blocks(cache.k_cache, cache.v_cache,
+                                                                  host_k, host_v, in_map))):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        ms = a.elapsed_time(b) / args.steps
+        res[name] = {"GB_per_s": moved / (ms * 1e-3) / 1e9, "us_per_call": 1e3 * ms}
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set during the swap benchmark")
+    if rank == 0:
+        print(json.dumps({
+            "metric": "pa_swap_blocks bytes moved per second (device <-> page-locked host)",
+            "value": min(r["GB_per_s"] for r in res.values()), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "swap: every block of the Llama-3-8B layer batch",
+                       "blocks": n, "bytes_per_call": moved},
+            "directions": res, "gpu_launches": 2 * args.steps}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     rank, world, local_rank = dist_env()
+    if args.workload == "swap":
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the oracle has no device/host memory to swap between"}))
+            return
+        run_swap(args, rank, world, local_rank)
+        return
     wl = make_workload(args.workload, args.block_size)
     if args.impl == "reference":
         run_reference(args, wl, rank)

@@ -107,6 +107,30 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, i
                    int num_blocks, int block_size, int num_kv_heads, int head_dim,
                    pa_dtype dtype, pa_stream_t stream);
 
+/*
+ * pa_swap_blocks — copy whole blocks between two pools, either of which may be
+ * device memory or page-locked host memory mapped for the device (e.g.
+ * cudaHostAlloc / cudaHostRegister; on unified-addressing systems the host
+ * pointer itself is used). For each pair: dst block := src block, K and V, bit
+ * for bit. This is the data movement of preemption by swapping: "Paged
+ * Attention" (klaylearn.com glossary), FAQ (move blocks to CPU memory); "What is
+ * paged attention in vLLM...", Follow-up questions (blocks swapped to CPU
+ * memory, later swapped back). Choosing between swapping and recomputing is
+ * the caller's policy.
+ *
+ *   dst_k_cache, dst_v_cache  [dst_num_blocks][block_size][num_kv_heads][head_dim]
+ *   src_k_cache, src_v_cache  [src_num_blocks][block_size][num_kv_heads][head_dim]
+ *   block_mapping  int64 [num_pairs][2] = (src id, dst id), readable by the
+ *                  device (device memory or mapped host memory). Destination
+ *                  ids must be distinct; an id outside its pool sets
+ *                  PA_DEVERR_COPY_PAIR and the pair is skipped.
+ * One launch for all pairs; asynchronous on `stream`.
+ */
+int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
+                   const void* src_k_cache, const void* src_v_cache, int src_num_blocks,
+                   const int64_t* block_mapping, int num_pairs, int block_size, int num_kv_heads,
+                   int head_dim, pa_dtype dtype, pa_stream_t stream);
+
 /* --------------------------------------------------------------- decode attention */
 
 /*

@@ -120,3 +120,17 @@ def copy_blocks(k_cache, v_cache, block_mapping):
         k_out[int(dst)] = k_out[int(src)]
         v_out[int(dst)] = v_out[int(src)]
     return k_out, v_out
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping):
+    """Copies of the destination pools with block dst := src-pool block src for
+    each (src, dst) pair: moving whole blocks between a device pool and a host
+    pool when a sequence is preempted and later resumed ("Paged Attention",
+    klaylearn.com glossary, FAQ; "What is paged attention in vLLM...",
+    Follow-up questions)."""
+    k_out = np.array(dst_k, copy=True)
+    v_out = np.array(dst_v, copy=True)
+    for src, dst in np.asarray(block_mapping).reshape(-1, 2).tolist():
+        k_out[int(dst)] = src_k[int(src)]
+        v_out[int(dst)] = src_v[int(src)]
+    return k_out, v_out

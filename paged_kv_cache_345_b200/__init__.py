@@ -9,6 +9,7 @@ has not been built (python paged_kv_cache_345_b200/build.py).
 Entry points (same names as the C ABI):
   pa_kv_append     write new tokens' K/V rows into their slots
   pa_copy_blocks   copy-on-write of shared blocks
+  pa_swap_blocks   copy blocks between device and (pinned) host pools
   pa_decode        paged decode attention (split-K over partitions)
   pa_decode_append one decode step: append each newest token, then attend
   BlockManager     host free list + reference counts + block tables
@@ -25,7 +26,8 @@ __all__ = [
     "PagedAttentionError", "PA_OK", "PA_ERR_INVALID", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_NO_BLOCKS", "PA_ERR_DEVICE_CHECK", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID",
     "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
-    "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_decode", "pa_decode_append",
+    "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode",
+    "pa_decode_append",
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
 ]
@@ -58,6 +60,7 @@ def _sig(name, restype, *argtypes):
 
 _sig("pa_kv_append", _i32, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
+_sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
@@ -93,7 +96,7 @@ _sig("pa_bm_append_slots", _i32, _vp, _i32p, _i32p, _i32, _i64p, _i64p, _i32,
 _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 
 EXPORTED = (
-    "pa_kv_append", "pa_copy_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
+    "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_append", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
@@ -175,6 +178,38 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", k_cache.dtype),
         _dev_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], nb, bs,
         hkv, d, _dtype_code(k_cache), _stream(stream, k_cache.device)))
+
+
+def _mapped_ptr(t, name, dtype=None):
+    """Pointer of a CUDA tensor, or of a page-locked CPU tensor (used by the
+    device through unified addressing)."""
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError(f"{name} must be a CUDA tensor or page-locked (pinned) host memory")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None) -> None:
+    """dst block := src block for each (src, dst) row of block_mapping [n, 2] (int64).
+    Pools are [num_blocks, bs, Hkv, d], each on the device or in pinned host memory."""
+    torch = _torch()
+    snb, bs, hkv, d = src_k.shape
+    dnb = dst_k.shape[0]
+    if tuple(dst_k.shape[1:]) != (bs, hkv, d) or dst_v.shape != dst_k.shape or \
+            src_v.shape != src_k.shape or dst_k.dtype != src_k.dtype:
+        raise ValueError("pool shape / dtype mismatch")
+    if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be [num_pairs, 2]")
+    dt = src_k.dtype
+    dev = dst_k.device if dst_k.is_cuda else (src_k.device if src_k.is_cuda else None)
+    _check(_lib.pa_swap_blocks(
+        _mapped_ptr(dst_k, "dst_k", dt), _mapped_ptr(dst_v, "dst_v", dt), dnb,
+        _mapped_ptr(src_k, "src_k", dt), _mapped_ptr(src_v, "src_v", dt), snb,
+        _mapped_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], bs, hkv,
+        d, _dtype_code(src_k), _stream(stream, dev)))
 
 
 def pa_decode_partition_size(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:

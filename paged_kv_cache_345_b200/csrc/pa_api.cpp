@@ -126,6 +126,32 @@ int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, i
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_copy_blocks launch", e);
 }
 
+int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
+                   const void* src_k_cache, const void* src_v_cache, int src_num_blocks,
+                   const int64_t* block_mapping, int num_pairs, int block_size, int num_kv_heads,
+                   int head_dim, pa_dtype dtype, pa_stream_t stream) {
+  if (num_pairs < 0) return pa_fail(PA_ERR_INVALID, "pa_swap_blocks: num_pairs < 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !block_mapping)
+    return pa_fail(PA_ERR_INVALID, "pa_swap_blocks: null pointer");
+  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_swap_blocks: dtype %d", dtype);
+  if (dst_num_blocks <= 0 || src_num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 ||
+      head_dim <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_swap_blocks: sizes must be positive");
+  if (num_pairs > 2147483647 / 2) return pa_fail(PA_ERR_INVALID, "pa_swap_blocks: too many pairs");
+  const int64_t block_bytes =
+      static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes(dtype);
+  if (block_bytes % 16 != 0)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_swap_blocks: block bytes not a multiple of 16");
+  if (!aligned(dst_k_cache, 16) || !aligned(dst_v_cache, 16) || !aligned(src_k_cache, 16) ||
+      !aligned(src_v_cache, 16) || !aligned(block_mapping, 8))
+    return pa_fail(PA_ERR_INVALID, "pa_swap_blocks: misaligned pointer");
+  cudaError_t e = pa::launch_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache,
+                                         block_mapping, num_pairs, src_num_blocks, dst_num_blocks,
+                                         block_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_swap_blocks launch", e);
+}
+
 int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
   // The bf16 kernel runs one CTA per (group of up to 4 KV heads, partition,
   // sequence), two per SM. Aim for about three CTAs per SM if every sequence

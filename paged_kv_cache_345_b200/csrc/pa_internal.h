@@ -42,6 +42,9 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
                                int num_pairs, int num_blocks, int64_t block_bytes,
                                cudaStream_t stream);
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* block_mapping, int num_pairs, int src_num_blocks,
+                               int dst_num_blocks, int64_t block_bytes, cudaStream_t stream);
 // Returns cudaErrorNotSupported when no kernel is built for the shape.
 // k_new / v_new non-null: fused append of each sequence's newest token.
 cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,

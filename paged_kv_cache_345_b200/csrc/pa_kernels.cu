@@ -149,6 +149,52 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* bloc
                     num_blocks, vec, err);
 }
 
+// -------------------------------------------------------------- swap blocks
+
+// Copies whole blocks between two pools (device memory or page-locked host
+// memory mapped into the device's address space): blockIdx.x = pair,
+// blockIdx.y = slice of the block. Plain (coherent) loads, since one side may
+// be host memory reached over the bus.
+__global__ void __launch_bounds__(256)
+    swap_blocks_kernel(uint4* dst_k, uint4* dst_v, const uint4* src_k, const uint4* src_v,
+                       const int64_t* block_mapping, int src_num_blocks, int dst_num_blocks,
+                       int64_t vec_per_block, unsigned* err) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t src = block_mapping[2 * blockIdx.x];
+  const int64_t dst = block_mapping[2 * blockIdx.x + 1];
+  if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(err, PA_DEVERR_COPY_PAIR);
+    return;
+  }
+  const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x; v < vec_per_block;
+       v += stride) {
+    const uint4 a = src_k[src * vec_per_block + v];
+    const uint4 b = src_v[src * vec_per_block + v];
+    dst_k[dst * vec_per_block + v] = a;
+    dst_v[dst * vec_per_block + v] = b;
+  }
+}
+
+cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* block_mapping, int num_pairs, int src_num_blocks,
+                               int dst_num_blocks, int64_t block_bytes, cudaStream_t stream) {
+  unsigned* err = nullptr;
+  cudaError_t e = device_error_word(&err);
+  if (e != cudaSuccess) return e;
+  const int64_t vec = block_bytes / 16;
+  const int threads = 256;
+  int64_t slices = (vec + threads * 4 - 1) / (threads * 4);
+  if (slices < 1) slices = 1;
+  if (slices > 65535) slices = 65535;
+  dim3 grid(num_pairs, static_cast<unsigned>(slices));
+  return launch_pdl(swap_blocks_kernel, grid, dim3(threads), 0, stream,
+                    static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v),
+                    static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v),
+                    block_mapping, src_num_blocks, dst_num_blocks, vec, err);
+}
+
 // ------------------------------------------------------------------ decode
 
 namespace {

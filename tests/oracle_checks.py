@@ -351,6 +351,44 @@ def check_append_and_copy_roundtrip():
         assert np.array_equal(k3[b], k2[b]) and np.array_equal(v3[b], v2[b])
 
 
+def check_swap_roundtrip():
+    """Swapping blocks out to another pool and back restores them exactly and
+    touches nothing else."""
+    rng = np.random.default_rng(13)
+    dev_k = rng.standard_normal((6, 4, 2, 3))
+    dev_v = rng.standard_normal((6, 4, 2, 3))
+    host_k = np.zeros((4, 4, 2, 3))
+    host_v = np.zeros((4, 4, 2, 3))
+    out_pairs = np.array([[5, 0], [1, 3], [2, 1]])
+    hk, hv = oatt.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs)
+    assert np.array_equal(hk[0], dev_k[5]) and np.array_equal(hv[3], dev_v[1])
+    assert np.array_equal(hk[2], host_k[2])
+    back_k, back_v = oatt.swap_blocks(np.zeros_like(dev_k), np.zeros_like(dev_v), hk, hv,
+                                      out_pairs[:, ::-1])
+    for src, _ in out_pairs:
+        assert np.array_equal(back_k[src], dev_k[src]) and np.array_equal(back_v[src], dev_v[src])
+    assert not back_k[0].any() and not back_v[4].any()
+
+
+def check_swap_roundtrip():
+    """Swapping blocks out to another pool and back restores them exactly and
+    touches nothing else."""
+    rng = np.random.default_rng(13)
+    dev_k = rng.standard_normal((6, 4, 2, 3))
+    dev_v = rng.standard_normal((6, 4, 2, 3))
+    host_k = np.zeros((4, 4, 2, 3))
+    host_v = np.zeros((4, 4, 2, 3))
+    out_pairs = np.array([[5, 0], [1, 3], [2, 1]])
+    hk, hv = oatt.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs)
+    assert np.array_equal(hk[0], dev_k[5]) and np.array_equal(hv[3], dev_v[1])
+    assert np.array_equal(hk[2], host_k[2])
+    back_k, back_v = oatt.swap_blocks(np.zeros_like(dev_k), np.zeros_like(dev_v), hk, hv,
+                                      out_pairs[:, ::-1])
+    for src, _ in out_pairs:
+        assert np.array_equal(back_k[src], dev_k[src]) and np.array_equal(back_v[src], dev_v[src])
+    assert not back_k[0].any() and not back_v[4].any()
+
+
 BLOCK_CHECKS = [
     check_seven_token_prompt, check_600_tokens, check_llama3_per_token, check_700_tokens,
     check_worked_example, check_capacity, check_worked_example_block_manager,
@@ -359,6 +397,7 @@ PLAIN_BLOCK_CHECKS = [check_sharing_and_copy_on_write, check_exhaustion_leaves_s
 ATTENTION_CHECKS = [
     check_brute_force_tiny, check_sdpa_identity_table, check_closed_forms,
     check_placement_and_sharing_invariance, check_append_and_copy_roundtrip,
+    check_swap_roundtrip,
 ]
 
 assert oracle is not None

@@ -104,3 +104,47 @@ def test_copy_then_diverge_keeps_sharers_apart():
     assert torch.equal(c.k_cache[own_tail, :2], before[shared_tail, :2])
     assert torch.equal(c.k_cache[own_tail, 2], new[0])
     assert int(slots[0]) == own_tail * 4 + 2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mapping_on_host", [False, True])
+def test_swap_out_to_pinned_host_and_back_bit_exact(dtype, mapping_on_host):
+    """Preemption by swapping: blocks go from the device pool to a page-locked
+    host pool and come back to other device blocks, bit for bit."""
+    rng = np.random.default_rng(21)
+    nb, hb, bs, hkv, d = 64, 40, 16, 8, 128
+    k_cache, v_cache = _random_cache(rng, nb, bs, hkv, d, dtype)
+    kd, vd = k_cache.cuda(), v_cache.cuda()
+    host_k = torch.zeros((hb, bs, hkv, d), dtype=DT[dtype]).pin_memory()
+    host_v = torch.zeros((hb, bs, hkv, d), dtype=DT[dtype]).pin_memory()
+    ids = rng.permutation(nb)[:30]
+    out_pairs = np.stack([ids, rng.permutation(hb)[:30]], axis=1).astype(np.int64)
+    mapping = torch.from_numpy(out_pairs)
+    mapping = mapping.pin_memory() if mapping_on_host else mapping.cuda()
+    pa.pa_swap_blocks(host_k, host_v, kd, vd, mapping)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    ref_k, ref_v = oatt.swap_blocks(_bits(torch.zeros_like(host_k)), _bits(torch.zeros_like(host_v)),
+                                    _bits(k_cache), _bits(v_cache), out_pairs)
+    assert np.array_equal(_bits(host_k), ref_k) and np.array_equal(_bits(host_v), ref_v)
+    # swap back into a fresh device pool at other block ids
+    kd2 = torch.zeros_like(kd)
+    vd2 = torch.zeros_like(vd)
+    in_pairs = np.stack([out_pairs[:, 1], rng.permutation(nb)[:30]], axis=1).astype(np.int64)
+    pa.pa_swap_blocks(kd2, vd2, host_k, host_v, torch.from_numpy(in_pairs).cuda())
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    for (src_dev, _), (_, dst_dev) in zip(out_pairs, in_pairs):
+        assert torch.equal(kd2[dst_dev].cpu(), k_cache[src_dev])
+        assert torch.equal(vd2[dst_dev].cpu(), v_cache[src_dev])
+
+
+def test_swap_bad_pair_is_flagged_and_skipped():
+    kd = torch.ones((4, 4, 2, 64), dtype=torch.bfloat16, device="cuda")
+    host = torch.zeros((4, 4, 2, 64), dtype=torch.bfloat16).pin_memory()
+    host_v = torch.zeros_like(host).pin_memory()
+    pairs = torch.tensor([[0, 1], [9, 2], [1, -1]], dtype=torch.int64, device="cuda")
+    pa.pa_swap_blocks(host, host_v, kd, kd, pairs)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() & pa.PA_DEVERR_COPY_PAIR
+    assert bool((host[1] == 1).all()) and not bool(host[2].any()) and not bool(host[0].any())

@@ -54,6 +54,14 @@ def _softmax_drop_last(q_vec, keys, values, scale):
     return (w / w.sum()) @ values
 
 
+def _swap_wrong_index(dk, dv, sk, sv, mapping):
+    k, v = np.array(dk, copy=True), np.array(dv, copy=True)
+    for src, dst in np.asarray(mapping).reshape(-1, 2).tolist():
+        k[int(src) % len(k)] = sk[int(src)]
+        v[int(src) % len(v)] = sv[int(src)]
+    return k, v
+
+
 MUTANTS = {
     "gqa_heads_interleaved": (oatt, "kv_head_of", lambda j, g: j % g),
     "gqa_always_head0": (oatt, "kv_head_of", lambda j, g: 0),
@@ -66,6 +74,8 @@ MUTANTS = {
     "softmax_not_normalised": (oatt, "softmax_attention", _softmax_unnormalised),
     "keys_used_as_values": (oatt, "softmax_attention", _softmax_keys_as_values),
     "last_token_dropped": (oatt, "softmax_attention", _softmax_drop_last),
+    "swap_writes_source_index": (oatt, "swap_blocks", lambda dk, dv, sk, sv, m: (
+        _swap_wrong_index(dk, dv, sk, sv, m))),
     "slot_without_block_size": (oblk, "slot_of",
                                 lambda table, t, bs: int(table[t // bs]) + t % bs),
 }
