@@ -566,6 +566,7 @@ def run_b200(args, wl, rank, world, local_rank):
                    "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
                    "partition_size": calls.partition_size,
                    "num_partitions": calls.num_partitions, "copy_on_write_pairs": cow_pairs,
+                   "placement": args.placement,
                    "l2": f"flushed between steps ({flush_w.numel() >> 20} MiB written, then "
                          f"{(flush_r.numel() * 4) >> 20} MiB of another buffer read; outside the "
                          "timed events)",
