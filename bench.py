@@ -90,6 +90,28 @@ def kv_bytes(wl) -> int:
     return sum(n + 1 for n in wl.context_lens) * wl.num_kv_heads * 2 * wl.head_dim * wl.elem_bytes
 
 
+# ------------------------------------------------------------- rank plumbing
+
+def max_over_ranks(value_ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank contributes its own measured time and
+    all get the max (NCCL on GPUs, gloo on CPU). One rank: the value itself."""
+    if world <= 1:
+        return float(value_ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value_ms)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step: float, steps: int, world: int, time_ms: float) -> float:
+    """Units per second of the whole job: every rank runs its own replica of the
+    step, so the job does world x steps x units in the slowest rank's time."""
+    return units_per_step * steps * world / (time_ms * 1e-3)
+
+
 # ------------------------------------------------------------------ GPU setup
 
 def build_on_gpu(wl, device, placement="random"):
@@ -444,11 +466,7 @@ def run_b200(args, wl, rank, world, local_rank):
     clk = clocks.stop()
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
     decode_ms = step_ms  # the step's kernels: (append +) decode + split-K merge
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, device)
     if pa.pa_device_errors() != 0:
         raise RuntimeError("device error word set during the timed steps")
 
@@ -477,12 +495,9 @@ def run_b200(args, wl, rank, world, local_rank):
             e2e_step()
             ee[i][1].record(stream)
         barrier()
-        e2e_ms = sum(ee[i][0].elapsed_time(ee[i][1]) for i in range(args.steps))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": bytes_step * args.steps * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = max_over_ranks(sum(ee[i][0].elapsed_time(ee[i][1]) for i in range(args.steps)),
+                                world, device)
+        e2e = {"value": whole_job_rate(bytes_step, args.steps, world, e2e_ms) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.steps}
 
@@ -555,7 +570,7 @@ def run_b200(args, wl, rank, world, local_rank):
             cpu = {"value": None, "unit": "GB/s", "cores": 0, "kind": "oracle",
                    "sample": f"not run: {exc}"}
 
-    value = bytes_step * args.steps * world / (total_ms * 1e-3) / 1e9
+    value = whole_job_rate(bytes_step, args.steps, world, total_ms) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -571,7 +586,7 @@ def run_b200(args, wl, rank, world, local_rank):
                          f"{(flush_r.numel() * 4) >> 20} MiB of another buffer read; outside the "
                          "timed events)",
                    "parallelism": f"replicas x{world}"},
-        "attended_tokens_per_s": tokens_step * args.steps * world / (total_ms * 1e-3),
+        "attended_tokens_per_s": whole_job_rate(tokens_step, args.steps, world, total_ms),
         "us_per_step": 1e3 * total_ms / args.steps,
         "step_us_p10_p50_p90": [1e3 * float(np.percentile(decode_ms, p)) for p in (10, 50, 90)],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
