@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import json
 import os
 import statistics
@@ -52,6 +53,8 @@ def parse_args():
                     help="physical block order: a seeded permutation (default) or identity "
                          "(each sequence's blocks contiguous in memory)")
     ap.add_argument("--block-size", type=int, default=16, help="long_context only")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8_e4m3"], default="bf16",
+                    help="cache element type (fp8_e4m3: 8-bit codes, per-KV-head scales)")
     ap.add_argument("--partition-size", type=int, default=-1,
                     help="tokens per split-K partition (-1: tuned default, 0: library choice)")
     ap.add_argument("--unfused", action="store_true",
@@ -87,7 +90,8 @@ TUNED_PARTITION = {"llama3_8b_layer": 0, "large_batch": 0, "shared_prefix": 0,
 
 def kv_bytes(wl) -> int:
     """K and V bytes the decode step reads: every attended token, every KV head."""
-    return sum(n + 1 for n in wl.context_lens) * wl.num_kv_heads * 2 * wl.head_dim * wl.elem_bytes
+    return (sum(n + 1 for n in wl.context_lens) * wl.num_kv_heads * 2 * wl.head_dim *
+            wl.cache_elem_bytes)
 
 
 # ------------------------------------------------------------- rank plumbing
@@ -126,8 +130,12 @@ def build_on_gpu(wl, device, placement="random"):
     max_blocks = max(-(-(n + 1) // bs) for n in wl.context_lens)
     order = synth.block_permutation(wl.num_blocks, wl.placement_seed) if placement == "random" \
         else np.arange(wl.num_blocks, dtype=np.int32)
-    cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.dtype, device,
-                         max_blocks_per_seq=max_blocks, free_order=order)
+    fp8 = wl.cache_dtype == "fp8_e4m3"
+    ks, vs = synth.e4m3_scales(wl.num_kv_heads) if fp8 else (None, None)
+    cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.cache_dtype, device,
+                         max_blocks_per_seq=max_blocks, free_order=order,
+                         k_scale=None if ks is None else torch.from_numpy(ks),
+                         v_scale=None if vs is None else torch.from_numpy(vs))
     ghosts = [cache.add_sequence() for _ in wl.ghost_lens]
     if ghosts:
         cache.bm.append_slots(ghosts, list(wl.ghost_lens))
@@ -157,8 +165,13 @@ def build_on_gpu(wl, device, placement="random"):
             if len(cows):
                 from paged_kv_cache_345_b200 import pa_copy_blocks
                 pa_copy_blocks(cache.k_cache, cache.v_cache, torch.from_numpy(cows).to(device))
-            from paged_kv_cache_345_b200 import pa_kv_append
-            pa_kv_append(k, v, torch.from_numpy(slots).to(device), cache.k_cache, cache.v_cache)
+            from paged_kv_cache_345_b200 import pa_kv_append, pa_kv_append_fp8
+            sd = torch.from_numpy(slots).to(device)
+            if fp8:
+                pa_kv_append_fp8(k, v, sd, cache.k_cache, cache.v_cache, cache.k_scale,
+                                 cache.v_scale)
+            else:
+                pa_kv_append(k, v, sd, cache.k_cache, cache.v_cache)
     torch.cuda.synchronize(device)
 
     # the decode step: one new token per sequence, appended then attended
@@ -193,6 +206,7 @@ class StepCalls:
         self.lib = pa._lib
         s, hq, d = dev["q"].shape
         nb, bs, hkv, _ = cache.k_cache.shape
+        self.fp8 = cache.k_cache.dtype == torch.uint8
         dt = pa.PA_BF16 if cache.k_cache.dtype == torch.bfloat16 else pa.PA_F32
         self.partition_size = partition_size or pa.pa_decode_partition_size(s, hkv, max_len)
         ws_bytes = pa.pa_decode_workspace_bytes(s, hq, hkv, d, max_len, self.partition_size)
@@ -201,37 +215,52 @@ class StepCalls:
         self.num_partitions = -(-max_len // self.partition_size)
         st = ctypes.c_void_p(stream.cuda_stream)
         p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-        self.append_args = (p(dev["k_new"]), p(dev["v_new"]), p(dev["slots"]), s,
-                            p(cache.k_cache), p(cache.v_cache), nb, bs, hkv, d, dt, st)
-        self.decode_args = (p(self.out), p(dev["q"]), p(cache.k_cache), p(cache.v_cache),
-                            p(dev["tables"]), p(dev["lens"]), s, hq, hkv, d, bs, nb,
-                            dev["tables"].shape[1], max_len, scale, self.partition_size,
-                            p(self.workspace), self.workspace.numel(), dt, st)
-        self.step_args = (p(self.out), p(dev["q"]), p(dev["k_new"]), p(dev["v_new"]),
-                          p(cache.k_cache), p(cache.v_cache), p(dev["tables"]), p(dev["lens"]),
-                          s, hq, hkv, d, bs, nb, dev["tables"].shape[1], max_len, scale,
-                          self.partition_size, p(self.workspace), self.workspace.numel(), dt, st)
+        ws = (p(self.workspace), self.workspace.numel())
+        mbps = dev["tables"].shape[1]
+        if self.fp8:
+            sc = (p(cache.k_scale), p(cache.v_scale))
+            self.append_args = (p(dev["k_new"]), p(dev["v_new"]), p(dev["slots"]), s,
+                                p(cache.k_cache), p(cache.v_cache), *sc, nb, bs, hkv, d, st)
+            self.decode_args = (p(self.out), p(dev["q"]), p(cache.k_cache), p(cache.v_cache),
+                                *sc, p(dev["tables"]), p(dev["lens"]), s, hq, hkv, d, bs, nb,
+                                mbps, max_len, scale, self.partition_size, *ws, st)
+            self.step_args = (p(self.out), p(dev["q"]), p(dev["k_new"]), p(dev["v_new"]),
+                              p(cache.k_cache), p(cache.v_cache), *sc, p(dev["tables"]),
+                              p(dev["lens"]), s, hq, hkv, d, bs, nb, mbps, max_len, scale,
+                              self.partition_size, *ws, st)
+            self.fns = (self.lib.pa_kv_append_fp8, self.lib.pa_decode_fp8,
+                        self.lib.pa_decode_append_fp8)
+        else:
+            self.append_args = (p(dev["k_new"]), p(dev["v_new"]), p(dev["slots"]), s,
+                                p(cache.k_cache), p(cache.v_cache), nb, bs, hkv, d, dt, st)
+            self.decode_args = (p(self.out), p(dev["q"]), p(cache.k_cache), p(cache.v_cache),
+                                p(dev["tables"]), p(dev["lens"]), s, hq, hkv, d, bs, nb,
+                                mbps, max_len, scale, self.partition_size, *ws, dt, st)
+            self.step_args = (p(self.out), p(dev["q"]), p(dev["k_new"]), p(dev["v_new"]),
+                              p(cache.k_cache), p(cache.v_cache), p(dev["tables"]),
+                              p(dev["lens"]), s, hq, hkv, d, bs, nb, mbps, max_len, scale,
+                              self.partition_size, *ws, dt, st)
+            self.fns = (self.lib.pa_kv_append, self.lib.pa_decode, self.lib.pa_decode_append)
         self.fused = fused
         self.launches_per_step = (1 if fused else 2) + (1 if self.num_partitions > 1 else 0)
 
-    def append(self):
-        st = self.lib.pa_kv_append(*self.append_args)
+    def _call(self, fn, args):
+        st = fn(*args)
         if st:
-            raise RuntimeError(f"pa_kv_append: {self.lib.pa_last_error().decode()}")
+            raise RuntimeError(f"{fn.__name__}: {self.lib.pa_last_error().decode()}")
+
+    def append(self):
+        self._call(self.fns[0], self.append_args)
 
     def decode(self):
-        st = self.lib.pa_decode(*self.decode_args)
-        if st:
-            raise RuntimeError(f"pa_decode: {self.lib.pa_last_error().decode()}")
+        self._call(self.fns[1], self.decode_args)
 
     def step(self):
         if not self.fused:
             self.append()
             self.decode()
             return
-        st = self.lib.pa_decode_append(*self.step_args)
-        if st:
-            raise RuntimeError(f"pa_decode_append: {self.lib.pa_last_error().decode()}")
+        self._call(self.fns[2], self.step_args)
 
 
 # --------------------------------------------------------------------- clocks
@@ -296,6 +325,15 @@ def oracle_inputs(wl):
     def stored(x):
         return synth.round_to_bf16(x) if wl.dtype == "bf16" else x
 
+    fp8 = wl.cache_dtype == "fp8_e4m3"
+    if fp8:
+        from oracle import quant as oquant
+        ks, vs = synth.e4m3_scales(wl.num_kv_heads)
+
+        def cache_values(rows, scales):   # the oracle's codes of the rows, dequantised
+            return np.stack([oquant.dequantize(oquant.quantize(rows[:, h], scales[h]), scales[h])
+                             for h in range(rows.shape[1])], axis=1)
+
     ob = oblk.BlockManager(wl.num_blocks, wl.block_size)
     ob.set_free_order(synth.block_permutation(wl.num_blocks, wl.placement_seed).tolist())
     kc = np.zeros((wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim))
@@ -308,6 +346,8 @@ def oracle_inputs(wl):
         k, v = synth.kv_rows(wl.value_seed, s, n, wl.num_kv_heads, wl.head_dim)
         k = np.concatenate([stored(k), stored(new_k[s:s + 1])])
         v = np.concatenate([stored(v), stored(new_v[s:s + 1])])
+        if fp8:
+            k, v = cache_values(k, ks), cache_values(v, vs)
         slots, _ = ob.add_tokens(sid, n + 1)
         kc, vc = oatt.kv_append(kc, vc, k, v, slots, wl.block_size)
     mb = max(len(ob.tables[s]) for s in seqs)
@@ -517,6 +557,8 @@ def run_b200(args, wl, rank, world, local_rank):
         for kc, vc in reps:
             view = type("CacheView", (), {})()
             view.k_cache, view.v_cache = kc, vc
+            if calls.fp8:
+                view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
             layer_calls.append(StepCalls(view, dev, max_len, wl.scale, calls.partition_size,
                                          stream, fused=calls.fused))
         for c in layer_calls:   # warm-up, eager
@@ -555,7 +597,7 @@ def run_b200(args, wl, rank, world, local_rank):
         b2b["frac_of_peak"] = b2b["kv_GB_per_s"] / peak
     dec_s = statistics.mean(decode_ms) * 1e-3
     achieved = bytes_step / dec_s / 1e9
-    traffic = load_traffic(f"pa_decode_{wl.name}")
+    traffic = load_traffic(f"pa_decode_{wl.name}" + ("_fp8" if calls.fp8 else ""))
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
     cpu = None
@@ -574,14 +616,14 @@ def run_b200(args, wl, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.cache_dtype, "data": "synthetic",
         "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "block_size": wl.block_size, "num_blocks": wl.num_blocks,
                    "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
                    "partition_size": calls.partition_size,
                    "num_partitions": calls.num_partitions, "copy_on_write_pairs": cow_pairs,
-                   "placement": args.placement,
+                   "placement": args.placement, "kv_cache": wl.cache_dtype,
                    "l2": f"flushed between steps ({flush_w.numel() >> 20} MiB written, then "
                          f"{(flush_r.numel() * 4) >> 20} MiB of another buffer read; outside the "
                          "timed events)",
@@ -674,6 +716,8 @@ def main():
         run_swap(args, rank, world, local_rank)
         return
     wl = make_workload(args.workload, args.block_size)
+    if args.kv_dtype != "bf16":
+        wl = dataclasses.replace(wl, kv_dtype=args.kv_dtype)
     if args.impl == "reference":
         run_reference(args, wl, rank)
         return

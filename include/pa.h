@@ -56,7 +56,18 @@ typedef enum {
   PA_ERR_DEVICE_CHECK = 5  /* a kernel found a bad device-side index              */
 } pa_status;
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+/*
+ * Element types of a cache. PA_FP8_E4M3: 8-bit E4M3 codes (1 sign, 4 exponent
+ * bits with bias 7, 3 mantissa bits, largest finite value 448) with one float32
+ * scale per KV head: cache value = decode(code) * scale[head]. "What is paged
+ * attention in vLLM, and why does it matter?" (interview.clozo.ai), "Trade-offs
+ * and edge cases", fourth point: narrower cache values shrink every block. The
+ * pages stop at 16-bit formats; the 8-bit format and its per-head scale are
+ * this library's extension. pa_copy_blocks and pa_swap_blocks take
+ * PA_FP8_E4M3 as a 1-byte element; writes and decode go through the _fp8
+ * entry points below.
+ */
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 /* Bits of the device error word (pa_device_errors). */
 #define PA_DEVERR_SLOT 0x1u       /* pa_kv_append: slot >= num_blocks * block_size       */
@@ -82,6 +93,7 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
  *                  distinct; slot >= num_blocks * block_size sets
  *                  PA_DEVERR_SLOT and skips the row.
  *   k_cache, v_cache  device, written in place.
+ * dtype PA_F32 or PA_BF16 (PA_FP8_E4M3 caches: pa_kv_append_fp8).
  * Rows are copied bit for bit. num_tokens == 0 is a no-op. Prefill and decode
  * use the same call (num_tokens = prompt tokens, or one per sequence).
  * Requires num_kv_heads * head_dim * element size to be a multiple of 16.
@@ -89,6 +101,23 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
 int pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
                  int num_tokens, void* k_cache, void* v_cache, int num_blocks, int block_size,
                  int num_kv_heads, int head_dim, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_kv_append_fp8 — pa_kv_append into an E4M3 cache (PA_FP8_E4M3): each
+ * bfloat16 value x of head h is stored as the E4M3 code of x / scale[h]
+ * (float32 division, round to nearest, then round to nearest even into E4M3;
+ * finite values beyond +-448 saturate to +-448, NaN stays NaN).
+ *
+ *   k_new, v_new   device, bfloat16 [num_tokens][num_kv_heads][head_dim].
+ *   k_scale, v_scale  device, float32 [num_kv_heads], positive and finite.
+ *   k_cache, v_cache  device, uint8 codes [num_blocks][block_size][num_kv_heads][head_dim].
+ * slot_mapping, padding and error behaviour as pa_kv_append. Requires
+ * num_kv_heads * head_dim to be a multiple of 16 and head_dim a multiple of 16.
+ */
+int pa_kv_append_fp8(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                     int num_tokens, void* k_cache, void* v_cache, const float* k_scale,
+                     const float* v_scale, int num_blocks, int block_size, int num_kv_heads,
+                     int head_dim, pa_stream_t stream);
 
 /*
  * pa_copy_blocks — copy-on-write of shared blocks: for each pair,
@@ -218,6 +247,46 @@ int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_
                      int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                      int max_context_len, float scale, int partition_size, void* workspace,
                      size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_decode_fp8 — pa_decode over E4M3 caches: K_s[t][h] and V_s[t][h] are the
+ * dequantised rows decode(code) * k_scale[h] and decode(code) * v_scale[h]
+ * (see PA_FP8_E4M3); the attention arithmetic is pa_decode's.
+ *
+ *   out, q         device, bfloat16 [num_seqs][num_heads][head_dim].
+ *   k_cache, v_cache  device, uint8 E4M3 codes, read only.
+ *   k_scale, v_scale  device, float32 [num_kv_heads].
+ * Products use float16 operands: E4M3 codes widen to float16 exactly, q is
+ * converted from bfloat16 to float16 (exact for magnitudes in [2^-14, 65504];
+ * smaller magnitudes lose low bits, larger ones overflow), softmax
+ * probabilities are rounded to float16; accumulation is float32.
+ * Supported: head_dim 128; num_heads / num_kv_heads in {1, 2, 4, 8};
+ * block_size a power of two in [1, 256]. Everything else as pa_decode,
+ * including the workspace (pa_decode_workspace_bytes) and the independence of
+ * the result from block_size and placement.
+ */
+int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                  const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                  int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                  int max_context_len, float scale, int partition_size, void* workspace,
+                  size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_decode_append_fp8 — pa_decode_append over E4M3 caches: each sequence's
+ * newest token (k_new / v_new, bfloat16 [num_seqs][num_kv_heads][head_dim]) is
+ * quantised exactly as pa_kv_append_fp8 does and written at position
+ * context_lens[s] - 1 through the block table, then the step attends as
+ * pa_decode_fp8. Conditions on the newest token's block as pa_decode_append.
+ */
+int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void* v_new,
+                         void* k_cache, void* v_cache, const float* k_scale,
+                         const float* v_scale, const int32_t* block_tables,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                         int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void* workspace, size_t workspace_bytes,
+                         pa_stream_t stream);
 
 /*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.

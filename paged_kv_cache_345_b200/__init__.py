@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
   pa_swap_blocks   copy blocks between device and (pinned) host pools
   pa_decode        paged decode attention (split-K over partitions)
   pa_decode_append one decode step: append each newest token, then attend
+  pa_kv_append_fp8, pa_decode_fp8, pa_decode_append_fp8
+                   the same over 8-bit E4M3 caches with per-KV-head scales
   BlockManager     host free list + reference counts + block tables
 """
 
@@ -27,14 +29,14 @@ __all__ = [
     "PA_ERR_NO_BLOCKS", "PA_ERR_DEVICE_CHECK", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID",
     "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
     "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode",
-    "pa_decode_append",
+    "pa_decode_append", "pa_kv_append_fp8", "pa_decode_fp8", "pa_decode_append_fp8", "PA_FP8_E4M3",
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
     range(6)
-PA_F32, PA_BF16 = 0, 1
+PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
 
@@ -59,6 +61,7 @@ def _sig(name, restype, *argtypes):
 
 
 _sig("pa_kv_append", _i32, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
+_sig("pa_kv_append_fp8", _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
@@ -67,6 +70,10 @@ _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i
      _i32, _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_decode_append", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _i32, _f32, _i32, _vp, _sz, _i32, _vp)
+_sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
+_sig("pa_decode_append_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _f32, _i32, _i32, _vp)
 _sig("pa_decode_noalloc_scratch_bytes", _sz)
@@ -96,8 +103,9 @@ _sig("pa_bm_append_slots", _i32, _vp, _i32p, _i32p, _i32, _i64p, _i64p, _i32,
 _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 
 EXPORTED = (
-    "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode_partition_size", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_decode_append", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
+    "pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_swap_blocks",
+    "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode", "pa_decode_append",
+    "pa_decode_fp8", "pa_decode_append_fp8", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
     "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
@@ -131,7 +139,14 @@ def _dtype_code(t) -> int:
         return PA_BF16
     if t.dtype == torch.float32:
         return PA_F32
-    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PA_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype} (float32, bfloat16, or uint8 E4M3 codes)")
+
+
+def _is_fp8(t) -> bool:
+    torch = _torch()
+    return t.dtype in (torch.uint8, torch.float8_e4m3fn)
 
 
 def _dev_ptr(t, name, dtype=None):
@@ -166,6 +181,29 @@ def pa_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> N
         _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", dt), nb, bs, hkv, d,
         _dtype_code(k_cache), _stream(stream, k_cache.device)))
+
+
+def pa_kv_append_fp8(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale,
+                     stream=None) -> None:
+    """Quantising append into E4M3 caches (uint8 codes [nb, bs, Hkv, d]): row i of
+    k_new/v_new (bfloat16 [N, Hkv, d]) goes to flat slot slot_mapping[i] as the codes
+    of value / scale[head]; k_scale/v_scale are float32 [Hkv] device tensors."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    if tuple(k_new.shape[1:]) != (hkv, d) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be [N, num_kv_heads, head_dim] matching the cache")
+    if v_cache.shape != k_cache.shape or slot_mapping.shape != (k_new.shape[0],):
+        raise ValueError("cache or slot_mapping shape mismatch")
+    if not (_is_fp8(k_cache) and _is_fp8(v_cache)):
+        raise TypeError("caches must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    if k_scale.shape != (hkv,) or v_scale.shape != (hkv,):
+        raise ValueError("k_scale/v_scale must be [num_kv_heads]")
+    _check(_lib.pa_kv_append_fp8(
+        _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
+        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(k_scale, "k_scale", torch.float32), _dev_ptr(v_scale, "v_scale", torch.float32),
+        nb, bs, hkv, d, _stream(stream, k_cache.device)))
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
@@ -276,6 +314,66 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, conte
         _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
         block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,
         ws_bytes, _dtype_code(k_cache), _stream(stream, q.device)))
+
+
+def _fp8_decode_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                     workspace):
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    s, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if not (_is_fp8(k_cache) and _is_fp8(v_cache)):
+        raise TypeError("caches must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    if k_scale.shape != (hkv,) or v_scale.shape != (hkv,):
+        raise ValueError("k_scale/v_scale must be [num_kv_heads]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    return dict(
+        k_cache=_dev_ptr(k_cache, "k_cache"), v_cache=_dev_ptr(v_cache, "v_cache"),
+        k_scale=_dev_ptr(k_scale, "k_scale", torch.float32),
+        v_scale=_dev_ptr(v_scale, "v_scale", torch.float32),
+        tables=_dev_ptr(block_tables, "block_tables", torch.int32),
+        lens=_dev_ptr(context_lens, "context_lens", torch.int32),
+        sizes=(s, hq, hkv, d, bs, nb, block_tables.shape[1]), ws=(ws_ptr, ws_bytes))
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                  max_context_len: int, scale: float, partition_size: int = 0, workspace=None,
+                  stream=None) -> None:
+    """pa_decode over E4M3 caches (uint8 codes, per-KV-head float32 scales);
+    q and out are bfloat16 [S, Hq, d]. See pa_decode_fp8 in include/pa.h."""
+    torch = _torch()
+    a = _fp8_decode_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                         workspace)
+    _check(_lib.pa_decode_fp8(
+        _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16), a["k_cache"],
+        a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"], *a["sizes"],
+        int(max_context_len), float(scale), int(partition_size), *a["ws"],
+        _stream(stream, q.device)))
+
+
+def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tables,
+                         context_lens, max_context_len: int, scale: float,
+                         partition_size: int = 0, workspace=None, stream=None) -> None:
+    """pa_decode_append over E4M3 caches: quantise and write each sequence's newest
+    token (k_new / v_new bfloat16 [S, Hkv, d]), then attend."""
+    torch = _torch()
+    a = _fp8_decode_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                         workspace)
+    s, _, hkv, d = a["sizes"][:4]
+    if k_new.shape != (s, hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new/v_new must be [S, num_kv_heads, head_dim]")
+    _check(_lib.pa_decode_append_fp8(
+        _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16),
+        _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
+        a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"],
+        *a["sizes"], int(max_context_len), float(scale), int(partition_size), *a["ws"],
+        _stream(stream, q.device)))
 
 
 def pa_device_errors(stream=None) -> int:

@@ -13,6 +13,11 @@ workspace. Each method marshals arguments and calls libpa.so:
       writes the new K/V rows and attends in one launch (fused=False: separate
       pa_kv_append and pa_decode calls, same result).
 
+dtype "fp8_e4m3": the caches hold uint8 E4M3 codes with one float32 scale per
+KV head (k_scale, v_scale); rows come in as bfloat16 and are quantised on the
+device (pa_kv_append_fp8 / pa_decode_append_fp8), decode reads the codes
+(pa_decode_fp8).
+
 "Paged Attention" (klaylearn.com glossary), definition: prefill allocates and
 fills blocks, decode appends into the tail block or triggers an allocation,
 finished requests return their blocks to the free list.
@@ -23,17 +28,24 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append,
-               pa_decode_partition_size, pa_decode_workspace_bytes, pa_kv_append)
+from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_decode_append_fp8,
+               pa_decode_fp8, pa_decode_partition_size, pa_decode_workspace_bytes, pa_kv_append,
+               pa_kv_append_fp8)
 
-_TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+_TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}
 
 
 class PagedKVCache:
     def __init__(self, num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
                  dtype="bf16", device="cuda", max_blocks_per_seq: int | None = None,
-                 free_order=None, stream=None):
+                 free_order=None, stream=None, k_scale=None, v_scale=None):
         self.dtype = _TORCH_DTYPES.get(dtype, dtype)
+        self.fp8 = self.dtype == torch.uint8
+        if self.fp8:
+            def per_head(x):
+                x = torch.ones(num_kv_heads) if x is None else torch.as_tensor(x)
+                return x.to(dtype=torch.float32).expand(num_kv_heads).contiguous().to(device)
+            self.k_scale, self.v_scale = per_head(k_scale), per_head(v_scale)
         self.device = torch.device(device)
         self.block_size = block_size
         self.num_blocks = num_blocks
@@ -74,8 +86,12 @@ class PagedKVCache:
         if len(cows):
             pa_copy_blocks(self.k_cache, self.v_cache, self._to_device(cows), stream=self.stream)
         if len(slots):
-            pa_kv_append(k_rows, v_rows, self._to_device(slots), self.k_cache, self.v_cache,
-                         stream=self.stream)
+            if self.fp8:
+                pa_kv_append_fp8(k_rows, v_rows, self._to_device(slots), self.k_cache,
+                                 self.v_cache, self.k_scale, self.v_scale, stream=self.stream)
+            else:
+                pa_kv_append(k_rows, v_rows, self._to_device(slots), self.k_cache, self.v_cache,
+                             stream=self.stream)
         return slots
 
     # --------------------------------------------------------------- decode
@@ -99,9 +115,14 @@ class PagedKVCache:
             partition_size = pa_decode_partition_size(num_seqs, self.num_kv_heads, max_len)
         out = torch.empty_like(q) if out is None else out
         scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
-        pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, max_len, scale,
-                  partition_size, self.workspace(num_seqs, num_heads, max_len, partition_size),
-                  stream=self.stream)
+        ws = self.workspace(num_seqs, num_heads, max_len, partition_size)
+        if self.fp8:
+            pa_decode_fp8(out, q, self.k_cache, self.v_cache, self.k_scale, self.v_scale,
+                          block_tables, context_lens, max_len, scale, partition_size, ws,
+                          stream=self.stream)
+        else:
+            pa_decode(out, q, self.k_cache, self.v_cache, block_tables, context_lens, max_len,
+                      scale, partition_size, ws, stream=self.stream)
         return out
 
     def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
@@ -118,8 +139,13 @@ class PagedKVCache:
             partition_size = pa_decode_partition_size(num_seqs, self.num_kv_heads, max_len)
         out = torch.empty_like(q) if out is None else out
         scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
-        pa_decode_append(out, q, k_new, v_new, self.k_cache, self.v_cache, block_tables,
-                         context_lens, max_len, scale, partition_size,
-                         self.workspace(num_seqs, num_heads, max_len, partition_size),
-                         stream=self.stream)
+        ws = self.workspace(num_seqs, num_heads, max_len, partition_size)
+        if self.fp8:
+            pa_decode_append_fp8(out, q, k_new, v_new, self.k_cache, self.v_cache, self.k_scale,
+                                 self.v_scale, block_tables, context_lens, max_len, scale,
+                                 partition_size, ws, stream=self.stream)
+        else:
+            pa_decode_append(out, q, k_new, v_new, self.k_cache, self.v_cache, block_tables,
+                             context_lens, max_len, scale, partition_size, ws,
+                             stream=self.stream)
         return out

@@ -14,8 +14,11 @@ thread_local std::string g_last_error;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
-int elem_bytes(pa_dtype dt) { return dt == PA_BF16 ? 2 : 4; }
-bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16; }
+int elem_bytes(pa_dtype dt) { return dt == PA_FP8_E4M3 ? 1 : dt == PA_BF16 ? 2 : 4; }
+// dtypes of calls that move whole rows or blocks bit for bit
+bool valid_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16 || dt == PA_FP8_E4M3; }
+// dtypes of pa_kv_append / pa_decode / pa_decode_append (E4M3: the _fp8 calls)
+bool valid_compute_dtype(int dt) { return dt == PA_F32 || dt == PA_BF16; }
 
 int cuda_fail(const char* what, cudaError_t e) {
   return pa_fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -85,7 +88,9 @@ int pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mappi
   if (num_tokens == 0) return PA_OK;
   if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache)
     return pa_fail(PA_ERR_INVALID, "pa_kv_append: null pointer");
-  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_kv_append: dtype %d", dtype);
+  if (!valid_compute_dtype(dtype))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_kv_append: dtype %d (E4M3 caches: pa_kv_append_fp8)",
+                   dtype);
   if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
     return pa_fail(PA_ERR_INVALID, "pa_kv_append: sizes must be positive");
   const int64_t row_bytes = static_cast<int64_t>(num_kv_heads) * head_dim * elem_bytes(dtype);
@@ -101,6 +106,30 @@ int pa_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mappi
                                        num_slots, static_cast<int>(row_bytes),
                                        reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_kv_append launch", e);
+}
+
+int pa_kv_append_fp8(const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                     int num_tokens, void* k_cache, void* v_cache, const float* k_scale,
+                     const float* v_scale, int num_blocks, int block_size, int num_kv_heads,
+                     int head_dim, pa_stream_t stream) {
+  if (num_tokens < 0) return pa_fail(PA_ERR_INVALID, "pa_kv_append_fp8: num_tokens < 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append_fp8: null pointer");
+  if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append_fp8: sizes must be positive");
+  if (head_dim % 16 != 0 || static_cast<int64_t>(num_kv_heads) * head_dim > (1 << 28))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_kv_append_fp8: head_dim %d not a multiple of 16",
+                   head_dim);
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(slot_mapping, 8) || !aligned(k_scale, 4) ||
+      !aligned(v_scale, 4))
+    return pa_fail(PA_ERR_INVALID, "pa_kv_append_fp8: misaligned pointer");
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  cudaError_t e = pa::launch_kv_append_fp8(k_new, v_new, slot_mapping, num_tokens, k_cache,
+                                           v_cache, k_scale, v_scale, num_slots, num_kv_heads,
+                                           head_dim, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_kv_append_fp8 launch", e);
 }
 
 int pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int num_pairs,
@@ -190,12 +219,21 @@ static int decode_common(void* out, const void* q, const void* k_cache, const vo
                          int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
                          int partition_size, void* workspace, size_t workspace_bytes,
                          pa_dtype dtype, const void* k_new, const void* v_new,
-                         pa_stream_t stream) {
+                         const float* k_scale, const float* v_scale, pa_stream_t stream) {
   if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode: num_seqs < 0");
   if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return pa_fail(PA_ERR_INVALID, "pa_decode: null pointer");
-  if (!valid_dtype(dtype)) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: dtype %d", dtype);
+  const bool fp8 = dtype == PA_FP8_E4M3;
+  if (!fp8 && !valid_compute_dtype(dtype))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: dtype %d (E4M3 caches: pa_decode_fp8)", dtype);
+  if (fp8) {
+    if (!k_scale || !v_scale) return pa_fail(PA_ERR_INVALID, "pa_decode_fp8: null scale");
+    if (!aligned(k_scale, 4) || !aligned(v_scale, 4))
+      return pa_fail(PA_ERR_INVALID, "pa_decode_fp8: misaligned scale");
+    if (head_dim != 128)
+      return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_fp8: head_dim %d (built: 128)", head_dim);
+  }
   if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
     return pa_fail(PA_ERR_INVALID, "pa_decode: num_heads %d not a multiple of num_kv_heads %d",
                    num_heads, num_kv_heads);
@@ -253,7 +291,7 @@ static int decode_common(void* out, const void* q, const void* k_cache, const vo
     return pa_fail(PA_ERR_INVALID, "pa_decode: workspace %zu B < %zu B needed",
                    workspace ? workspace_bytes : size_t(0), need);
   cudaError_t e = pa::launch_decode(sh, out, q, k_cache, v_cache, block_tables, context_lens,
-                                    workspace, k_new, v_new,
+                                    workspace, k_new, v_new, k_scale, v_scale,
                                     reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: no kernel for this shape");
@@ -265,10 +303,12 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               int num_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
               int max_blocks_per_seq, int max_context_len, float scale, int partition_size,
               void* workspace, size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (dtype == PA_FP8_E4M3)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: E4M3 caches decode through pa_decode_fp8");
   return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
-                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype,
-                       nullptr, nullptr, stream);
+                       max_context_len, scale, partition_size, workspace, workspace_bytes,
+                       dtype, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
@@ -277,14 +317,47 @@ int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_
                      int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                      int max_context_len, float scale, int partition_size, void* workspace,
                      size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (dtype == PA_FP8_E4M3)
+    return pa_fail(PA_ERR_UNSUPPORTED,
+                   "pa_decode_append: E4M3 caches decode through pa_decode_append_fp8");
   if (num_seqs > 0 && (!k_new || !v_new))
     return pa_fail(PA_ERR_INVALID, "pa_decode_append: null k_new or v_new");
   if (num_seqs > 0 && (!aligned(k_new, 16) || !aligned(v_new, 16)))
     return pa_fail(PA_ERR_INVALID, "pa_decode_append: misaligned k_new or v_new");
   return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
-                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype,
-                       k_new, v_new, stream);
+                       max_context_len, scale, partition_size, workspace, workspace_bytes,
+                       dtype, k_new, v_new, nullptr, nullptr, stream);
+}
+
+int pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                  const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                  int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                  int max_context_len, float scale, int partition_size, void* workspace,
+                  size_t workspace_bytes, pa_stream_t stream) {
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes,
+                       PA_FP8_E4M3, nullptr, nullptr, k_scale, v_scale, stream);
+}
+
+int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void* v_new,
+                         void* k_cache, void* v_cache, const float* k_scale,
+                         const float* v_scale, const int32_t* block_tables,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                         int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void* workspace, size_t workspace_bytes,
+                         pa_stream_t stream) {
+  if (num_seqs > 0 && (!k_new || !v_new))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_append_fp8: null k_new or v_new");
+  if (num_seqs > 0 && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_append_fp8: misaligned k_new or v_new");
+  return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes,
+                       PA_FP8_E4M3, k_new, v_new, k_scale, v_scale, stream);
 }
 
 int pa_device_errors(pa_stream_t stream, unsigned int* flags) {

@@ -55,6 +55,9 @@ struct DecodeParams {
   uint8_t* k_cache_w;
   uint8_t* v_cache_w;
   unsigned* err;
+  // E4M3 caches: cache value = code * scale, one scale per KV head [Hkv]. Null otherwise.
+  const float* k_scale;
+  const float* v_scale;
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks;
   int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
   float q_scale;  // scale * log2(e)
@@ -76,6 +79,28 @@ __device__ __forceinline__ void append_newest_rows(const DecodeParams& p, int s,
     const uint4 b = ldg_stream(p.v_new + src + i * 16);
     *reinterpret_cast<uint4*>(p.k_cache_w + dst + i * 16) = a;
     *reinterpret_cast<uint4*>(p.v_cache_w + dst + i * 16) = b;
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncwarp();
+}
+
+// The same for an E4M3 cache: k_new / v_new hold bfloat16 rows of head_dim
+// values; each value is stored as the E4M3 code of value / scale[head].
+__device__ __forceinline__ void append_newest_rows_fp8(const DecodeParams& p, int s, int blk,
+                                                       int off, int h0, int nh, int head_dim,
+                                                       int lane) {
+  const int units = nh * head_dim / 16;  // 16 values per unit
+  const int64_t src = (static_cast<int64_t>(s) * p.num_kv_heads + h0) * head_dim * 2;
+  const int64_t dst =
+      ((static_cast<int64_t>(blk) * p.block_size + off) * p.num_kv_heads + h0) * head_dim;
+  for (int i = lane; i < units; i += 32) {
+    const int h = h0 + i * 16 / head_dim;
+    const uint4* ks = reinterpret_cast<const uint4*>(p.k_new + src) + 2 * i;
+    const uint4* vs = reinterpret_cast<const uint4*>(p.v_new + src) + 2 * i;
+    const uint4 kc = bf16x16_to_e4m3(ldg_stream(ks), ldg_stream(ks + 1), __ldg(p.k_scale + h));
+    const uint4 vc = bf16x16_to_e4m3(ldg_stream(vs), ldg_stream(vs + 1), __ldg(p.v_scale + h));
+    *reinterpret_cast<uint4*>(p.k_cache_w + dst + i * 16) = kc;
+    *reinterpret_cast<uint4*>(p.v_cache_w + dst + i * 16) = vc;
   }
   asm volatile("fence.proxy.async.global;" ::: "memory");
   __syncwarp();

@@ -40,6 +40,25 @@
 //  * Chunks hold the same 16 logical tokens and are reduced in the same order
 //    whatever the block size or placement, so results are bit-identical across
 //    both.
+//
+// E4M3 (fp8) caches (FP8 = true, head_dim 128): the same pipeline moves rows
+// of head_dim bytes (+16 zero bytes of padding, again from out-of-range box
+// columns). No 8-bit ldmatrix transpose is used; each lane instead reads its
+// operand bytes with 16-byte shared loads and widens them in registers
+// (E4M3 -> float16 is exact), and the stage is released as soon as the loads
+// are done. The inner products use float16 MMAs:
+//  * S^T: lane (g, t) loads the 16-byte columns 2t and 2t+1 of token rows g
+//    and g+8. The contraction index is permuted (the same permutation for K
+//    and for Q, which is loaded to match), so each loaded 32-bit word becomes
+//    the a0/a2 (row g) or a1/a3 (row g+8) register of one k-step directly.
+//  * O^T: lane (g, t) loads column g (head_dim values 16g .. 16g+15) of token
+//    rows 2t, 2t+1, 2t+8, 2t+9; a byte permute pairs the two tokens of each
+//    A register. MMA row r of tile dt stands for head_dim index 16g + 2dt (+1
+//    for r = g + 8), which the epilogue maps back.
+//  * With a padded row stride of 144 bytes both load patterns touch 8
+//    distinct 16-byte bank groups per quarter warp.
+//  * Scores are scaled by scale * log2(e) * k_scale[head], the output by
+//    v_scale[head].
 #pragma once
 
 #include <cmath>
@@ -50,10 +69,10 @@
 
 namespace pa {
 
-template <int D, int G, int HB, int NS>
+template <int D, int G, int HB, int NS, bool FP8 = false>
 struct GroupConfig {
   static constexpr int kC = 16;                       // tokens per chunk / stage
-  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRowBytes = FP8 ? D : D * 2;
   static constexpr int kRS = kRowBytes + 16;          // padded row stride in shared memory
   // One chunk of K (or V) for the group: up to 16 boxes (block_size 1) of HB
   // rows each, every box padded to a 128-byte boundary; fewer, larger boxes
@@ -66,6 +85,7 @@ struct GroupConfig {
   static constexpr int kSmemBytes = 128 + kRingBytes + kBarBytes;
   static_assert(G >= 1 && G <= 8, "group must fit the 8 real rows of an m16 tile");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert(!FP8 || D == 128, "the E4M3 operand layout is built for head_dim 128");
 };
 
 // Bytes between consecutive TMA boxes of one chunk (rows_per_box tokens of HB
@@ -74,11 +94,11 @@ __host__ __device__ constexpr int box_stride_bytes(int hb, int rows_per_box, int
   return (hb * rows_per_box * rs + 127) & ~127;
 }
 
-template <int D, int G, int HB, int NS>
-__global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
+template <int D, int G, int HB, int NS, bool FP8>
+__global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     pa_decode_mma_kernel(const __grid_constant__ CUtensorMap k_map,
                          const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
-  using Cfg = GroupConfig<D, G, HB, NS>;
+  using Cfg = GroupConfig<D, G, HB, NS, FP8>;
   constexpr int C = Cfg::kC, RS = Cfg::kRS, TB = Cfg::kTensorBytes;
 
   extern __shared__ uint8_t smem_raw[];
@@ -119,14 +139,31 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
   const int qc = lane & 3;   // fragment column pair
   const bool real_row = qr < G;
   const int64_t out_row = static_cast<int64_t>(s) * p.num_heads + kvh * G;
-  uint32_t qa[D / 16][2];  // Q as the A operand: rows = heads of the group, bf16 pairs
+  uint32_t qa[D / 16][2];  // Q as the B operand (column = head of the group), 16-bit pairs
   if (warp < HB) {
     const uint32_t* qp = reinterpret_cast<const uint32_t*>(
         static_cast<const __nv_bfloat16*>(p.q) + (out_row + (real_row ? qr : 0)) * D);
+    if constexpr (!FP8) {
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      qa[ks][0] = real_row ? __ldg(qp + ks * 8 + qc) : 0u;
-      qa[ks][1] = real_row ? __ldg(qp + ks * 8 + 4 + qc) : 0u;
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa[ks][0] = real_row ? __ldg(qp + ks * 8 + qc) : 0u;
+        qa[ks][1] = real_row ? __ldg(qp + ks * 8 + 4 + qc) : 0u;
+      }
+    } else {
+      // k-step 4kq + j covers head_dim 16 (2 qc + kq) + 4j .. +3 (b0: +0, +1; b1: +2, +3),
+      // the order in which the K loads below deliver them; float16 pairs.
+#pragma unroll
+      for (int kq = 0; kq < D / 64; ++kq) {
+        const uint4* q4 = reinterpret_cast<const uint4*>(qp) + 2 * (2 * qc + kq);
+        const uint4 lo = real_row ? __ldg(q4) : make_uint4(0, 0, 0, 0);
+        const uint4 hi = real_row ? __ldg(q4 + 1) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          qa[4 * kq + j][0] = bf16x2_to_f16x2(w[2 * j]);
+          qa[4 * kq + j][1] = bf16x2_to_f16x2(w[2 * j + 1]);
+        }
+      }
     }
   }
 
@@ -172,9 +209,12 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
         // this CTA holds the sequence's newest token: write it before reading it
         const int tn = L - 1;
         const int bn = __shfl_sync(kFullMask, ent, (tn >> lg) - base);
-        if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks))
-          append_newest_rows(p, s, bn, tn & (bs - 1), hg * HB, HB, Cfg::kRowBytes, lane);
-        else if (lane == 0)
+        if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks)) {
+          if constexpr (FP8)
+            append_newest_rows_fp8(p, s, bn, tn & (bs - 1), hg * HB, HB, D, lane);
+          else
+            append_newest_rows(p, s, bn, tn & (bs - 1), hg * HB, HB, Cfg::kRowBytes, lane);
+        } else if (lane == 0)
           atomicOr(p.err, PA_DEVERR_BLOCK_ID);
       }
       const int nbox = lb_hi - lb_lo + 1;  // blocks holding valid tokens of this chunk
@@ -203,8 +243,12 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
   //   O^T[d][head]    += V^T[d][token] . P^T[token][head]   (A = V^T, B = P^T)
   // Fragment coordinates: g = lane / 4 (row), t = lane % 4 (column pair).
   const int g = lane >> 2, t = lane & 3;
-  const float qscale = p.q_scale;
-  float o[D / 16][4];  // O^T fragments: (d = 16i + g (+8), head 2t (+1))
+  float qscale = p.q_scale, vscale = 1.0f;
+  if constexpr (FP8) {
+    qscale *= __ldg(p.k_scale + kvh);
+    vscale = __ldg(p.v_scale + kvh);
+  }
+  float o[D / 16][4];  // O^T fragments: (d = 16i + g (+8), head 2t (+1)); E4M3: see the top
 #pragma unroll
   for (int i = 0; i < D / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
   float m[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.0f, 0.0f};  // heads 2t, 2t+1
@@ -231,24 +275,58 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
     uint8_t* stage = smem + st * Cfg::kStageBytes;
     const uint32_t ks_u32 = smem_u32(stage), vs_u32 = ks_u32 + TB;
     const int nvalid = min(C, t1 - (t0 + c * C));
-    if (nvalid < C) {
-      // rows past the context hold stale bits: zero this head's V rows so 0 * stale = 0
-      for (int i = lane; i < (C - nvalid) * (D / 8); i += 32) {
-        const int r = nvalid + i / (D / 8), cc = i % (D / 8);
-        *reinterpret_cast<uint4*>(stage + TB + at(r, cc)) = make_uint4(0, 0, 0, 0);
-      }
-      // order these generic-proxy writes before the next async copy into the stage
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-    }
 
     // S^T: two accumulation chains (even / odd k-steps) for latency
     float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint4 vr[4];  // E4M3: V bytes of tokens 2t, 2t+1, 2t+8, 2t+9, head_dim 16g .. 16g+15
+    if constexpr (!FP8) {
+      if (nvalid < C) {
+        // rows past the context hold stale bits: zero this head's V rows so 0 * stale = 0
+        for (int i = lane; i < (C - nvalid) * (D / 8); i += 32) {
+          const int r = nvalid + i / (D / 8), cc = i % (D / 8);
+          *reinterpret_cast<uint4*>(stage + TB + at(r, cc)) = make_uint4(0, 0, 0, 0);
+        }
+        // order these generic-proxy writes before the next async copy into the stage
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      uint32_t a[4];
-      ldmatrix_x4(a, ks_u32 + k_lane + ks * 32);
-      mma_bf16_16816(ks & 1 ? s1 : s0, a, qa[ks][0], qa[ks][1]);
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(a, ks_u32 + k_lane + ks * 32);
+        mma_bf16_16816(ks & 1 ? s1 : s0, a, qa[ks][0], qa[ks][1]);
+      }
+    } else {
+      uint4 kr[2][D / 64];  // tokens g, g+8; 16-byte columns 2t + kq
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int kq = 0; kq < D / 64; ++kq) kr[h][kq] = lds128(ks_u32 + at(g + 8 * h, 2 * t + kq));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // rows past the context hold stale bytes (possibly NaN codes): use zeros
+        const int r = 2 * t + (i & 1) + 8 * (i >> 1);
+        const uint4 x = lds128(vs_u32 + at(r, g));
+        vr[i] = r < nvalid ? x : make_uint4(0, 0, 0, 0);
+      }
+      // every operand byte is in registers: hand the stage back to the producer
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(bars + NS + st));
+#pragma unroll
+      for (int kq = 0; kq < D / 64; ++kq) {
+        const uint32_t w0[4] = {kr[0][kq].x, kr[0][kq].y, kr[0][kq].z, kr[0][kq].w};
+        const uint32_t w1[4] = {kr[1][kq].x, kr[1][kq].y, kr[1][kq].z, kr[1][kq].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int ks = 4 * kq + j;
+          uint32_t a[4];
+          a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[j]));
+          a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[j]));
+          a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(w0[j] >> 16));
+          a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(w1[j] >> 16));
+          mma_f16_16816(ks & 1 ? s1 : s0, a, qa[ks][0], qa[ks][1]);
+        }
+      }
     }
     // x[0], x[1]: token g, heads 2t, 2t+1; x[2], x[3]: token g + 8
     float x[4];
@@ -279,17 +357,40 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
       o[i][2] *= al0;
       o[i][3] *= al1;
     }
-    // P^T as B: (token 2t, 2t+1 (+8), head g) = transpose of the (token g, head 2t..) pairs
-    const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
-    const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
+    if constexpr (!FP8) {
+      // P^T as B: (token 2t, 2t+1 (+8), head g) = transpose of the (token g, head 2t..) pairs
+      const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
+      const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
 #pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt) {
-      uint32_t a[4];
-      ldmatrix_x4_trans(a, vs_u32 + v_lane + dt * 32);
-      mma_bf16_16816(o[dt], a, b0, b1);
+      for (int dt = 0; dt < D / 16; ++dt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vs_u32 + v_lane + dt * 32);
+        mma_bf16_16816(o[dt], a, b0, b1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(bars + NS + st));
+    } else {
+      const uint32_t b0 = movmatrix_trans(pack_f16x2(p0, p1));
+      const uint32_t b1 = movmatrix_trans(pack_f16x2(p2, p3));
+      const uint32_t v0[4] = {vr[0].x, vr[0].y, vr[0].z, vr[0].w};
+      const uint32_t v1[4] = {vr[1].x, vr[1].y, vr[1].z, vr[1].w};
+      const uint32_t v2[4] = {vr[2].x, vr[2].y, vr[2].z, vr[2].w};
+      const uint32_t v3[4] = {vr[3].x, vr[3].y, vr[3].z, vr[3].w};
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt) {
+        // head_dim 16g + 2dt (row g) and +1 (row g + 8): bytes 2(dt&1), +1 of word dt/2;
+        // the byte permute puts token 2t next to 2t+1 (and 2t+8 next to 2t+9)
+        const uint32_t sel = (dt & 1) ? 0x7362u : 0x5140u;
+        const uint32_t x01 = prmt(v0[dt >> 1], v1[dt >> 1], sel);
+        const uint32_t x89 = prmt(v2[dt >> 1], v3[dt >> 1], sel);
+        uint32_t a[4];
+        a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01));
+        a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(x01 >> 16));
+        a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89));
+        a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(x89 >> 16));
+        mma_f16_16816(o[dt], a, b0, b1);
+      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(bars + NS + st));
   }
 
   // softmax denominators per head: sum over the 8 row groups
@@ -300,6 +401,55 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS>::kThreads)
     l1 += __shfl_xor_sync(kFullMask, l1, off);
   }
   const bool h0_real = 2 * t < G, h1_real = 2 * t + 1 < G;
+
+  if constexpr (FP8) {
+    // lane (g, t) holds head_dim 16g .. 16g+15 of heads 2t and 2t+1:
+    // o[dt][0] / o[dt][1] at 16g + 2dt, o[dt][2] / o[dt][3] at 16g + 2dt + 1
+    if (n_part_s == 1) {
+      const float i0 = l0 > 0.0f ? vscale / l0 : 0.0f, i1 = l1 > 0.0f ? vscale / l1 : 0.0f;
+      uint32_t w0[8], w1[8];
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt) {
+        w0[dt] = pack_bf16x2(o[dt][0] * i0, o[dt][2] * i0);
+        w1[dt] = pack_bf16x2(o[dt][1] * i1, o[dt][3] * i1);
+      }
+      uint4* o0 = reinterpret_cast<uint4*>(out + (out_row + 2 * t) * D + 16 * g);
+      uint4* o1 = reinterpret_cast<uint4*>(out + (out_row + 2 * t + 1) * D + 16 * g);
+      if (h0_real) {
+        o0[0] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+        o0[1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
+      }
+      if (h1_real) {
+        o1[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        o1[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+      }
+      return;
+    }
+    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + part;
+    const int64_t w1 = w0 + p.num_partitions;
+    float4* a0 = reinterpret_cast<float4*>(p.ws_acc + w0 * D + 16 * g);
+    float4* a1 = reinterpret_cast<float4*>(p.ws_acc + w1 * D + 16 * g);
+#pragma unroll
+    for (int q4 = 0; q4 < D / 32; ++q4) {
+      if (h0_real)
+        a0[q4] = make_float4(o[2 * q4][0] * vscale, o[2 * q4][2] * vscale,
+                             o[2 * q4 + 1][0] * vscale, o[2 * q4 + 1][2] * vscale);
+      if (h1_real)
+        a1[q4] = make_float4(o[2 * q4][1] * vscale, o[2 * q4][3] * vscale,
+                             o[2 * q4 + 1][1] * vscale, o[2 * q4 + 1][3] * vscale);
+    }
+    if (g == 0) {
+      if (h0_real) {
+        p.ws_m[w0] = m[0];
+        p.ws_l[w0] = l0;
+      }
+      if (h1_real) {
+        p.ws_m[w1] = m[1];
+        p.ws_l[w1] = l1;
+      }
+    }
+    return;
+  }
 
   if (n_part_s == 1) {
     const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;

@@ -170,6 +170,68 @@ __device__ __forceinline__ void mma_bf16_16816_rows0to7(float& d0, float& d1, ui
       : "f"(d0), "f"(d1), "r"(a0), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// Same MMA with float16 inputs (used for the fp8 cache: E4M3 values are exact in float16).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+      " {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two floats to a float16 pair (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (low byte first) to a float16 pair (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+
+// Two floats to E4M3 codes (round to nearest even, finite values saturate at
+// +-448); `lo` in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte permute: bytes 0-3 of `a` and 4-7 of `b`, picked by the four selector nibbles.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// A bfloat16 pair to a float16 pair (exact for magnitudes in [2^-14, 65504]).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Sixteen bfloat16 values (a: 0-7, b: 8-15) to E4M3 codes of value / scale,
+// byte i = value i. The division is IEEE float32 (round to nearest), then
+// round to nearest even into E4M3 with saturation at +-448.
+__device__ __forceinline__ uint4 bf16x16_to_e4m3(const uint4& a, const uint4& b, float scale) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float f0 = __fdiv_rn(__uint_as_float(w[2 * i] << 16), scale);
+    const float f1 = __fdiv_rn(__uint_as_float(w[2 * i] & 0xffff0000u), scale);
+    const float f2 = __fdiv_rn(__uint_as_float(w[2 * i + 1] << 16), scale);
+    const float f3 = __fdiv_rn(__uint_as_float(w[2 * i + 1] & 0xffff0000u), scale);
+    r[i] = static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) |
+           (static_cast<uint32_t>(f32x2_to_e4m3x2(f2, f3)) << 16);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 // Transpose an 8x8 matrix of b16 held as an MMA fragment (lane i: row i / 4,
 // columns 2 (i % 4), +1) into the same fragment layout.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {

@@ -39,6 +39,12 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, 
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
                              int num_tokens, void* k_cache, void* v_cache, int64_t num_slots,
                              int row_bytes, cudaStream_t stream);
+// E4M3 caches: bfloat16 rows in, code of value / scale[head] stored.
+cudaError_t launch_kv_append_fp8(const void* k_new, const void* v_new,
+                                 const int64_t* slot_mapping, int num_tokens, void* k_cache,
+                                 void* v_cache, const float* k_scale, const float* v_scale,
+                                 int64_t num_slots, int num_kv_heads, int head_dim,
+                                 cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
                                int num_pairs, int num_blocks, int64_t block_bytes,
                                cudaStream_t stream);
@@ -47,10 +53,12 @@ cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, cons
                                int dst_num_blocks, int64_t block_bytes, cudaStream_t stream);
 // Returns cudaErrorNotSupported when no kernel is built for the shape.
 // k_new / v_new non-null: fused append of each sequence's newest token.
+// k_scale / v_scale: per-KV-head scales of an E4M3 cache (null otherwise).
 cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* block_tables,
                           const int32_t* context_lens, void* workspace, const void* k_new,
-                          const void* v_new, cudaStream_t stream);
+                          const void* v_new, const float* k_scale, const float* v_scale,
+                          cudaStream_t stream);
 // Device error word of the current device (address in device memory).
 cudaError_t device_error_word(unsigned int** ptr);
 

@@ -107,6 +107,58 @@ cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t
                     static_cast<uint4*>(v_cache), num_slots, row_bytes / 16, err);
 }
 
+// One warp per token row, E4M3 caches: 16 values per lane step (32 bytes of
+// bfloat16 in, 16 codes out), each divided by its KV head's scale.
+__global__ void __launch_bounds__(256)
+    kv_append_fp8_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                         const int64_t* __restrict__ slot_mapping, int num_tokens,
+                         uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                         const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+                         int64_t num_slots, int head_dim, int units_per_row, unsigned* err) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t tok = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       tok < num_tokens; tok += warps) {
+    const int64_t slot = __ldg(slot_mapping + tok);
+    if (slot < 0) continue;  // padding row
+    if (slot >= num_slots) {
+      if (lane == 0) atomicOr(err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const uint4* ks = k_new + tok * units_per_row * 2;
+    const uint4* vs = v_new + tok * units_per_row * 2;
+    uint4* kd = k_cache + slot * units_per_row;
+    uint4* vd = v_cache + slot * units_per_row;
+    for (int u = lane; u < units_per_row; u += 32) {
+      const int h = u * 16 / head_dim;
+      kd[u] = bf16x16_to_e4m3(ldg_stream(ks + 2 * u), ldg_stream(ks + 2 * u + 1),
+                              __ldg(k_scale + h));
+      vd[u] = bf16x16_to_e4m3(ldg_stream(vs + 2 * u), ldg_stream(vs + 2 * u + 1),
+                              __ldg(v_scale + h));
+    }
+  }
+}
+
+cudaError_t launch_kv_append_fp8(const void* k_new, const void* v_new,
+                                 const int64_t* slot_mapping, int num_tokens, void* k_cache,
+                                 void* v_cache, const float* k_scale, const float* v_scale,
+                                 int64_t num_slots, int num_kv_heads, int head_dim,
+                                 cudaStream_t stream) {
+  unsigned* err = nullptr;
+  cudaError_t e = device_error_word(&err);
+  if (e != cudaSuccess) return e;
+  const int threads = 256, warps_per_cta = threads / 32;
+  int64_t ctas = (static_cast<int64_t>(num_tokens) + warps_per_cta - 1) / warps_per_cta;
+  if (ctas > 148 * 16) ctas = 148 * 16;
+  return launch_pdl(kv_append_fp8_kernel, dim3(static_cast<unsigned>(ctas)), dim3(threads), 0,
+                    stream, static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                    slot_mapping, num_tokens, static_cast<uint4*>(k_cache),
+                    static_cast<uint4*>(v_cache), k_scale, v_scale, num_slots, head_dim,
+                    num_kv_heads * head_dim / 16, err);
+}
+
 // -------------------------------------------------------------- copy blocks
 
 // blockIdx.x = pair, blockIdx.y = slice of the block; 16-byte vector copies.
@@ -279,40 +331,44 @@ cudaError_t launch_decode_f32(const DecodeShape& sh, const DecodeParams& p, cons
 }
 
 // 4-D view of a cache with the dimensions ordered (column, token, head, block)
-// so that a box {head_dim + 8, rows, heads, 1} lands in shared memory as
-// [head][token][head_dim + 8]; the 8 columns past head_dim are outside the
-// tensor and arrive as zeros (row padding against bank conflicts).
+// so that a box {head_dim + 16 bytes, rows, heads, 1} lands in shared memory
+// as [head][token][row + 16 bytes]; the columns past head_dim are outside the
+// tensor and arrive as zeros (row padding against bank conflicts). bfloat16
+// or, for E4M3 caches, bytes.
 cudaError_t encode_group_map(CUtensorMap* map, const void* base, const DecodeShape& sh,
                              int box_rows, int box_heads) {
   auto enc = tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
-  const cuuint64_t row = static_cast<cuuint64_t>(sh.head_dim) * 2;
+  const bool fp8 = sh.dtype == PA_FP8_E4M3;
+  const cuuint64_t row = static_cast<cuuint64_t>(sh.head_dim) * (fp8 ? 1 : 2);
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(sh.head_dim),
                               static_cast<cuuint64_t>(sh.block_size),
                               static_cast<cuuint64_t>(sh.num_kv_heads),
                               static_cast<cuuint64_t>(sh.num_blocks)};
   const cuuint64_t strides[3] = {row * sh.num_kv_heads, row,
                                  row * sh.num_kv_heads * static_cast<cuuint64_t>(sh.block_size)};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(sh.head_dim + 8),
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(sh.head_dim + (fp8 ? 16 : 8)),
                              static_cast<cuuint32_t>(box_rows),
                              static_cast<cuuint32_t>(box_heads), 1u};
   const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+  const CUtensorMapDataType type =
+      fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = enc(map, type, 4, const_cast<void*>(base), dims, strides,
                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// bfloat16 caches: tensor-core kernel over groups of HB KV heads.
-template <int D, int G, int HB>
-cudaError_t launch_decode_bf16_t(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
-                                 const void* v_cache, cudaStream_t stream) {
+// bfloat16 and E4M3 caches: tensor-core kernel over groups of HB KV heads.
+template <int D, int G, int HB, bool FP8>
+cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
+                                  const void* k_cache, const void* v_cache, cudaStream_t stream) {
   // stages: as many as fit ~112 KB of ring (two CTAs per SM), at most 4
-  constexpr int kStage = 2 * GroupConfig<D, G, HB, 1>::kTensorBytes;
+  constexpr int kStage = 2 * GroupConfig<D, G, HB, 1, FP8>::kTensorBytes;
   constexpr int kNSfit = 114688 / kStage;
   constexpr int NS = kNSfit < 2 ? 2 : (kNSfit > 4 ? 4 : kNSfit);
-  using Cfg = GroupConfig<D, G, HB, NS>;
-  auto kernel = pa_decode_mma_kernel<D, G, HB, NS>;
+  using Cfg = GroupConfig<D, G, HB, NS, FP8>;
+  auto kernel = pa_decode_mma_kernel<D, G, HB, NS, FP8>;
   static std::atomic<unsigned long long> configured{0};
   cudaError_t e = ensure_smem(kernel, Cfg::kSmemBytes, configured);
   if (e != cudaSuccess) return e;
@@ -326,17 +382,41 @@ cudaError_t launch_decode_bf16_t(const DecodeShape& sh, const DecodeParams& p, c
   return launch_merge<__nv_bfloat16, D>(sh, p, stream);
 }
 
+template <int D, int G, bool FP8>
+cudaError_t launch_decode_group(const DecodeShape& sh, const DecodeParams& p, const void* kc,
+                                const void* vc, cudaStream_t st) {
+  if (sh.num_kv_heads % 4 == 0) return launch_decode_group_t<D, G, 4, FP8>(sh, p, kc, vc, st);
+  if (sh.num_kv_heads % 2 == 0) return launch_decode_group_t<D, G, 2, FP8>(sh, p, kc, vc, st);
+  return launch_decode_group_t<D, G, 1, FP8>(sh, p, kc, vc, st);
+}
+
 template <int D, int G>
 cudaError_t launch_decode_bf16(const DecodeShape& sh, const DecodeParams& p, const void* k_cache,
                                const void* v_cache, cudaStream_t stream) {
-  if (sh.num_kv_heads % 4 == 0) return launch_decode_bf16_t<D, G, 4>(sh, p, k_cache, v_cache, stream);
-  if (sh.num_kv_heads % 2 == 0) return launch_decode_bf16_t<D, G, 2>(sh, p, k_cache, v_cache, stream);
-  return launch_decode_bf16_t<D, G, 1>(sh, p, k_cache, v_cache, stream);
+  return launch_decode_group<D, G, false>(sh, p, k_cache, v_cache, stream);
+}
+
+// E4M3 caches: head_dim 128 only.
+template <int D>
+cudaError_t dispatch_fp8(const DecodeShape& sh, const DecodeParams& p, const void* kc,
+                         const void* vc, cudaStream_t st) {
+  if constexpr (D != 128) {
+    return cudaErrorNotSupported;
+  } else {
+    switch (sh.num_heads / sh.num_kv_heads) {
+      case 1: return launch_decode_group<D, 1, true>(sh, p, kc, vc, st);
+      case 2: return launch_decode_group<D, 2, true>(sh, p, kc, vc, st);
+      case 4: return launch_decode_group<D, 4, true>(sh, p, kc, vc, st);
+      case 8: return launch_decode_group<D, 8, true>(sh, p, kc, vc, st);
+      default: return cudaErrorNotSupported;
+    }
+  }
 }
 
 template <int D>
 cudaError_t dispatch_group(const DecodeShape& sh, const DecodeParams& p, const void* kc,
                            const void* vc, cudaStream_t st) {
+  if (sh.dtype == PA_FP8_E4M3) return dispatch_fp8<D>(sh, p, kc, vc, st);
   const bool bf = sh.dtype == PA_BF16;
   switch (sh.num_heads / sh.num_kv_heads) {
     case 1: return bf ? launch_decode_bf16<D, 1>(sh, p, kc, vc, st) : launch_decode_f32<D, 1>(sh, p, kc, vc, st);
@@ -352,9 +432,12 @@ cudaError_t dispatch_group(const DecodeShape& sh, const DecodeParams& p, const v
 cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const void* k_cache,
                           const void* v_cache, const int32_t* block_tables,
                           const int32_t* context_lens, void* workspace, const void* k_new,
-                          const void* v_new, cudaStream_t stream) {
+                          const void* v_new, const float* k_scale, const float* v_scale,
+                          cudaStream_t stream) {
   DecodeParams p{};
   p.out = out;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   p.k_new = static_cast<const uint8_t*>(k_new);
   p.v_new = static_cast<const uint8_t*>(v_new);
   p.k_cache_w = static_cast<uint8_t*>(const_cast<void*>(k_cache));

@@ -15,6 +15,7 @@ import numpy as np
 import torch
 
 from oracle import attention as oatt
+from oracle import quant as oquant
 from workloads import synth
 
 TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -43,6 +44,29 @@ def assert_close(got, ref, dtype: str, what: str = ""):
     return float(err.max())
 
 
+FP8 = "fp8_e4m3"
+NAN_BITS = {torch.float32: (torch.int32, 0x7FC00000), torch.bfloat16: (torch.int16, 0x7FC0),
+            torch.uint8: (torch.uint8, 0x7F)}
+
+
+def e4m3_codes(rows: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Oracle E4M3 codes of rows [n, Hkv, d] with one scale per KV head."""
+    return np.stack([oquant.quantize(rows[:, h], scales[h]) for h in range(rows.shape[1])], axis=1)
+
+
+def e4m3_values(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Oracle cache values (float64) of codes [n, Hkv, d]."""
+    return np.stack([oquant.dequantize(codes[:, h], scales[h]) for h in range(codes.shape[1])],
+                    axis=1)
+
+
+def poison(t: torch.Tensor) -> None:
+    """Fill a cache with NaN bit patterns: any read of a row that was never
+    written (or of a slot past a sequence's end) shows up as NaN."""
+    view, bits = NAN_BITS[t.dtype]
+    t.view(view).fill_(bits)
+
+
 @dataclass
 class Case:
     cache: object          # PagedKVCache
@@ -53,6 +77,8 @@ class Case:
     out: torch.Tensor      # GPU output of the decode step
     scale: float
     dtype: str
+    k_scale: np.ndarray = None   # E4M3 caches: per-KV-head scales
+    v_scale: np.ndarray = None
 
 
 def sequence_rows(wl, s, n, prefix_rows=None):
@@ -92,8 +118,10 @@ def stage_rows(wl, device="cuda", keep=None):
 
 
 def build_case(wl, device="cuda", free_order=None, partition_size=None, share_prefix=True,
-               staged=None, keep=None, fused=True):
-    """Prefill every sequence, then one decode step (append one token each + attend)."""
+               staged=None, keep=None, fused=True, poisoned=False):
+    """Prefill every sequence, then one decode step (append one token each + attend).
+    E4M3 caches (wl.kv_dtype): rows are quantised on the device; the kept rows
+    are replaced by the oracle's cache values of the same rows."""
     from paged_kv_cache_345_b200.cache import PagedKVCache
 
     bs = wl.block_size
@@ -104,8 +132,15 @@ def build_case(wl, device="cuda", free_order=None, partition_size=None, share_pr
     if free_order is None:
         free_order = synth.block_permutation(wl.num_blocks, wl.placement_seed)
     max_blocks = max(-(-(n + 1) // bs) for n in wl.context_lens)
-    cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.dtype, device,
-                         max_blocks_per_seq=max_blocks, free_order=free_order)
+    fp8 = wl.cache_dtype == FP8
+    ks, vs = synth.e4m3_scales(wl.num_kv_heads) if fp8 else (None, None)
+    cache = PagedKVCache(wl.num_blocks, bs, wl.num_kv_heads, wl.head_dim, wl.cache_dtype, device,
+                         max_blocks_per_seq=max_blocks, free_order=free_order,
+                         k_scale=None if ks is None else torch.from_numpy(ks),
+                         v_scale=None if vs is None else torch.from_numpy(vs))
+    if poisoned:
+        poison(cache.k_cache)
+        poison(cache.v_cache)
     tdt = TORCH_DTYPES[wl.dtype]
     sk, sv, offs, rows_k, rows_v = staged if staged is not None else stage_rows(wl, device, keep)
 
@@ -137,7 +172,10 @@ def build_case(wl, device="cuda", free_order=None, partition_size=None, share_pr
     qd = torch.from_numpy(q).to(device=device, dtype=tdt)
     out = cache.decode_step(qd, k_new, v_new, seqs, wl.scale, ps, fused=fused)
     torch.cuda.synchronize()
-    return Case(cache, seqs, rows_k, rows_v, q, out, wl.scale, wl.dtype)
+    if fp8:
+        rows_k = {s: e4m3_values(e4m3_codes(r, ks), ks) for s, r in rows_k.items()}
+        rows_v = {s: e4m3_values(e4m3_codes(r, vs), vs) for s, r in rows_v.items()}
+    return Case(cache, seqs, rows_k, rows_v, q, out, wl.scale, wl.dtype, ks, vs)
 
 
 def expected_one(case: Case, s: int, j: int) -> np.ndarray:

@@ -15,6 +15,7 @@ import numpy as np
 import oracle
 from oracle import attention as oatt
 from oracle import blocks as oblk
+from oracle import quant as oq
 
 
 # ------------------------------------------------------------ block arithmetic
@@ -389,6 +390,46 @@ def check_swap_roundtrip():
     assert not back_k[0].any() and not back_v[4].any()
 
 
+
+# ---------------------------------------------------------------- E4M3 codes
+
+def check_e4m3_against_torch():
+    """Inside the finite range the encoder agrees bit for bit with torch's
+    float8_e4m3fn cast (round to nearest even), ties included."""
+    import torch
+
+    rng = np.random.default_rng(17)
+    x = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32) * 4,
+        (rng.standard_normal(2000) * 2.0 ** -8).astype(np.float32),
+        rng.uniform(-447, 447, 2000).astype(np.float32),
+        # exact ties between neighbouring codes at several exponents
+        np.array([(1 + (2 * k + 1) / 16) * 2.0 ** e for k in range(7) for e in range(-6, 8)],
+                 dtype=np.float32),
+        np.array([(2 * k + 1) * 2.0 ** -10 for k in range(8)], dtype=np.float32),
+    ])
+    x = x[np.abs(x) < 447.0]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oq.e4m3_encode(x), ref)
+
+
+def check_e4m3_hand_values():
+    cases = {1.0: 0x38, 448.0: 0x7E, 1000.0: 0x7E, -1000.0: 0xFE, 2.0 ** -9: 0x01,
+             2.0 ** -10: 0x00, 3 * 2.0 ** -10: 0x02, 1.0625: 0x38, 1.1875: 0x3A,
+             2.0 ** -6: 0x08, -3.0: 0xC4, 240.0: 0x77}
+    got = oq.e4m3_encode(np.array(list(cases), dtype=np.float32))
+    assert got.tolist() == list(cases.values())
+    assert oq.e4m3_decode(np.array([0x7E, 0x01, 0x38, 0xC4])).tolist() == [448.0, 2.0 ** -9, 1.0,
+                                                                             -3.0]
+
+
+def check_e4m3_roundtrip():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    assert np.array_equal(oq.e4m3_encode(oq.e4m3_decode(codes).astype(np.float32)), codes)
+    vals = oq.e4m3_decode(codes)
+    assert np.nanmax(vals) == 448.0 and np.nanmin(vals) == -448.0
+
+
 BLOCK_CHECKS = [
     check_seven_token_prompt, check_600_tokens, check_llama3_per_token, check_700_tokens,
     check_worked_example, check_capacity, check_worked_example_block_manager,
@@ -397,7 +438,7 @@ PLAIN_BLOCK_CHECKS = [check_sharing_and_copy_on_write, check_exhaustion_leaves_s
 ATTENTION_CHECKS = [
     check_brute_force_tiny, check_sdpa_identity_table, check_closed_forms,
     check_placement_and_sharing_invariance, check_append_and_copy_roundtrip,
-    check_swap_roundtrip,
+    check_swap_roundtrip, check_e4m3_against_torch, check_e4m3_hand_values, check_e4m3_roundtrip,
 ]
 
 assert oracle is not None

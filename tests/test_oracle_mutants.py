@@ -11,6 +11,7 @@ import pytest
 import oracle_checks as oc
 from oracle import attention as oatt
 from oracle import blocks as oblk
+from oracle import quant as oq
 
 
 def _fails_some_check(golden):
@@ -54,6 +55,16 @@ def _softmax_drop_last(q_vec, keys, values, scale):
     return (w / w.sum()) @ values
 
 
+def _e4m3_flush_subnormals(x):
+    import oracle.quant as q
+    x = np.asarray(x, dtype=np.float32)
+    out = _ORIG_E4M3(x)
+    return np.where(np.abs(x) < 2.0 ** -6, out & 0x80, out).astype(np.uint8)
+
+
+_ORIG_E4M3 = oq.e4m3_encode
+
+
 def _swap_wrong_index(dk, dv, sk, sv, mapping):
     k, v = np.array(dk, copy=True), np.array(dv, copy=True)
     for src, dst in np.asarray(mapping).reshape(-1, 2).tolist():
@@ -63,6 +74,8 @@ def _swap_wrong_index(dk, dv, sk, sv, mapping):
 
 
 MUTANTS = {
+    "e4m3_round_half_up": (oq, "_round_half_even", lambda v: np.floor(np.asarray(v) + 0.5)),
+    "e4m3_no_subnormals": (oq, "e4m3_encode", lambda x: _e4m3_flush_subnormals(x)),
     "gqa_heads_interleaved": (oatt, "kv_head_of", lambda j, g: j % g),
     "gqa_always_head0": (oatt, "kv_head_of", lambda j, g: 0),
     "offset_off_by_one": (oblk, "logical_position", lambda t, bs: (t // bs, (t + 1) % bs)),

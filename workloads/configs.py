@@ -34,6 +34,9 @@ class Workload:
     ghost_lens: tuple = field(default_factory=tuple)
     partition_size: int = 0   # 0 = let the library choose
     decode_steps: int = 1
+    # Cache element type when it differs from `dtype`: "fp8_e4m3" stores E4M3
+    # codes with per-KV-head scales (queries, new rows and output stay bf16).
+    kv_dtype: str = ""
 
     @property
     def num_seqs(self) -> int:
@@ -46,6 +49,14 @@ class Workload:
     @property
     def elem_bytes(self) -> int:
         return 4 if self.dtype == "f32" else 2
+
+    @property
+    def cache_dtype(self) -> str:
+        return self.kv_dtype or self.dtype
+
+    @property
+    def cache_elem_bytes(self) -> int:
+        return 1 if self.cache_dtype == "fp8_e4m3" else self.elem_bytes
 
 
 def tiny() -> Workload:
