@@ -363,9 +363,11 @@ cudaError_t encode_group_map(CUtensorMap* map, const void* base, const DecodeSha
 template <int D, int G, int HB, bool FP8>
 cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
                                   const void* k_cache, const void* v_cache, cudaStream_t stream) {
-  // stages: as many as fit ~112 KB of ring (two CTAs per SM), at most 4
+  // stages: as many as fit ~112 KB of ring (two CTAs per SM), at most 4; E4M3
+  // stages are half the size and its consumers hold more registers per byte,
+  // so its ring is capped at ~64 KB for three CTAs per SM
   constexpr int kStage = 2 * GroupConfig<D, G, HB, 1, FP8>::kTensorBytes;
-  constexpr int kNSfit = 114688 / kStage;
+  constexpr int kNSfit = (FP8 ? 65536 : 114688) / kStage;
   constexpr int NS = kNSfit < 2 ? 2 : (kNSfit > 4 ? 4 : kNSfit);
   using Cfg = GroupConfig<D, G, HB, NS, FP8>;
   auto kernel = pa_decode_mma_kernel<D, G, HB, NS, FP8>;
