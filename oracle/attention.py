@@ -1,4 +1,4 @@
-"""Cache writes and decode attention in float64 (oracle, test infrastructure).
+"""Cache writes, decode and prefill attention in float64 (oracle, test infrastructure).
 
 What the method computes. Paging changes where the KV cache lives, not the
 arithmetic: "PagedAttention — AI Glossary" (modelrefs.com), "Example: Where the
@@ -134,3 +134,54 @@ def swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping):
         k_out[int(dst)] = src_k[int(src)]
         v_out[int(dst)] = src_v[int(src)]
     return k_out, v_out
+
+
+def chunk_positions(length: int, n: int) -> np.ndarray:
+    """Absolute positions of a sequence's last n tokens (its query chunk)."""
+    return length - n + np.arange(n)
+
+
+def causal_visible(length: int, positions: np.ndarray) -> np.ndarray:
+    """[n, length] mask: row i sees key t iff t <= positions[i]."""
+    return np.arange(length)[None, :] <= np.asarray(positions)[:, None]
+
+
+def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale: float,
+            block_size: int):
+    """Causal attention of a chunk of new queries per sequence over its paged
+    context (chunked prefill; a whole prompt is the chunk that starts at 0).
+
+    "Paged Attention" (klaylearn.com glossary), definition: prefill fills blocks
+    as the prompt's tokens produce K and V, and attention reads the context
+    through the table; "What is paged attention in vLLM...", Steps 3-4 (the
+    prompt's blocks, then decoding). Reading taken (the pages do not spell out
+    prefill attention): the chunk's K/V are already in the cache; sequence s
+    has L = context_lens[s] tokens, its n = query_start[s+1] - query_start[s]
+    query rows are its last n positions, and row i (position p = L - n + i)
+    attends the keys t <= p, each query head j through KV head j // G.
+
+    q: [total_q, Hq, d] with sequence s's rows at query_start[s] .. query_start[s+1] - 1.
+    Returns [total_q, Hq, d] float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    total_q, num_heads, head_dim = q.shape
+    num_kv_heads = k_cache.shape[2]
+    group = num_heads // num_kv_heads
+    out = np.zeros((total_q, num_heads, head_dim), dtype=np.float64)
+    for s in range(len(context_lens)):
+        r0, r1 = int(query_start[s]), int(query_start[s + 1])
+        n, length = r1 - r0, int(context_lens[s])
+        if n == 0:
+            continue
+        keys = gather_context(k_cache, block_tables[s], length, block_size)
+        values = gather_context(v_cache, block_tables[s], length, block_size)
+        pos = chunk_positions(length, n)
+        visible = causal_visible(length, pos)
+        for j in range(num_heads):
+            h = kv_head_of(j, group)
+            x = scale * (q[r0:r1, j, :] @ keys[:, h, :].T)    # [n, L] scores
+            x = np.where(visible, x, -np.inf)
+            w = np.exp(x - x.max(axis=1, keepdims=True))
+            w = w / w.sum(axis=1, keepdims=True)
+            out[r0:r1, j, :] = w @ values[:, h, :]
+    return out

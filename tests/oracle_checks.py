@@ -430,6 +430,99 @@ def check_e4m3_roundtrip():
     assert np.nanmax(vals) == 448.0 and np.nanmin(vals) == -448.0
 
 
+# ------------------------------------------------------------------ prefill
+
+def _prefill_case(rng, lens, chunks, hq=4, hkv=2, d=16, bs=4, shuffle=True):
+    nb = sum(-(-n // bs) for n in lens) + 3
+    kc = rng.standard_normal((nb, bs, hkv, d))
+    vc = rng.standard_normal((nb, bs, hkv, d))
+    ids = rng.permutation(nb) if shuffle else np.arange(nb)
+    mb = max(-(-n // bs) for n in lens)
+    tables = np.zeros((len(lens), mb), dtype=np.int64)
+    k = 0
+    for s, n in enumerate(lens):
+        nbk = -(-n // bs)
+        tables[s, :nbk] = ids[k:k + nbk]
+        k += nbk
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int64)
+    q = rng.standard_normal((int(qs[-1]), hq, d))
+    return q, kc, vc, tables, qs
+
+
+def check_prefill_single_query_is_decode():
+    """A one-token chunk is the decode step: it sees the whole context."""
+    rng = np.random.default_rng(31)
+    lens = [1, 5, 13, 40]
+    q, kc, vc, tables, qs = _prefill_case(rng, lens, [1, 1, 1, 1])
+    got = oatt.prefill(q, kc, vc, tables, lens, qs, 0.3, 4)
+    ref = oatt.decode(q, kc, vc, tables, lens, 0.3, 4)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def check_prefill_full_matches_causal_sdpa():
+    """A whole prompt (chunk = context) against torch's float64 causal attention."""
+    import torch
+
+    rng = np.random.default_rng(32)
+    L, hq, hkv, d, bs = 37, 8, 2, 16, 4
+    q, kc, vc, tables, qs = _prefill_case(rng, [L], [L], hq, hkv, d, bs, shuffle=False)
+    got = oatt.prefill(q, kc, vc, tables, [L], qs, 0.25, bs)
+    keys = kc.reshape(-1, hkv, d)[:L]
+    vals = vc.reshape(-1, hkv, d)[:L]
+    g = hq // hkv
+    tq = torch.from_numpy(q).permute(1, 0, 2)                         # [Hq, L, d]
+    tk = torch.from_numpy(keys).permute(1, 0, 2).repeat_interleave(g, 0)
+    tv = torch.from_numpy(vals).permute(1, 0, 2).repeat_interleave(g, 0)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
+                                                           scale=0.25)
+    assert np.allclose(got, ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+def check_prefill_first_row_and_chunks():
+    """Row 0 of a prompt sees only itself (its value row exactly); a chunk is
+    the matching suffix of the whole prompt's rows, wherever the blocks sit."""
+    rng = np.random.default_rng(33)
+    L, n = 29, 6
+    q, kc, vc, tables, qs = _prefill_case(rng, [L], [L])
+    full = oatt.prefill(q, kc, vc, tables, [L], qs, 0.4, 4)
+    v0 = oatt.gather_context(vc, tables[0], 1, 4)[0]
+    for j in range(q.shape[1]):
+        assert np.array_equal(full[0, j], v0[j // 2])
+    chunk = oatt.prefill(q[L - n:], kc, vc, tables, [L], np.array([0, n]), 0.4, 4)
+    assert np.allclose(chunk, full[L - n:], rtol=0, atol=1e-12)
+    # identical logical contents in other physical blocks
+    perm = rng.permutation(kc.shape[0])
+    inv = np.argsort(perm)
+    kc2, vc2 = kc[perm], vc[perm]
+    tables2 = inv[tables]
+    moved = oatt.prefill(q, kc2, vc2, tables2, [L], qs, 0.4, 4)
+    assert np.array_equal(moved, full)
+
+
+def check_prefill_brute_force():
+    """Python loops and math.exp on a tiny chunked case."""
+    import math
+
+    rng = np.random.default_rng(34)
+    lens, chunks = [6, 9], [2, 4]
+    q, kc, vc, tables, qs = _prefill_case(rng, lens, chunks, hq=2, hkv=1, d=3, bs=2)
+    got = oatt.prefill(q, kc, vc, tables, lens, qs, 0.7, 2)
+    for s, (L, n) in enumerate(zip(lens, chunks)):
+        for i in range(n):
+            p = L - n + i
+            for j in range(2):
+                xs = []
+                for t in range(p + 1):
+                    blk, off = tables[s][t // 2], t % 2
+                    xs.append(0.7 * sum(q[qs[s] + i, j, c] * kc[blk, off, 0, c] for c in range(3)))
+                m = max(xs)
+                w = [math.exp(x - m) for x in xs]
+                tot = sum(w)
+                for c in range(3):
+                    ref = sum(w[t] * vc[tables[s][t // 2], t % 2, 0, c] for t in range(p + 1)) / tot
+                    assert abs(got[qs[s] + i, j, c] - ref) < 1e-12
+
+
 BLOCK_CHECKS = [
     check_seven_token_prompt, check_600_tokens, check_llama3_per_token, check_700_tokens,
     check_worked_example, check_capacity, check_worked_example_block_manager,
@@ -439,6 +532,8 @@ ATTENTION_CHECKS = [
     check_brute_force_tiny, check_sdpa_identity_table, check_closed_forms,
     check_placement_and_sharing_invariance, check_append_and_copy_roundtrip,
     check_swap_roundtrip, check_e4m3_against_torch, check_e4m3_hand_values, check_e4m3_roundtrip,
+    check_prefill_single_query_is_decode, check_prefill_full_matches_causal_sdpa,
+    check_prefill_first_row_and_chunks, check_prefill_brute_force,
 ]
 
 assert oracle is not None

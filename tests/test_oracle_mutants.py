@@ -74,6 +74,11 @@ def _swap_wrong_index(dk, dv, sk, sv, mapping):
 
 
 MUTANTS = {
+    "prefill_diagonal_hidden": (oatt, "causal_visible",
+                                lambda L, pos: np.arange(L)[None, :] < np.asarray(pos)[:, None]),
+    "prefill_unmasked": (oatt, "causal_visible",
+                         lambda L, pos: np.ones((len(pos), L), dtype=bool)),
+    "prefill_positions_from_zero": (oatt, "chunk_positions", lambda L, n: np.arange(n)),
     "e4m3_round_half_up": (oq, "_round_half_even", lambda v: np.floor(np.asarray(v) + 0.5)),
     "e4m3_no_subnormals": (oq, "e4m3_encode", lambda x: _e4m3_flush_subnormals(x)),
     "gqa_heads_interleaved": (oatt, "kv_head_of", lambda j, g: j % g),
