@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="llama3_8b_layer",
                     choices=["llama3_8b_layer", "large_batch", "shared_prefix", "long_context",
-                             "swap"])
+                             "swap", "prefill", "chunked_prefill"])
     ap.add_argument("--placement", choices=["random", "identity"], default="random",
                     help="physical block order: a seeded permutation (default) or identity "
                          "(each sequence's blocks contiguous in memory)")
@@ -702,11 +702,182 @@ def run_swap(args, rank, world, local_rank):
             "directions": res, "gpu_launches": 2 * args.steps}), flush=True)
 
 
+# ------------------------------------------------------------------ prefill
+
+PREFILL_METRIC = "paged causal prefill attention TFLOP/s (fraction of bf16 tensor peak)"
+
+
+def prefill_shape(name: str):
+    """(cached tokens before the chunk, chunk tokens) per sequence: the worked
+    example's eight prompts prefilled whole, or a 512-token chunk on top of
+    each of those contexts."""
+    from workloads import synth
+
+    lens = list(synth.LLAMA3_8B_BATCH_LENGTHS)
+    if name == "prefill":
+        return [0] * len(lens), lens
+    return lens, [512] * len(lens)
+
+
+def prefill_flops(before, chunks, num_heads=32, head_dim=128) -> float:
+    """q.k and p.v multiply-adds over every (query row, visible key) pair, all heads."""
+    pairs = sum(c * (b + 1) + c * (c - 1) // 2 for b, c in zip(before, chunks))
+    return 4.0 * head_dim * num_heads * pairs
+
+
+def run_prefill(args, rank, world, local_rank):
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+    from paged_kv_cache_345_b200.cache import PagedKVCache
+    from workloads import synth
+
+    hq, hkv, d, bs, seed = 32, 8, 128, args.block_size, 1007
+    before, chunks = prefill_shape(args.workload)
+    lens = [b + c for b, c in zip(before, chunks)]
+    flops = prefill_flops(before, chunks, hq, d)
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    total_q = int(qs[-1])
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from oracle import attention as oatt
+        # bounded sample: the 700-token sequence alone, float64 NumPy, whole steps
+        s = 1
+        k, v = synth.kv_rows(seed, s, lens[s], hkv, d)
+        q1 = synth.queries(seed, 1 + s, chunks[s], hq, d)
+        kc, vc = k[:, None], v[:, None]
+        tables = np.arange(lens[s])[None]
+        f1 = prefill_flops([before[s]], [chunks[s]], hq, d)
+        for _ in range(max(1, args.warmup)):
+            oatt.prefill(q1, kc, vc, tables, [lens[s]], [0, chunks[s]], 1 / np.sqrt(d), 1)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oatt.prefill(q1, kc, vc, tables, [lens[s]], [0, chunks[s]], 1 / np.sqrt(d), 1)
+        dt = time.perf_counter() - t0
+        value = f1 * args.steps / dt / 1e12
+        print(json.dumps({
+            "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample": f"sequence {s} only"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+                             "kind": "oracle", "sample": f"sequence {s} ({chunks[s]} rows)"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
+    nb = sum(-(-L // bs) for L in lens) + 16
+    cache = PagedKVCache(nb, bs, hkv, d, "bf16", device, max_blocks_per_seq=max(-(-L // bs) for L in lens),
+                         free_order=synth.block_permutation(nb, 2007))
+    seqs = [cache.add_sequence() for _ in lens]
+    for s, L in enumerate(lens):   # every token's K/V, chunk included, written through the library
+        k, v = synth.kv_rows(seed, s, L, hkv, d)
+        cache.write([seqs[s]], [L], torch.from_numpy(k).to(device, torch.bfloat16),
+                    torch.from_numpy(v).to(device, torch.bfloat16))
+    q_host = torch.from_numpy(np.concatenate(
+        [synth.queries(seed, 1 + s, c, hq, d) for s, c in enumerate(chunks)])).to(torch.bfloat16)
+    q_host = q_host.pin_memory()
+    q = q_host.to(device)
+    out = torch.empty_like(q)
+    out_host = torch.empty_like(q_host).pin_memory()
+    tables, ctx, _ = cache.tables(seqs)
+    qs_dev = torch.from_numpy(qs).to(device)
+    torch.cuda.synchronize(device)
+    lib = pa._lib
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = ctypes.c_void_p(stream.cuda_stream)
+    call_args = (ptr(out), ptr(q), ptr(cache.k_cache), ptr(cache.v_cache), ptr(tables), ptr(ctx),
+                 ptr(qs_dev), len(lens), total_q, hq, hkv, d, bs, nb, tables.shape[1],
+                 int(max(chunks)), 1 / float(np.sqrt(d)), pa.PA_BF16, st)
+
+    def step():
+        if lib.pa_prefill(*call_args):
+            raise RuntimeError(f"pa_prefill: {lib.pa_last_error().decode()}")
+
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush_w = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
+    flush_r = torch.ones((2 * l2 + (64 << 20)) // 4, dtype=torch.float32, device=device)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(device)
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    torch.cuda.synchronize(device)
+    for i in range(args.steps):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(ms), world, device)
+    e2e = None
+    if not args.no_e2e:
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush()
+            ee[i][0].record(stream)
+            q.copy_(q_host, non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+            ee[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee), world, device)
+        nbytes = q_host.numel() * 2
+        e2e = {"value": whole_job_rate(flops, args.steps, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "ms_per_step": e2e_ms / args.steps}
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        peak, src = float(json.load(open(peaks_path))["bf16_tflops"]), "measured bf16_tflops (burst)"
+    else:
+        peak, src = 1590.0, "fallback"
+    achieved = flops / (statistics.mean(ms) * 1e-3) / 1e12
+    value = whole_job_rate(flops, args.steps, world, total_ms) / 1e12
+    if rank == 0:
+        print(json.dumps({
+            "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "num_seqs": len(lens), "cached_before": before,
+                       "chunk_tokens": chunks, "num_heads": hq, "num_kv_heads": hkv,
+                       "head_dim": d, "block_size": bs, "causal_flops_per_step": flops,
+                       "l2": "flushed between steps (outside the timed events)"},
+            "step_us_p10_p50_p90": [1e3 * float(np.percentile(ms, p)) for p in (10, 50, 90)],
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "pa_prefill_kernel",
+                         "peak_source": src},
+            "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     rank, world, local_rank = dist_env()
+    if args.workload in ("prefill", "chunked_prefill"):
+        run_prefill(args, rank, world, local_rank)
+        return
     if args.workload == "swap":
         if args.impl == "reference":
             if rank == 0:

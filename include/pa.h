@@ -289,6 +289,40 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                          pa_stream_t stream);
 
 /*
+ * pa_prefill — causal attention of each sequence's newest chunk of query rows
+ * over its paged context (prompt prefill, or chunked prefill on top of an
+ * already-cached prefix). "Paged Attention" (klaylearn.com glossary),
+ * definition: during prefill blocks are filled as prompt tokens produce K and
+ * V, and attention reads the context through the block table; "What is paged
+ * attention in vLLM, and why does it matter?", Steps 3-4. The chunk's own K
+ * and V must already be in the cache (pa_kv_append). For sequence s with
+ * L = context_lens[s] cached tokens and n = query_start[s+1] - query_start[s]
+ * query rows, row i is position p = L - n + i and, for query head j
+ * (KV head h = j / (num_heads / num_kv_heads)),
+ *     out[row][j] = sum_{t <= p} softmax_t(scale * q[row][j] . K_s[t][h]) V_s[t][h]
+ * with K_s[t] read through block_tables[s] as in pa_decode.
+ *
+ *   out, q         device, bf16 [total_q][num_heads][head_dim]; sequence s's
+ *                  rows are query_start[s] .. query_start[s+1] - 1.
+ *   query_start    device, int32 [num_seqs + 1], non-decreasing, from 0 to at
+ *                  most total_q; 0 <= n <= context_lens[s] for every s, else
+ *                  PA_DEVERR_CONTEXT is set and that sequence is skipped.
+ *   max_query_len  host upper bound of n over the batch (sizes the grid).
+ *   Everything else as pa_decode. Products in bf16 on the tensor cores
+ *   (tcgen05), softmax and accumulation in fp32; softmax weights are rounded to
+ *   bf16 before the product with V.
+ * Supported: dtype PA_BF16; head_dim 128; num_heads / num_kv_heads in
+ * {1, 2, 4, 8}; block_size a power of two in [8, 256]. The result does not
+ * depend on block_size or on the physical placement of the blocks.
+ */
+int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* block_tables, const int32_t* context_lens,
+               const int32_t* query_start, int num_seqs, int total_q, int num_heads,
+               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               int max_blocks_per_seq, int max_query_len, float scale, pa_dtype dtype,
+               pa_stream_t stream);
+
+/*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
  * The pages have no counterpart: this is an interface convenience of this
  * library, not part of the method.

@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
   pa_swap_blocks   copy blocks between device and (pinned) host pools
   pa_decode        paged decode attention (split-K over partitions)
   pa_decode_append one decode step: append each newest token, then attend
+  pa_prefill       causal (chunked) prefill attention over the paged context
   pa_kv_append_fp8, pa_decode_fp8, pa_decode_append_fp8
                    the same over 8-bit E4M3 caches with per-KV-head scales
   BlockManager     host free list + reference counts + block tables
@@ -30,6 +31,7 @@ __all__ = [
     "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
     "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode",
     "pa_decode_append", "pa_kv_append_fp8", "pa_decode_fp8", "pa_decode_append_fp8", "PA_FP8_E4M3",
+    "pa_prefill",
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
 ]
@@ -74,6 +76,8 @@ _sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, 
      _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
 _sig("pa_decode_append_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
      _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
+_sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+     _i32, _i32, _f32, _i32, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _f32, _i32, _i32, _vp)
 _sig("pa_decode_noalloc_scratch_bytes", _sz)
@@ -105,7 +109,7 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 EXPORTED = (
     "pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_swap_blocks",
     "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode", "pa_decode_append",
-    "pa_decode_fp8", "pa_decode_append_fp8", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
+    "pa_decode_fp8", "pa_decode_append_fp8", "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
     "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
@@ -373,6 +377,32 @@ def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scal
         _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
         a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"],
         *a["sizes"], int(max_context_len), float(scale), int(partition_size), *a["ws"],
+        _stream(stream, q.device)))
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+               max_query_len: int, scale: float, stream=None) -> None:
+    """Causal attention of each sequence's newest query rows over its paged context.
+
+    q, out: bf16 [total_q, Hq, 128]; sequence s's rows are query_start[s] ..
+    query_start[s+1] - 1 (int32 [S + 1], device) and are its last positions; the
+    chunk's K/V must already be in the caches. See pa_prefill in include/pa.h.
+    """
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    total_q, hq, dq = q.shape
+    s = context_lens.shape[0]
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or query_start.shape != (s + 1,):
+        raise ValueError("block_tables must be [S, max_blocks], query_start [S + 1]")
+    bf = torch.bfloat16
+    _check(_lib.pa_prefill(
+        _dev_ptr(out, "out", bf), _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf),
+        _dev_ptr(v_cache, "v_cache", bf), _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(context_lens, "context_lens", torch.int32),
+        _dev_ptr(query_start, "query_start", torch.int32), s, total_q, hq, hkv, d, bs, nb,
+        block_tables.shape[1], int(max_query_len), float(scale), PA_BF16,
         _stream(stream, q.device)))
 
 

@@ -7,6 +7,9 @@ workspace. Each method marshals arguments and calls libpa.so:
   write(seq_ids, counts, k_rows, v_rows)  reserve slots (native), copy shared
       tail blocks first when needed (pa_copy_blocks), then scatter the rows
       (pa_kv_append). Serves both prefill (many tokens) and decode (one token).
+  prefill(q, k_rows, v_rows, seq_ids, counts)  append each sequence's chunk
+      of counts[i] tokens (write), then causal attention of the chunk's query
+      rows over the whole context (pa_prefill); bf16 caches.
   decode(q, seq_ids)  block tables to the device, then pa_decode.
   decode_step(q, k_new, v_new, seq_ids)  one decode step: reserve each sequence's
       next slot (native; shared tail blocks copied first), then pa_decode_append
@@ -30,7 +33,7 @@ import torch
 
 from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_decode_append_fp8,
                pa_decode_fp8, pa_decode_partition_size, pa_decode_workspace_bytes, pa_kv_append,
-               pa_kv_append_fp8)
+               pa_kv_append_fp8, pa_prefill)
 
 _TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}
 
@@ -93,6 +96,21 @@ class PagedKVCache:
                 pa_kv_append(k_rows, v_rows, self._to_device(slots), self.k_cache, self.v_cache,
                              stream=self.stream)
         return slots
+
+    # -------------------------------------------------------------- prefill
+    def prefill(self, q, k_rows, v_rows, seq_ids, counts, scale: float | None = None, out=None):
+        """Append counts[i] tokens to seq_ids[i] and attend them causally: q, k_rows,
+        v_rows are [sum(counts), H, d] device tensors in sequence order."""
+        if self.fp8:
+            raise NotImplementedError("pa_prefill reads bf16 caches")
+        self.write(seq_ids, counts, k_rows, v_rows)
+        block_tables, context_lens, _ = self.tables(seq_ids)
+        qs = np.concatenate([[0], np.cumsum(np.asarray(counts, dtype=np.int64))]).astype(np.int32)
+        out = torch.empty_like(q) if out is None else out
+        scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+        pa_prefill(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                   self._to_device(qs), int(max(counts, default=0)), scale, stream=self.stream)
+        return out
 
     # --------------------------------------------------------------- decode
     def tables(self, seq_ids, max_blocks_per_seq: int | None = None):

@@ -360,6 +360,62 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                        PA_FP8_E4M3, k_new, v_new, k_scale, v_scale, stream);
 }
 
+int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* block_tables, const int32_t* context_lens,
+               const int32_t* query_start, int num_seqs, int total_q, int num_heads,
+               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               int max_blocks_per_seq, int max_query_len, float scale, pa_dtype dtype,
+               pa_stream_t stream) {
+  if (num_seqs < 0 || total_q < 0 || max_query_len < 0)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: negative size");
+  if (num_seqs == 0 || total_q == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: null pointer");
+  if (dtype != PA_BF16) return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: dtype %d (built: bf16)", dtype);
+  if (head_dim != 128)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: head_dim %d (built: 128)", head_dim);
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: num_heads %d not a multiple of num_kv_heads %d",
+                   num_heads, num_kv_heads);
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: group size %d (built: 1, 2, 4, 8)", group);
+  if (!pow2(block_size) || block_size < 8 || block_size > 256)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: block_size %d (built: powers of two 8..256)",
+                   block_size);
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: num_blocks and max_blocks_per_seq must be > 0");
+  if (max_query_len > total_q)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: max_query_len %d > total_q %d", max_query_len,
+                   total_q);
+  if (!std::isfinite(scale)) return pa_fail(PA_ERR_INVALID, "pa_prefill: scale not finite");
+  const int tok = 128 / group;
+  if (num_seqs > 65535 || (max_query_len + tok - 1) / tok > 65535 || num_kv_heads > 65535)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: grid too large");
+  if (static_cast<int64_t>(num_blocks) * block_size * num_kv_heads * head_dim * 2 / 16 >
+      (int64_t(1) << 36))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: cache larger than 1 TiB");
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: misaligned pointer");
+  pa::PrefillShape sh{};
+  sh.num_seqs = num_seqs;
+  sh.total_q = total_q;
+  sh.num_heads = num_heads;
+  sh.num_kv_heads = num_kv_heads;
+  sh.head_dim = head_dim;
+  sh.block_size = block_size;
+  sh.num_blocks = num_blocks;
+  sh.max_blocks_per_seq = max_blocks_per_seq;
+  sh.max_query_len = max_query_len;
+  sh.scale = scale;
+  cudaError_t e = pa::launch_prefill(sh, out, q, k_cache, v_cache, block_tables, context_lens,
+                                     query_start, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: no kernel for this shape");
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_prefill launch", e);
+}
+
 int pa_device_errors(pa_stream_t stream, unsigned int* flags) {
   unsigned int* word = nullptr;
   cudaError_t e = pa::device_error_word(&word);

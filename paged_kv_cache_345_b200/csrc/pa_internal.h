@@ -59,6 +59,17 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
                           const int32_t* context_lens, void* workspace, const void* k_new,
                           const void* v_new, const float* k_scale, const float* v_scale,
                           cudaStream_t stream);
+// Sizes of one pa_prefill call after validation.
+struct PrefillShape {
+  int num_seqs, total_q, num_heads, num_kv_heads, head_dim, block_size, num_blocks;
+  int max_blocks_per_seq, max_query_len;
+  float scale;
+};
+// Causal chunked-prefill attention (pa_prefill.cu); bf16, head_dim 128.
+cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* block_tables,
+                           const int32_t* context_lens, const int32_t* query_start,
+                           cudaStream_t stream);
 // Device error word of the current device (address in device memory).
 cudaError_t device_error_word(unsigned int** ptr);
 

@@ -249,8 +249,7 @@ cudaError_t launch_swap_blocks(void* dst_k, void* dst_v, const void* src_k, cons
 
 // ------------------------------------------------------------------ decode
 
-namespace {
-
+// cuTensorMapEncodeTiled from the driver, looked up once (also used by pa_prefill.cu).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -264,6 +263,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   });
   return fn;
 }
+
+namespace {
 
 // 4-D view of a cache [num_blocks][block_size][num_kv_heads][head_dim]; a box is
 // `box_rows` consecutive tokens of one block for one KV head and `box_cols`
