@@ -311,9 +311,10 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
  *   Everything else as pa_decode. Products in bf16 on the tensor cores
  *   (tcgen05), softmax and accumulation in fp32; softmax weights are rounded to
  *   bf16 before the product with V.
- * Supported: dtype PA_BF16; head_dim 128; num_heads / num_kv_heads in
- * {1, 2, 4, 8}; block_size a power of two in [8, 256]. The result does not
- * depend on block_size or on the physical placement of the blocks.
+ * scale must be finite and > 0. Supported: dtype PA_BF16; head_dim 128;
+ * num_heads / num_kv_heads in {1, 2, 4, 8}; block_size a power of two in
+ * [8, 256]. The result does not depend on block_size or on the physical
+ * placement of the blocks.
  */
 int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                const int32_t* block_tables, const int32_t* context_lens,

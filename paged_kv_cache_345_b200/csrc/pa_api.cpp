@@ -388,8 +388,9 @@ int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cach
   if (max_query_len > total_q)
     return pa_fail(PA_ERR_INVALID, "pa_prefill: max_query_len %d > total_q %d", max_query_len,
                    total_q);
-  if (!std::isfinite(scale)) return pa_fail(PA_ERR_INVALID, "pa_prefill: scale not finite");
-  const int tok = 128 / group;
+  if (!std::isfinite(scale) || scale <= 0.0f)
+    return pa_fail(PA_ERR_INVALID, "pa_prefill: scale must be finite and > 0");
+  const int tok = 256 / group;  // query tokens per CTA
   if (num_seqs > 65535 || (max_query_len + tok - 1) / tok > 65535 || num_kv_heads > 65535)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: grid too large");
   if (static_cast<int64_t>(num_blocks) * block_size * num_kv_heads * head_dim * 2 / 16 >

@@ -9,24 +9,29 @@
 // n positions, and row i (position p = L - n + i) attends keys t <= p with
 // softmax(scale * q . k) weights, query head j reading KV head j / G.
 //
-// Layout and pipeline (one CTA = one KV head x 128 query rows x one sequence):
-//  * The 128 rows are 128 / G tokens x the G query heads of the KV head
-//    (row = token * G + g), so every K/V tile is loaded once for the group.
-//  * Warp 0 (producer): TMA loads Q once, then per tile of 128 keys one box
-//    per cache block {64 columns, min(block_size, 128) tokens} for each half of
-//    head_dim, for K and for V, into a 2-stage ring. Boxes use the 128-byte
-//    swizzle, which is the shared-memory operand layout of the MMA.
-//  * Warp 1 (MMA): one thread issues tcgen05.mma. S_j = Q K_j^T (M 128, N 128,
-//    K 128) goes to one of two tensor-memory buffers, so S_{j+1} runs while the
-//    softmax warps read S_j; O += P_j V_j accumulates in tensor memory (V is
-//    the MN-major operand, P the K-major one). Completion is signalled to
-//    mbarriers with tcgen05.commit.
-//  * Warps 2-5 (softmax): thread = row (tensor-memory lane). Per tile: load the
-//    row of S, scale by scale * log2(e), mask keys past the row's position,
-//    online softmax in base 2, write P (bf16) into shared memory in the swizzled
-//    K-major layout, and when the row maximum grew rescale the row of O in
-//    tensor memory (after the previous P V finished). The end divides by the
-//    row sum and stores bf16.
+// Layout and pipeline. One CTA = one sequence x one KV head x two query tiles
+// of 128 rows (each 128 / G tokens x the G query heads of the KV head, row =
+// token * G + g). Both tiles share every K/V tile, which halves the K/V bytes
+// per flop: with one 128-row tile per CTA the kernel was bound by L2-to-SM
+// bandwidth, not by the tensor cores. The grid counts tiles from each
+// sequence's end, so the tiles that see the most keys start first.
+//  * Warp 0 (producer): TMA loads both Q tiles once, then per tile of 64 keys
+//    one box per cache block {64 columns, min(block_size, 64) tokens} for each
+//    half of head_dim, for K and for V, into a 3-stage ring. Boxes use the
+//    128-byte swizzle, which is the shared-memory operand layout of the MMA.
+//  * Warp 1 (MMA): one thread issues tcgen05.mma. For key tile j+1 it issues
+//    S_x = Q_x K^T (M 128, N 64, K 128) for both query tiles x into
+//    double-buffered tensor memory, then O_x += P_x V (M 128, N 128, K 64) for
+//    tile j as each P_x becomes ready (V is the MN-major operand, P the K-major
+//    one). Completion is signalled to mbarriers with tcgen05.commit.
+//  * Warps 2-5 and 6-9 (softmax, one warpgroup per query tile): thread = row
+//    (tensor-memory lane). Per key tile: load the row of S, mask keys past the
+//    row's position, exponentials in base 2 against a reference maximum that
+//    moves only when the row maximum exceeds it by 2^8 (so O is rarely
+//    rescaled; numerator and denominator share it), computed while the
+//    previous P V runs; then write P (bf16) into shared memory in the swizzled
+//    K-major layout and, if the reference moved, rescale the row of O in
+//    tensor memory. The end divides by the row sum and stores bf16.
 //  * Results depend only on the logical key tiles, so they are bit-identical
 //    across block sizes and placements.
 #include <cudaTypedefs.h>
@@ -59,23 +64,35 @@ struct PrefillParams {
 
 template <int G>
 struct PrefillConfig {
-  static constexpr int kRows = 128;             // query rows per CTA (MMA M)
-  static constexpr int kKeys = 128;             // keys per tile (MMA N of S, K of P V)
-  static constexpr int kD = 128;                // head_dim
-  static constexpr int kTok = kRows / G;        // query tokens per CTA
-  static constexpr int kTile = kRows * kD * 2;  // one bf16 128 x 128 operand: 32 KB
-  static constexpr int kHalf = kTile / 2;       // 64 columns of it: 16 KB
-  static constexpr int kQ = 0, kP = kTile, kStage0 = 2 * kTile;
-  static constexpr int kNS = 2;                 // K/V stages
-  static constexpr int kBars = kStage0 + kNS * 2 * kTile;
-  static constexpr int kSmemBytes = kBars + 256 + 1024;  // + 1024-byte alignment slack
-  static constexpr int kThreads = 192;
-  static constexpr uint32_t kTmemCols = 512;    // S0, S1, O (128 columns each)
+  static constexpr int kRows = 128;                  // rows of one query tile (MMA M)
+  static constexpr int kQT = 2;                      // query tiles per CTA
+  static constexpr int kKeys = 64;                   // keys per K/V tile
+  static constexpr int kD = 128;                     // head_dim
+  static constexpr int kTok = kRows / G;             // tokens per query tile
+  static constexpr int kQBytes = kRows * kD * 2;     // a Q tile: two 64-column halves of 16 KB
+  static constexpr int kQHalf = kQBytes / 2;
+  static constexpr int kKVBytes = kKeys * kD * 2;    // a K or V tile: two halves of 8 KB
+  static constexpr int kKVHalf = kKVBytes / 2;
+  static constexpr int kPBytes = kRows * kKeys * 2;  // a P tile: one 16 KB swizzle atom wide
+  static constexpr int kNS = 3;                      // K/V stages
+  static constexpr int kQ = 0, kP = kQT * kQBytes, kStage0 = kP + kQT * kPBytes;
+  static constexpr int kBars = kStage0 + kNS * 2 * kKVBytes;
+  static constexpr int kSmemBytes = kBars + 256;     // the base is 1024-byte aligned
+  static constexpr int kThreads = 320;               // producer, MMA, 2 x 4 softmax warps
+  static constexpr uint32_t kTmemCols = 512;         // S[x][2] (64 each), O[x] (128 each)
   static_assert(kRows % G == 0, "group must divide the row tile");
 };
 
 // mbarrier slots
-enum : int { kQFull = 0, kKVFull = 1, kKVEmpty = 3, kSFull = 5, kPFull = 7, kODone = 8 };
+enum : int {
+  kQFull = 0,
+  kKVFull = 1,    // [kNS]
+  kKVEmpty = 4,   // [kNS]
+  kSFull = 7,     // [query tile][2]
+  kPFull = 11,    // [query tile]
+  kODone = 13,    // [query tile]
+  kNumBars = 15
+};
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint32_t bar) {
@@ -86,24 +103,33 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 2^x by the MUFU unit (approximate; results below 2^-126 flush to 0, -inf gives 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int G>
 __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     pa_prefill_kernel(const __grid_constant__ CUtensorMap q_map,
                       const __grid_constant__ CUtensorMap k_map,
                       const __grid_constant__ CUtensorMap v_map, const PrefillParams p) {
   using Cfg = PrefillConfig<G>;
-  constexpr int TOK = Cfg::kTok, HALF = Cfg::kHalf;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
+  constexpr int TOK = Cfg::kTok, QHALF = Cfg::kQHalf, KVHALF = Cfg::kKVHalf, KEYN = Cfg::kKeys;
+  constexpr int NS = Cfg::kNS;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kBars + 128);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  const uint32_t q_s = smem_u32(sm + Cfg::kQ), p_s = smem_u32(sm + Cfg::kP);
-  auto k_s = [&](int st) { return smem_u32(sm + Cfg::kStage0 + st * 2 * Cfg::kTile); };
-  auto v_s = [&](int st) { return k_s(st) + Cfg::kTile; };
+  auto q_s = [&](int x) { return smem_u32(sm + Cfg::kQ + x * Cfg::kQBytes); };
+  auto p_s = [&](int x) { return smem_u32(sm + Cfg::kP + x * Cfg::kPBytes); };
+  auto k_s = [&](int st) { return smem_u32(sm + Cfg::kStage0 + st * 2 * Cfg::kKVBytes); };
+  auto v_s = [&](int st) { return k_s(st) + Cfg::kKVBytes; };
 
-  const int h = blockIdx.x, qt = blockIdx.y, s = blockIdx.z;
+  // grid (sequence, KV head, pair of query tiles counted from the end)
+  const int s = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bs = p.block_size, lg = p.log2_block_size;
   // every lane polls; the warp proceeds only if all saw the phase complete
@@ -119,26 +145,34 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   const int n = q1 - q0;
   if (q0 < 0 || q1 > p.total_q || n < 0 || L < n ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
-    if (threadIdx.x == 0 && h == 0 && qt == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+    if (threadIdx.x == 0 && h == 0 && blockIdx.z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
     return;
   }
-  const int tq0 = qt * TOK;
-  if (tq0 >= n) return;                      // no rows of this sequence in the tile
-  const int ntok = min(TOK, n - tq0);        // valid query tokens in the tile
-  const int pos0 = L - n + tq0;              // position of the tile's first token
-  const int pos_last = pos0 + ntok - 1;      // <= L - 1
-  const int nt = pos_last / Cfg::kKeys + 1;  // key tiles to visit
+  constexpr int CTOK = Cfg::kQT * TOK;  // tokens per CTA
+  const int npairs = (n + CTOK - 1) / CTOK;
+  if (static_cast<int>(blockIdx.z) >= npairs) return;  // no rows of this sequence here
+  const int tq0 = (npairs - 1 - static_cast<int>(blockIdx.z)) * CTOK;
+  const int ntok_all = min(CTOK, n - tq0);
+  const int pos_last = L - n + tq0 + ntok_all - 1;  // <= L - 1
+  const int nt = pos_last / KEYN + 1;                // key tiles to visit
+  if (smem_u32(sm) & 1023) {                         // the swizzled operand layout needs this
+    if (threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+    return;
+  }
   const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kQFull), 1);
-    for (int i = 0; i < Cfg::kNS; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(bar(kKVFull + i), 1);   // producer arrival + TMA bytes
-      mbar_init(bar(kKVEmpty + i), 1);  // MMA commit after P V of the tile
-      mbar_init(bar(kSFull + i), 1);    // MMA commit after S of the tile
+      mbar_init(bar(kKVEmpty + i), 1);  // MMA commit after both P V of the tile
     }
-    mbar_init(bar(kPFull), 128);        // every softmax thread
-    mbar_init(bar(kODone), 1);          // MMA commit after P V
+    for (int x = 0; x < Cfg::kQT; ++x) {
+      mbar_init(bar(kSFull + 2 * x), 1);  // MMA commit after S of the tile
+      mbar_init(bar(kSFull + 2 * x + 1), 1);
+      mbar_init(bar(kPFull + x), 128);    // every thread of the softmax warpgroup
+      mbar_init(bar(kODone + x), 1);      // MMA commit after P V
+    }
     fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
@@ -146,7 +180,8 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_o = tmem + 256;  // O columns; S buffers at columns 0 and 128
+  auto t_s = [&](int x, int b) { return tmem + (2 * x + b) * KEYN; };
+  auto t_o = [&](int x) { return tmem + 4 * KEYN + x * 128; };
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
@@ -154,21 +189,23 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       prefetch_tensormap(&q_map);
       prefetch_tensormap(&k_map);
       prefetch_tensormap(&v_map);
-      mbar_arrive_expect_tx(bar(kQFull), Cfg::kTile);
-      tma_load_3d(q_s, &q_map, 0, h * G, q0 + tq0, bar(kQFull));
-      tma_load_3d(q_s + HALF, &q_map, 64, h * G, q0 + tq0, bar(kQFull));
+      mbar_arrive_expect_tx(bar(kQFull), Cfg::kQT * Cfg::kQBytes);
+      for (int x = 0; x < Cfg::kQT; ++x) {
+        tma_load_3d(q_s(x), &q_map, 0, h * G, q0 + tq0 + x * TOK, bar(kQFull));
+        tma_load_3d(q_s(x) + QHALF, &q_map, 64, h * G, q0 + tq0 + x * TOK, bar(kQFull));
+      }
     }
-    const int rows = bs < Cfg::kKeys ? bs : Cfg::kKeys;  // tokens per box
+    const int rows = bs < KEYN ? bs : KEYN;  // tokens per box
     for (int j = 0; j < nt; ++j) {
-      const int st = j & 1, u = j >> 1;
+      const int st = j % NS, u = j / NS;
       if (u >= 1) {
         bool ok = true;
         if (lane == 0) ok = mbar_wait(bar(kKVEmpty + st), (u - 1) & 1, p.err);
         if (!__shfl_sync(kFullMask, ok, 0)) break;
       }
-      const int key0 = j * Cfg::kKeys;
-      const int nkeys = min(Cfg::kKeys, L - key0);
-      const int nbox = (nkeys + rows - 1) / rows;  // boxes holding this tile's keys (<= 16)
+      const int key0 = j * KEYN;
+      const int nkeys = min(KEYN, L - key0);
+      const int nbox = (nkeys + rows - 1) / rows;  // boxes holding this tile's keys (<= 8)
       int blk = 0;
       if (lane < nbox) blk = __ldg(trow + ((key0 + lane * rows) >> lg));
       if (lane == 0)
@@ -181,84 +218,127 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
         const int off = (key0 + lane * rows) & (bs - 1);
         const uint32_t dk = k_s(st) + lane * rows * 128, dv = v_s(st) + lane * rows * 128;
         tma_load_4d(dk, &k_map, 0, off, h, blk, bar(kKVFull + st));
-        tma_load_4d(dk + HALF, &k_map, 64, off, h, blk, bar(kKVFull + st));
+        tma_load_4d(dk + KVHALF, &k_map, 64, off, h, blk, bar(kKVFull + st));
         tma_load_4d(dv, &v_map, 0, off, h, blk, bar(kKVFull + st));
-        tma_load_4d(dv + HALF, &v_map, 64, off, h, blk, bar(kKVFull + st));
+        tma_load_4d(dv + KVHALF, &v_map, 64, off, h, blk, bar(kKVFull + st));
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
-    constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, 128, 0);   // B = K rows (K-major)
+    constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, KEYN, 0);  // B = K rows (K-major)
     constexpr uint32_t kIdPV = tc::idesc_bf16_f32(128, 128, 1);  // B = V rows (MN-major)
-    auto issue_s = [&](int j) {
-      const uint32_t kb = k_s(j & 1), d = tmem + (j & 1) * 128;
+    auto issue_s = [&](int j) {  // S_x = Q_x K_j^T for both query tiles
+      const uint32_t kb = k_s(j % NS);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * HALF + (ks & 3) * 32;
-        tc::mma_bf16(d, tc::smem_desc_sw128(q_s + off, 16, 1024),
-                     tc::smem_desc_sw128(kb + off, 16, 1024), kIdS, ks > 0);
+      for (int x = 0; x < Cfg::kQT; ++x) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks & 3) * 32;
+          tc::mma_bf16(t_s(x, j & 1), tc::smem_desc_sw128(q_s(x) + (ks >> 2) * QHALF + off, 16, 1024),
+                       tc::smem_desc_sw128(kb + (ks >> 2) * KVHALF + off, 16, 1024), kIdS, ks > 0);
+        }
+        tc::commit(bar(kSFull + 2 * x + (j & 1)));
       }
-      tc::commit(bar(kSFull + (j & 1)));
     };
-    const bool ok = wait_all(bar(kQFull), 0) && wait_all(bar(kKVFull), 0);
+    bool ok = wait_all(bar(kQFull), 0) && wait_all(bar(kKVFull), 0);
     if (ok) {
       tc::fence_after_sync();
       if (lane == 0) issue_s(0);
       for (int j = 0; j < nt; ++j) {
         if (j + 1 < nt) {
-          if (!wait_all(bar(kKVFull + ((j + 1) & 1)), ((j + 1) >> 1) & 1)) break;
+          // the S buffers of tile j+1 held tile j-1, read before its P was published
+          if (!wait_all(bar(kKVFull + (j + 1) % NS), ((j + 1) / NS) & 1)) break;
           tc::fence_after_sync();
           if (lane == 0) issue_s(j + 1);
         }
-        if (!wait_all(bar(kPFull), j & 1)) break;
-        tc::fence_after_sync();
-        if (lane == 0) {
-          const uint32_t vb = v_s(j & 1);
+        const uint32_t vb = v_s(j % NS);
+        for (int x = 0; x < Cfg::kQT && ok; ++x) {
+          if (!wait_all(bar(kPFull + x), j & 1)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          if (lane == 0) {
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            tc::mma_bf16(t_o, tc::smem_desc_sw128(p_s + (ks >> 2) * HALF + (ks & 3) * 32, 16, 1024),
-                         tc::smem_desc_sw128(vb + ks * 2048, HALF, 1024), kIdPV, j > 0 || ks > 0);
-          tc::commit(bar(kODone));
-          tc::commit(bar(kKVEmpty + (j & 1)));
+            for (int ks = 0; ks < KEYN / 16; ++ks)
+              tc::mma_bf16(t_o(x), tc::smem_desc_sw128(p_s(x) + ks * 32, 16, 1024),
+                           tc::smem_desc_sw128(vb + ks * 2048, KVHALF, 1024), kIdPV,
+                           j > 0 || ks > 0);
+            tc::commit(bar(kODone + x));
+          }
         }
+        if (!ok) break;
+        if (lane == 0) tc::commit(bar(kKVEmpty + j % NS));
         __syncwarp();
       }
     }
   } else {
     // -------------------------------------------------------------- softmax
-    const int wq = warp & 3;  // this warp reaches tensor-memory lanes 32 wq .. 32 wq + 31
+    const int x = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int wq = warp & 3;        // this warp reaches tensor-memory lanes 32 wq .. 32 wq + 31
     const int r = wq * 32 + lane;
     const int tok = r / G, g = r - (r / G) * G;
+    const int tx0 = tq0 + x * TOK;                  // first token of this query tile
+    const int ntok = max(0, min(TOK, n - tx0));     // valid tokens of this query tile
+    const int pos0 = min(L - n + tx0, pos_last);    // position of its first token
     const int prow = tok < ntok ? pos0 + tok : pos_last;  // last visible key of this row
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float qs = p.q_scale;
-    float m_run = -INFINITY, l_run = 0.0f;
+    float m_use = -INFINITY, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < nt && ok; ++j) {
-      if (!wait_all(bar(kSFull + (j & 1)), (j >> 1) & 1)) {
+      if (!wait_all(bar(kSFull + 2 * x + (j & 1)), (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::ld32(tmem + (j & 1) * 128 + lane_off + c * 32, sv[c]);
+      uint32_t sv[2][32];
+      tc::ld32(t_s(x, j & 1) + lane_off, sv[0]);
+      tc::ld32(t_s(x, j & 1) + lane_off + 32, sv[1]);
       tc::wait_ld();
-      const int lim = prow - j * Cfg::kKeys;  // keys 0 .. lim of this tile are visible
-      float mx = -INFINITY;
+      // the row maximum of the raw scores (scale > 0), masking only tiles that
+      // reach past some row's position
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (j * KEYN + KEYN - 1 <= pos0) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = c * 32 + i <= lim ? __uint_as_float(sv[c][i]) * qs : -INFINITY;
-          sv[c][i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
-      const float m_new = fmaxf(m_run, mx);  // finite: key 0 is visible to every row
-      const float alpha = exp2f(m_run - m_new);
+          for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(sv[c][i]));
+      } else {
+        const int lim = prow - j * KEYN;  // keys 0 .. lim of this tile are visible
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float v = c * 32 + i <= lim ? __uint_as_float(sv[c][i]) : -INFINITY;
+            sv[c][i] = __float_as_uint(v);
+            mx4[i & 3] = fmaxf(mx4[i & 3], v);
+          }
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * qs;
+      // key 0 is visible to every row, so m_use is finite from the first tile on;
+      // a row whose keys of this tile are all masked has mx = -inf and keeps m_use
+      const bool move = mx > m_use + 8.0f;
+      const float m_new = move ? mx : m_use;
+      const float alpha = move ? ex2_approx(m_use - m_new) : 1.0f;  // 0 on the first tile
+      // P = 2^(score * scale - m) as bf16 pairs, computed while the previous P V runs
+      float rs0 = 0.0f, rs1 = 0.0f;
+      uint32_t pw[KEYN / 2];
+#pragma unroll
+      for (int e = 0; e < KEYN / 2; ++e) {
+        const int i0 = 2 * e;
+        const float a = ex2_approx(fmaf(__uint_as_float(sv[i0 >> 5][i0 & 31]), qs, -m_new));
+        const float b =
+            ex2_approx(fmaf(__uint_as_float(sv[(i0 + 1) >> 5][(i0 + 1) & 31]), qs, -m_new));
+        rs0 += a;
+        rs1 += b;
+        pw[e] = pack_bf16x2(a, b);
+      }
+      l_run = l_run * alpha + (rs0 + rs1);
+      m_use = m_new;
       // the previous P V must be done before P is rewritten or O rescaled
       if (j > 0) {
-        if (!wait_all(bar(kODone), (j - 1) & 1)) {
+        if (!wait_all(bar(kODone + x), (j - 1) & 1)) {
           ok = false;
           break;
         }
@@ -267,46 +347,35 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t ov[32];
-            tc::ld32(t_o + lane_off + c * 32, ov);
+            tc::ld32(t_o(x) + lane_off + c * 32, ov);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tc::st32(t_o + lane_off + c * 32, ov);
+            tc::st32(t_o(x) + lane_off + c * 32, ov);
           }
           tc::wait_st();
         }
       }
-      // P = 2^(x - m) as bf16 into the swizzled K-major tile: 16-byte chunk cc of
-      // row r in half hh sits at hh * 16 KB + r * 128 + ((cc ^ (r % 8)) * 16)
-      float rs = 0.0f;
+      // P into the swizzled K-major tile: 16-byte chunk cc of row r sits at
+      // r * 128 + ((cc ^ (r % 8)) * 16)
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = c8 * 8 + 2 * e;
-          const float a = exp2f(__uint_as_float(sv[i0 >> 5][i0 & 31]) - m_new);
-          const float b = exp2f(__uint_as_float(sv[(i0 + 1) >> 5][(i0 + 1) & 31]) - m_new);
-          rs += a + b;
-          w[e] = pack_bf16x2(a, b);
-        }
-        const uint32_t addr = p_s + (c8 >> 3) * HALF + r * 128 + (((c8 & 7) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]), "r"(w[1]),
-                     "r"(w[2]), "r"(w[3])
+      for (int c8 = 0; c8 < KEYN / 8; ++c8) {
+        const uint32_t addr = p_s(x) + r * 128 + (((c8 & 7) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[4 * c8]),
+                     "r"(pw[4 * c8 + 1]), "r"(pw[4 * c8 + 2]), "r"(pw[4 * c8 + 3])
                      : "memory");
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      if (j == nt - 1) {
+      if (x == 0 && j == nt - 1) {
         // keys past the context in the last tile: stale or unwritten V rows become
-        // zeros (their P is 0, but 0 * NaN would not be)
-        const int nkeys = L - j * Cfg::kKeys;
-        if (nkeys < Cfg::kKeys) {
-          const uint32_t vb = v_s(j & 1);
-          for (int i = r; i < (Cfg::kKeys - nkeys) * 16; i += 128) {
+        // zeros (their P is 0, but 0 * NaN would not be); both P V of the tile
+        // are issued after this warpgroup's P is published
+        const int nkeys = L - j * KEYN;
+        if (nkeys < KEYN) {
+          const uint32_t vb = v_s(j % NS);
+          for (int i = r; i < (KEYN - nkeys) * 16; i += 128) {
             const int row = nkeys + (i >> 4), c = i & 15;
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
-                             vb + (c >> 3) * HALF + row * 128 + ((c & 7) << 4)),
+                             vb + (c >> 3) * KVHALF + row * 128 + ((c & 7) << 4)),
                          "r"(0u)
                          : "memory");
           }
@@ -315,27 +384,27 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       // generic-proxy writes (P, zeroed V) before the MMA's async-proxy reads
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc::fence_before_sync();
-      mbar_arrive(bar(kPFull));
+      mbar_arrive(bar(kPFull + x));
     }
-    if (ok && wait_all(bar(kODone), (nt - 1) & 1)) {
+    if (ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
-      __nv_bfloat16* dst = p.out + ((static_cast<int64_t>(q0) + tq0 + tok) * p.num_heads +
+      __nv_bfloat16* dst = p.out + ((static_cast<int64_t>(q0) + tx0 + tok) * p.num_heads +
                                     h * G + g) * Cfg::kD;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
-        tc::ld32(t_o + lane_off + c * 32, ov);
+        tc::ld32(t_o(x) + lane_off + c * 32, ov);
         tc::wait_ld();
         if (tok < ntok) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            uint4 x;
-            x.x = pack_bf16x2(__uint_as_float(ov[8 * v]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
-            x.y = pack_bf16x2(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
-            x.z = pack_bf16x2(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
-            x.w = pack_bf16x2(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + v * 8) = x;
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[8 * v]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + v * 8) = w;
           }
         }
       }
@@ -396,6 +465,12 @@ cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, con
     e = cudaFuncSetAttribute(pa_prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // all of the unified L1 / shared storage as shared memory (a per-kernel
+    // preference, not a device setting)
+    e = cudaFuncSetAttribute(pa_prefill_kernel<G>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   CUtensorMap qmap, kmap, vmap;
@@ -407,9 +482,10 @@ cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, con
   if ((e = encode_kv_map(&vmap, v_cache, sh.num_blocks, sh.block_size, sh.num_kv_heads, rows)) !=
       cudaSuccess)
     return e;
-  const unsigned tiles = static_cast<unsigned>((sh.max_query_len + Cfg::kTok - 1) / Cfg::kTok);
+  constexpr int kCtaTok = Cfg::kQT * Cfg::kTok;
+  const unsigned tiles = static_cast<unsigned>((sh.max_query_len + kCtaTok - 1) / kCtaTok);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(sh.num_kv_heads), tiles, static_cast<unsigned>(sh.num_seqs));
+  cfg.gridDim = dim3(static_cast<unsigned>(sh.num_seqs), static_cast<unsigned>(sh.num_kv_heads), tiles);
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = stream;
