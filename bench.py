@@ -180,16 +180,38 @@ def build_on_gpu(wl, device, placement="random"):
     slots, cows = cache.bm.append_slots(seqs, [1] * len(seqs))
     assert len(cows) == 0
     tables, lens = cache.bm.block_tables(seqs, max_blocks)
-    host = {
-        "q": torch.from_numpy(q).to(tdt).pin_memory(),
-        "k_new": torch.from_numpy(new_k).to(tdt).pin_memory(),
-        "v_new": torch.from_numpy(new_v).to(tdt).pin_memory(),
-        "slots": torch.from_numpy(slots).pin_memory(),
-        "tables": torch.from_numpy(tables).pin_memory(),
-        "lens": torch.from_numpy(lens).pin_memory(),
-    }
-    dev = {k: v.to(device) for k, v in host.items()}
+    host, dev = pack_step_inputs({
+        "q": torch.from_numpy(q).to(tdt),
+        "k_new": torch.from_numpy(new_k).to(tdt),
+        "v_new": torch.from_numpy(new_v).to(tdt),
+        "slots": torch.from_numpy(slots),
+        "tables": torch.from_numpy(tables),
+        "lens": torch.from_numpy(lens),
+    }, device)
     return cache, seqs, host, dev, int(lens.max()), cow_pairs
+
+
+def pack_step_inputs(arrays, device):
+    """One page-locked host buffer and one device buffer holding every per-step
+    input at 256-byte-aligned offsets, with typed views into both: a step's
+    inputs then travel host -> device in a single copy. The views are returned
+    by name; "_pack" is the whole buffer."""
+    import torch
+
+    offs, total = {}, 0
+    for name, t in arrays.items():
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    host_pack = torch.zeros(total, dtype=torch.uint8).pin_memory()
+    dev_pack = torch.zeros(total, dtype=torch.uint8, device=device)
+    host, dev = {"_pack": host_pack}, {"_pack": dev_pack}
+    for name, t in arrays.items():
+        nbytes = t.numel() * t.element_size()
+        host[name] = host_pack[offs[name]:offs[name] + nbytes].view(t.dtype).view(t.shape)
+        host[name].copy_(t)
+        dev[name] = dev_pack[offs[name]:offs[name] + nbytes].view(t.dtype).view(t.shape)
+    dev_pack.copy_(host_pack)
+    return host, dev
 
 
 class StepCalls:
@@ -409,19 +431,22 @@ def run_reference(args, wl, rank):
     }), flush=True)
 
 
-def kernel_source_digest() -> str:
-    """sha256 (first 16 hex digits) over the decode kernels' sources."""
-    import glob
+DECODE_SOURCES = ("pa_decode.cuh", "pa_decode_mma.cuh", "pa_device.cuh", "pa_kernels.cu")
+PREFILL_SOURCES = ("pa_prefill.cu", "pa_tc.cuh", "pa_device.cuh")
+
+
+def kernel_source_digest(files=DECODE_SOURCES) -> str:
+    """sha256 (first 16 hex digits) over the sources of a kernel."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_345_b200", "csrc")
-    for path in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + [os.path.join(csrc, "pa_kernels.cu")]):
-        h.update(open(path, "rb").read())
+    for name in files:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel_key: str):
+def load_traffic(kernel_key: str, files=DECODE_SOURCES):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source (matching source hash), else None."""
     path = os.path.join(ROOT, "profiles", f"{kernel_key}.traffic.txt")
@@ -432,7 +457,7 @@ def load_traffic(kernel_key: str):
         if ":" in line:
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    digest = kernel_source_digest()
+    digest = kernel_source_digest(files)
     if vals.get("source_sha256_16") != digest:
         return None
     try:
@@ -514,13 +539,12 @@ def run_b200(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         out_host = torch.empty(calls.out.shape, dtype=calls.out.dtype).pin_memory()
-        names = ("q", "k_new", "v_new", "tables", "lens") + (() if calls.fused else ("slots",))
-        h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+        # q, new K/V rows, slot mapping, tables and lengths: one packed copy
+        h2d = host["_pack"].numel()
         d2h = out_host.numel() * out_host.element_size()
 
         def e2e_step():
-            for k in names:
-                dev[k].copy_(host[k], non_blocking=True)
+            dev["_pack"].copy_(host["_pack"], non_blocking=True)
             calls.step()
             out_host.copy_(calls.out, non_blocking=True)
 
@@ -865,7 +889,9 @@ def run_prefill(args, rank, world, local_rank):
                        "l2": "flushed between steps (outside the timed events)"},
             "step_us_p10_p50_p90": [1e3 * float(np.percentile(ms, p)) for p in (10, 50, 90)],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "pa_prefill_kernel",
+                         "frac": achieved / peak,
+                         "traffic": load_traffic(f"pa_prefill_{args.workload}", PREFILL_SOURCES),
+                         "kernel": "pa_prefill_kernel",
                          "peak_source": src},
             "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
