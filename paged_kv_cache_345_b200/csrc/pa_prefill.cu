@@ -19,11 +19,14 @@
 //    one box per cache block {64 columns, min(block_size, 64) tokens} for each
 //    half of head_dim, for K and for V, into a 3-stage ring. Boxes use the
 //    128-byte swizzle, which is the shared-memory operand layout of the MMA.
-//  * Warp 1 (MMA): one thread issues tcgen05.mma. For key tile j+1 it issues
+//  * Warps 1 and 10 (MMA): one thread each issues tcgen05.mma. Warp 1 issues
 //    S_x = Q_x K^T (M 128, N 64, K 128) for both query tiles x into
-//    double-buffered tensor memory, then O_x += P_x V (M 128, N 128, K 64) for
-//    tile j as each P_x becomes ready (V is the MN-major operand, P the K-major
-//    one). Completion is signalled to mbarriers with tcgen05.commit.
+//    double-buffered tensor memory, two key tiles ahead; warp 10 issues
+//    O_x += P_x V (M 128, N 128, K 64) as each P_x becomes ready (V is the
+//    MN-major operand, P the K-major one). An MMA issue blocks while the
+//    tensor pipe's queue is full; with one issuer a ready P V waited behind a
+//    batch of S (measured), with two it does not. Completion is signalled to
+//    mbarriers with tcgen05.commit.
 //  * Warps 2-5 and 6-9 (softmax, one warpgroup per query tile): thread = row
 //    (tensor-memory lane). Per key tile: load the row of S, mask keys past the
 //    row's position, exponentials in base 2 against a reference maximum that
@@ -74,25 +77,29 @@ struct PrefillConfig {
   static constexpr int kKVBytes = kKeys * kD * 2;    // a K or V tile: two halves of 8 KB
   static constexpr int kKVHalf = kKVBytes / 2;
   static constexpr int kPBytes = kRows * kKeys * 2;  // a P tile: one 16 KB swizzle atom wide
-  static constexpr int kNS = 3;                      // K/V stages
+  static constexpr int kNS = 4;                      // K/V stages
   static constexpr int kQ = 0, kP = kQT * kQBytes, kStage0 = kP + kQT * kPBytes;
   static constexpr int kBars = kStage0 + kNS * 2 * kKVBytes;
   static constexpr int kSmemBytes = kBars + 256;     // the base is 1024-byte aligned
-  static constexpr int kThreads = 320;               // producer, MMA, 2 x 4 softmax warps
+  // producer, S-MMA issuer, 2 x 4 softmax warps, P V-MMA issuer
+  static constexpr int kThreads = 352;
   static constexpr uint32_t kTmemCols = 512;         // S[x][2] (64 each), O[x] (128 each)
   static_assert(kRows % G == 0, "group must divide the row tile");
 };
 
 // mbarrier slots
+// Barriers that two warps wait on with different lags come in pairs by tile
+// parity ([query tile][j % 2]), so that no waiter can fall two phases behind.
 enum : int {
   kQFull = 0,
   kKVFull = 1,    // [kNS]
-  kKVEmpty = 4,   // [kNS]
-  kSFull = 7,     // [query tile][2]
-  kPFull = 11,    // [query tile]
-  kODone = 13,    // [query tile]
-  kNumBars = 15
+  kKVEmpty = 5,   // [kNS]: a commit of each MMA issuer
+  kSFull = 9,     // [query tile][j % 2]
+  kPFull = 13,    // [query tile][j % 2]
+  kODone = 17,    // [query tile]
+  kNumBars = 19
 };
+constexpr int kTmemSlotOffset = 192;  // after the barriers
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint32_t bar) {
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Cfg::kBars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kBars + 128);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kBars + kTmemSlotOffset);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   auto q_s = [&](int x) { return smem_u32(sm + Cfg::kQ + x * Cfg::kQBytes); };
   auto p_s = [&](int x) { return smem_u32(sm + Cfg::kP + x * Cfg::kPBytes); };
@@ -165,14 +172,13 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     mbar_init(bar(kQFull), 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(bar(kKVFull + i), 1);   // producer arrival + TMA bytes
-      mbar_init(bar(kKVEmpty + i), 1);  // MMA commit after both P V of the tile
+      mbar_init(bar(kKVEmpty + i), 2);  // commits of both MMA issuers (S, then P V)
     }
-    for (int x = 0; x < Cfg::kQT; ++x) {
-      mbar_init(bar(kSFull + 2 * x), 1);  // MMA commit after S of the tile
-      mbar_init(bar(kSFull + 2 * x + 1), 1);
-      mbar_init(bar(kPFull + x), 128);    // every thread of the softmax warpgroup
-      mbar_init(bar(kODone + x), 1);      // MMA commit after P V
+    for (int i = 0; i < 2 * Cfg::kQT; ++i) {
+      mbar_init(bar(kSFull + i), 1);    // MMA commit after S of the tile
+      mbar_init(bar(kPFull + i), 128);  // every thread of the softmax warpgroup
     }
+    for (int x = 0; x < Cfg::kQT; ++x) mbar_init(bar(kODone + x), 1);  // commit after P V
     fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
@@ -224,9 +230,12 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA
+    // -------------------------------------------------------- S = Q K^T MMAs
+    // A tcgen05.mma issue blocks while the tensor pipe's queue is full, so the
+    // S and P V MMAs come from two warps: a ready P V never waits behind a
+    // batch of S. Tile j + 2's S reuses the tensor-memory buffers of tile j once
+    // both P of tile j are published (their S was read).
     constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, KEYN, 0);  // B = K rows (K-major)
-    constexpr uint32_t kIdPV = tc::idesc_bf16_f32(128, 128, 1);  // B = V rows (MN-major)
     auto issue_s = [&](int j) {  // S_x = Q_x K_j^T for both query tiles
       const uint32_t kb = k_s(j % NS);
 #pragma unroll
@@ -239,38 +248,43 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
         }
         tc::commit(bar(kSFull + 2 * x + (j & 1)));
       }
+      tc::commit(bar(kKVEmpty + j % NS));  // K of tile j read (first of two commits)
     };
-    bool ok = wait_all(bar(kQFull), 0) && wait_all(bar(kKVFull), 0);
-    if (ok) {
-      tc::fence_after_sync();
-      if (lane == 0) issue_s(0);
-      for (int j = 0; j < nt; ++j) {
-        if (j + 1 < nt) {
-          // the S buffers of tile j+1 held tile j-1, read before its P was published
-          if (!wait_all(bar(kKVFull + (j + 1) % NS), ((j + 1) / NS) & 1)) break;
-          tc::fence_after_sync();
-          if (lane == 0) issue_s(j + 1);
-        }
-        const uint32_t vb = v_s(j % NS);
-        for (int x = 0; x < Cfg::kQT && ok; ++x) {
-          if (!wait_all(bar(kPFull + x), j & 1)) {
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
-          if (lane == 0) {
-#pragma unroll
-            for (int ks = 0; ks < KEYN / 16; ++ks)
-              tc::mma_bf16(t_o(x), tc::smem_desc_sw128(p_s(x) + ks * 32, 16, 1024),
-                           tc::smem_desc_sw128(vb + ks * 2048, KVHALF, 1024), kIdPV,
-                           j > 0 || ks > 0);
-            tc::commit(bar(kODone + x));
-          }
-        }
+    bool ok = wait_all(bar(kQFull), 0);
+    for (int j = 0; j < nt && ok; ++j) {
+      if (j >= 2) {
+        for (int x = 0; x < Cfg::kQT && ok; ++x)
+          ok = wait_all(bar(kPFull + 2 * x + (j & 1)), ((j - 2) >> 1) & 1);
         if (!ok) break;
-        if (lane == 0) tc::commit(bar(kKVEmpty + j % NS));
-        __syncwarp();
       }
+      if (!wait_all(bar(kKVFull + j % NS), (j / NS) & 1)) break;
+      tc::fence_after_sync();
+      if (lane == 0) issue_s(j);
+      __syncwarp();
+    }
+  } else if (warp == 2 + 4 * Cfg::kQT) {
+    // ------------------------------------------------------------ P V MMAs
+    constexpr uint32_t kIdPV = tc::idesc_bf16_f32(128, 128, 1);  // B = V rows (MN-major)
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      const uint32_t vb = v_s(j % NS);
+      for (int x = 0; x < Cfg::kQT && ok; ++x) {
+        if (!wait_all(bar(kPFull + 2 * x + (j & 1)), (j >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        if (lane == 0) {
+#pragma unroll
+          for (int ks = 0; ks < KEYN / 16; ++ks)
+            tc::mma_bf16(t_o(x), tc::smem_desc_sw128(p_s(x) + ks * 32, 16, 1024),
+                         tc::smem_desc_sw128(vb + ks * 2048, KVHALF, 1024), kIdPV,
+                         j > 0 || ks > 0);
+          tc::commit(bar(kODone + x));
+        }
+      }
+      if (ok && lane == 0) tc::commit(bar(kKVEmpty + j % NS));  // V of tile j read
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------------------- softmax
@@ -384,7 +398,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       // generic-proxy writes (P, zeroed V) before the MMA's async-proxy reads
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc::fence_before_sync();
-      mbar_arrive(bar(kPFull + x));
+      mbar_arrive(bar(kPFull + 2 * x + (j & 1)));
     }
     if (ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
       tc::fence_after_sync();
