@@ -17,7 +17,7 @@
 // sequence's end, so the tiles that see the most keys start first.
 //  * Warp 0 (producer): TMA loads both Q tiles once, then per tile of 64 keys
 //    one box per cache block {64 columns, min(block_size, 64) tokens} for each
-//    half of head_dim, for K and for V, into a 3-stage ring. Boxes use the
+//    half of head_dim, for K and for V, into a 4-stage ring. Boxes use the
 //    128-byte swizzle, which is the shared-memory operand layout of the MMA.
 //  * Warps 1 and 10 (MMA): one thread each issues tcgen05.mma. Warp 1 issues
 //    S_x = Q_x K^T (M 128, N 64, K 128) for both query tiles x into
