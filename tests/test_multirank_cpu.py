@@ -73,3 +73,22 @@ def test_reference_arm_under_two_ranks_prints_once():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_prefill_flop_count_is_the_causal_pair_count():
+    """bench.py's prefill flops: 4 * head_dim * heads per (query row, visible key)
+    pair, the pairs counted here one by one."""
+    bench = _bench()
+    for before, chunks in (([0], [5]), ([3], [4]), ([0, 7], [7, 2]), ([128], [1])):
+        pairs = sum(b + i + 1 for b, c in zip(before, chunks) for i in range(c))
+        assert bench.prefill_flops(before, chunks, 2, 8) == 4 * 8 * 2 * pairs
+    before, chunks = bench.prefill_shape("prefill")
+    assert before == [0] * 8 and sum(chunks) == 10_578
+    assert bench.prefill_flops(before, chunks) == 4 * 128 * 32 * sum(L * (L + 1) // 2 for L in chunks)
+
+
+def _bench():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    return bench
