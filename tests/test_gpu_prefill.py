@@ -176,3 +176,14 @@ def test_prefill_refusals():
     assert st == pa.PA_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert bool((out == 5.0).all())
+
+
+def test_prefill_empty_chunks_and_empty_sequences():
+    """Sequences with no query rows in the batch (a zero-row chunk, or nothing
+    cached at all) produce nothing and disturb nothing."""
+    before, chunks = [5, 0, 40, 0], [3, 0, 0, 70]
+    got, q, rows, lens = _run(before, chunks)
+    keep = [s for s, c in enumerate(chunks) if c]
+    ref = _expected(q, [rows[s] for s in keep], [lens[s] for s in keep],
+                    [chunks[s] for s in keep], 32)
+    gh.assert_close(got, ref, "bf16", "prefill with empty chunks")
