@@ -166,7 +166,7 @@ int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
  * pa_decode_partition_size — the partition length (tokens) pa_decode uses when
  * passed partition_size = 0. Chosen from the grid size alone (sequences, KV
  * heads, max_context_len), never from block_size or placement, so results do
- * not depend on either. Always a multiple of 16.
+ * not depend on either. Always a multiple of 16, between 64 and 768.
  */
 int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len);
 
