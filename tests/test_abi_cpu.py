@@ -102,7 +102,7 @@ def test_append_and_copy_reject_on_host():
 def test_partition_size_and_workspace():
     for s, h, n in [(8, 8, 4101), (256, 8, 4096), (1, 1, 7), (16, 8, 32768), (64, 8, 3054)]:
         p = pa.pa_decode_partition_size(s, h, n)
-        assert p % 16 == 0 and 64 <= p <= 512
+        assert p % 16 == 0 and 64 <= p <= 768
     assert pa.pa_decode_partition_size(8, 8, 4101) == 160
     # one partition: no workspace
     assert pa.pa_decode_workspace_bytes(2, 4, 2, 64, 34, 64) == 0
