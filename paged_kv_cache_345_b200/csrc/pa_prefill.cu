@@ -12,9 +12,10 @@
 // Layout and pipeline. One CTA = one sequence x one KV head x two query tiles
 // of 128 rows (each 128 / G tokens x the G query heads of the KV head, row =
 // token * G + g). Both tiles share every K/V tile, which halves the K/V bytes
-// per flop: with one 128-row tile per CTA the kernel was bound by L2-to-SM
-// bandwidth, not by the tensor cores. The grid counts tiles from each
-// sequence's end, so the tiles that see the most keys start first.
+// per flop: with one 128-row tile per CTA the K/V tile loads (the per-SM load
+// path and its latency), not the tensor cores, set the pace. The grid counts
+// tiles from each sequence's end, so the tiles that see the most keys start
+// first.
 //  * Warp 0 (producer): TMA loads both Q tiles once, then per tile of 64 keys
 //    one box per cache block {64 columns, min(block_size, 64) tokens} for each
 //    half of head_dim, for K and for V, into a 4-stage ring. Boxes use the
