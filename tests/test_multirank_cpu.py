@@ -92,3 +92,21 @@ def _bench():
     import bench
 
     return bench
+
+
+def test_reference_arm_sample_is_bounded_and_valid():
+    """The CPU reference arm runs the worked-example batch whole and the larger
+    workloads on their first sequences in a compact, unshared pool."""
+    bench = _bench()
+    from workloads import configs
+
+    wl, note = bench.reference_workload(configs.llama3_8b_layer())
+    assert wl.context_lens == configs.llama3_8b_layer().context_lens and "whole" in note
+    for big in (configs.large_batch(steps=1), configs.shared_prefix(), configs.long_context(16)):
+        small, note = bench.reference_workload(big)
+        assert 1 <= small.num_seqs <= big.num_seqs
+        assert sum(n + 1 for n in small.context_lens) <= 40_000 or small.num_seqs == 1
+        assert small.context_lens == big.context_lens[:small.num_seqs]
+        assert small.shared_prefix == 0 and small.ghost_lens == ()
+        assert small.num_blocks >= sum(-(-(n + 1) // small.block_size) for n in small.context_lens)
+        assert str(small.num_seqs) in note
