@@ -73,7 +73,8 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 #define PA_DEVERR_SLOT 0x1u       /* pa_kv_append: slot >= num_blocks * block_size       */
 #define PA_DEVERR_BLOCK_ID 0x2u   /* pa_decode: table entry outside [0, num_blocks)       */
 #define PA_DEVERR_CONTEXT 0x4u    /* pa_decode: context_lens[s] < 0, > max_context_len,
-                                     or > max_blocks_per_seq * block_size                 */
+                                     or > max_blocks_per_seq * block_size; pa_prefill:
+                                     a bad query_start range or chunk length (below)      */
 #define PA_DEVERR_COPY_PAIR 0x8u  /* pa_copy_blocks: src or dst outside [0, num_blocks)  */
 #define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up               */
 
@@ -307,7 +308,9 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
  *   query_start    device, int32 [num_seqs + 1], non-decreasing, from 0 to at
  *                  most total_q; 0 <= n <= context_lens[s] for every s, else
  *                  PA_DEVERR_CONTEXT is set and that sequence is skipped.
- *   max_query_len  host upper bound of n over the batch (sizes the grid).
+ *   max_query_len  host upper bound of n over the batch (sizes the grid); a
+ *                  sequence with n > max_query_len sets PA_DEVERR_CONTEXT and
+ *                  is skipped (its rows are not written).
  *   Everything else as pa_decode. Products in bf16 on the tensor cores
  *   (tcgen05), softmax and accumulation in fp32; softmax weights are rounded to
  *   bf16 before the product with V.

@@ -62,7 +62,7 @@ struct PrefillParams {
   const int32_t* query_start;
   unsigned* err;
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks, max_blocks_per_seq;
-  int total_q;
+  int total_q, max_query_len;
   float q_scale;  // scale * log2(e)
 };
 
@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   const int q0 = __ldg(p.query_start + s), q1 = __ldg(p.query_start + s + 1);
   const int L = __ldg(p.context_lens + s);
   const int n = q1 - q0;
-  if (q0 < 0 || q1 > p.total_q || n < 0 || L < n ||
+  // n above the host bound would leave rows outside the grid: flag, never drop silently
+  if (q0 < 0 || q1 > p.total_q || n < 0 || n > p.max_query_len || L < n ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
     if (threadIdx.x == 0 && h == 0 && blockIdx.z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
     return;
@@ -535,6 +536,7 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
   p.num_blocks = sh.num_blocks;
   p.max_blocks_per_seq = sh.max_blocks_per_seq;
   p.total_q = sh.total_q;
+  p.max_query_len = sh.max_query_len;
   p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
   switch (sh.num_heads / sh.num_kv_heads) {
     case 1: return launch_prefill_g<1>(sh, p, q, k_cache, v_cache, stream);

@@ -187,3 +187,19 @@ def test_prefill_empty_chunks_and_empty_sequences():
     ref = _expected(q, [rows[s] for s in keep], [lens[s] for s in keep],
                     [chunks[s] for s in keep], 32)
     gh.assert_close(got, ref, "bf16", "prefill with empty chunks")
+
+
+def test_prefill_chunk_above_host_bound_is_flagged_and_skipped():
+    """A chunk longer than max_query_len would have rows outside the grid: the
+    sequence is flagged and skipped, the others are computed as usual."""
+    k = torch.zeros((4, 16, 2, D), dtype=torch.bfloat16, device="cuda")
+    q = torch.ones((9, 4, D), dtype=torch.bfloat16, device="cuda")
+    out = torch.full_like(q, 5.0)
+    tables = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device="cuda")
+    lens = torch.tensor([20, 20], dtype=torch.int32, device="cuda")
+    qs = torch.tensor([0, 5, 9], dtype=torch.int32, device="cuda")   # seq 0: 5 rows > bound 4
+    st = _raw_prefill(out, q, k, k, tables, lens, qs, 2, 9, 4, 2, 16, 4, 2, 4, pa.PA_BF16)
+    assert st == pa.PA_OK
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT
+    assert bool((out[:5] == 5.0).all())          # skipped
+    assert bool((out[5:] == 0.0).all())          # V = 0 everywhere -> zeros
