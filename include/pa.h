@@ -413,6 +413,9 @@ int pa_alloc_set_free_order(pa_alloc* a, const int32_t* ids, int n);
  *   "PagedAttention — AI Glossary", How it works 4-5: sequences sharing a
  *   prefix point at the same reference-counted blocks; a shared block is
  *   copied when one sharer writes into it.
+ * A call that cannot get host memory returns PA_ERR_INVALID ("out of host
+ * memory" in pa_last_error) and changes nothing; no C++ exception leaves the
+ * library.
  */
 typedef struct pa_bm pa_bm;
 

@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <new>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "pa.h"
@@ -136,7 +137,12 @@ int pa_alloc_set_free_order(pa_alloc* a, const int32_t* ids, int n) {
   if (static_cast<size_t>(n) != a->free_stack.size())
     return pa_fail(PA_ERR_INVALID, "pa_alloc_set_free_order: %d ids for %zu free blocks", n,
                    a->free_stack.size());
-  std::vector<char> seen(a->refcount.size(), 0);
+  std::vector<char> seen;
+  try {
+    seen.assign(a->refcount.size(), 0);
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_alloc_set_free_order: out of host memory");
+  }
   for (int i = 0; i < n; ++i) {
     int32_t b = ids[i];
     if (!valid_id(a, b) || a->refcount[b] != 0 || seen[b])
@@ -178,7 +184,12 @@ int pa_bm_block_size(const pa_bm* bm) { return bm ? bm->block_size : -1; }
 
 int pa_bm_add_seq(pa_bm* bm, int32_t* seq_id) {
   if (!bm || !seq_id) return pa_fail(PA_ERR_INVALID, "pa_bm_add_seq: null argument");
-  int32_t id = bm->new_id();
+  int32_t id;
+  try {
+    id = bm->new_id();
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_add_seq: out of host memory");
+  }
   Seq& s = bm->seqs[id];
   s.live = true;
   s.length = 0;
@@ -190,13 +201,21 @@ int pa_bm_add_seq(pa_bm* bm, int32_t* seq_id) {
 int pa_bm_fork(pa_bm* bm, int32_t parent, int32_t* child) {
   if (!bm || !child) return pa_fail(PA_ERR_INVALID, "pa_bm_fork: null argument");
   if (!bm->get(parent)) return pa_fail(PA_ERR_INVALID, "pa_bm_fork: unknown sequence %d", parent);
-  int32_t id = bm->new_id();  // may grow seqs: take the parent's pointer afterwards
+  // Everything that can fail to allocate comes before the first change.
+  std::vector<int32_t> blocks;
+  int32_t id;
+  try {
+    blocks = bm->seqs[parent].blocks;
+    id = bm->new_id();  // may grow seqs: index the parent again afterwards
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_fork: out of host memory");
+  }
   const Seq& p = bm->seqs[parent];
   Seq& c = bm->seqs[id];
-  for (int32_t b : p.blocks) bm->pool->refcount[b] += 1;
+  for (int32_t b : blocks) bm->pool->refcount[b] += 1;
   c.live = true;
   c.length = p.length;
-  c.blocks = p.blocks;
+  c.blocks = std::move(blocks);
   *child = id;
   return PA_OK;
 }
@@ -205,6 +224,11 @@ int pa_bm_free_seq(pa_bm* bm, int32_t seq_id) {
   if (!bm) return pa_fail(PA_ERR_INVALID, "pa_bm_free_seq: null manager");
   Seq* s = bm->get(seq_id);
   if (!s) return pa_fail(PA_ERR_INVALID, "pa_bm_free_seq: unknown sequence %d", seq_id);
+  try {
+    bm->free_ids.reserve(bm->free_ids.size() + 1);  // the push below cannot fail then
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_free_seq: out of host memory");
+  }
   for (int32_t b : s->blocks) pa_decref(bm->pool, b);
   s->live = false;
   s->length = 0;
@@ -230,7 +254,12 @@ int pa_bm_append_slots(pa_bm* bm, const int32_t* seq_ids, const int32_t* counts,
     return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: null or negative argument");
   // Validate everything and count what is needed before changing anything.
   int64_t need = 0, total = 0, cows = 0;
-  std::vector<int32_t> sorted(seq_ids, seq_ids + n);
+  std::vector<int32_t> sorted;
+  try {
+    sorted.assign(seq_ids, seq_ids + n);
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: out of host memory");
+  }
   std::sort(sorted.begin(), sorted.end());
   if (std::adjacent_find(sorted.begin(), sorted.end()) != sorted.end())
     return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: a sequence id appears twice");
@@ -253,6 +282,16 @@ int pa_bm_append_slots(pa_bm* bm, const int32_t* seq_ids, const int32_t* counts,
   if (need > static_cast<int64_t>(bm->pool->free_stack.size()))
     return pa_fail(PA_ERR_NO_BLOCKS, "pa_bm_append_slots: need %lld blocks, %zu free",
                    static_cast<long long>(need), bm->pool->free_stack.size());
+  // Room for every new table entry first, so that the loop below cannot fail
+  // half-way (reserving changes no table).
+  try {
+    for (int i = 0; i < n; ++i) {
+      Seq& s = *bm->get(seq_ids[i]);
+      s.blocks.reserve(static_cast<size_t>(ceil_div(s.length + counts[i], bs)));
+    }
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: out of host memory");
+  }
 
   int64_t k = 0;
   int ncow = 0;
