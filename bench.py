@@ -490,7 +490,7 @@ def run_reference(args, wl, rank):
 
 
 DECODE_SOURCES = ("pa_decode.cuh", "pa_decode_mma.cuh", "pa_device.cuh", "pa_kernels.cu")
-PREFILL_SOURCES = ("pa_prefill.cu", "pa_tc.cuh", "pa_device.cuh")
+PREFILL_SOURCES = ("pa_prefill.cu", "pa_prefill_order.h", "pa_tc.cuh", "pa_device.cuh")
 
 
 def kernel_source_digest(files=DECODE_SOURCES) -> str:

@@ -317,7 +317,8 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
  * scale must be finite and > 0. Supported: dtype PA_BF16; head_dim 128;
  * num_heads / num_kv_heads in {1, 2, 4, 8}; block_size a power of two in
  * [8, 256]. The result does not depend on block_size or on the physical
- * placement of the blocks.
+ * placement of the blocks. Work is handed to CTAs longest first (an order
+ * over all sequences' items found in the kernel); this affects speed only.
  */
 int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                const int32_t* block_tables, const int32_t* context_lens,

@@ -393,7 +393,8 @@ int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cach
   if (!std::isfinite(scale) || scale <= 0.0f)
     return pa_fail(PA_ERR_INVALID, "pa_prefill: scale must be finite and > 0");
   const int tok = 256 / group;  // query tokens per CTA
-  if (num_seqs > 65535 || (max_query_len + tok - 1) / tok > 65535 || num_kv_heads > 65535)
+  if (static_cast<int64_t>(num_seqs) * ((max_query_len + tok - 1) / tok) * num_kv_heads >
+      0x7fffffff)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: grid too large");
   if (static_cast<int64_t>(num_blocks) * block_size * num_kv_heads * head_dim * 2 / 16 >
       (int64_t(1) << 36))

@@ -47,6 +47,7 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "pa_prefill_order.h"
 #include "pa_tc.cuh"
 
 namespace pa {
@@ -62,7 +63,7 @@ struct PrefillParams {
   const int32_t* query_start;
   unsigned* err;
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks, max_blocks_per_seq;
-  int total_q, max_query_len;
+  int num_seqs, total_q, max_query_len;
   float q_scale;  // scale * log2(e)
 };
 
@@ -118,6 +119,81 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Longest-first order over at most kOrderMaxSeqs sequences; larger batches
+// take their items pair by pair across the sequences.
+constexpr int kOrderMaxSeqs = 256;
+
+// The work item (sequence *s, item *z) of work index j in longest-first
+// order: items sorted by cost (key tiles visited) downward, then by sequence,
+// then by z. Every lane of the warp returns the same answer. Each lane holds
+// sequences lane, lane + 32, ... (PER of them); the search finds the cost
+// level c with count(c + 1) <= j < count(c), count(c) = items costing at
+// least c, then the item among those costing exactly c. *bad tells whether
+// any sequence has unusable arguments (it then has no items). Returns false
+// when j is past the last item.
+template <int PER, int CTOK, int KEYN>
+__device__ __forceinline__ bool work_item(const PrefillParams& p, int S, int j, int lane, int* s,
+                                          int* z, bool* bad) {
+  namespace po = prefill_order;
+  constexpr int LG = CTOK == 32 ? 5 : CTOK == 64 ? 6 : CTOK == 128 ? 7 : 8;
+  static_assert((1 << LG) == CTOK, "query rows per item must be a power of two");
+  po::ItemCosts q[PER];
+  bool any_bad = false;
+  int cmax = 0;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int t = lane + 32 * k;
+    q[k] = po::ItemCosts{0, 0, 0};
+    if (t < S) {
+      const int q0 = __ldg(p.query_start + t), q1 = __ldg(p.query_start + t + 1);
+      const int L = __ldg(p.context_lens + t);
+      if (po::chunk_ok(q0, q1, L, p.total_q, p.max_query_len,
+                       static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size))
+        q[k] = po::item_costs(L, q1 - q0, CTOK, KEYN);
+      else
+        any_bad = true;
+    }
+    cmax = max(cmax, q[k].top);
+  }
+  *bad = __any_sync(kFullMask, any_bad);
+  auto count = [&](int c) {
+    int acc = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc += po::items_at_least(q[k], c, LG, KEYN);
+    return __reduce_add_sync(kFullMask, acc);
+  };
+  cmax = __reduce_max_sync(kFullMask, cmax);
+  if (cmax == 0 || j >= count(1)) return false;
+  int lo = 1, hi = cmax + 1;  // count(lo) > j >= count(hi)
+  while (hi - lo > 1) {       // at most 31 rounds: cmax < 2^31
+    const int mid = lo + ((hi - lo) >> 1);
+    if (count(mid) > j) lo = mid;
+    else hi = mid;
+  }
+  int o = j - count(lo + 1);  // rank among the items costing exactly lo
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int above = po::items_at_least(q[k], lo + 1, LG, KEYN);
+    const int e = po::items_at_least(q[k], lo, LG, KEYN) - above;
+    int incl = e;  // inclusive prefix over the lanes: sequences 32k .. 32k + lane
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(kFullMask, incl, d);
+      if (lane >= d) incl += v;
+    }
+    const int here = __shfl_sync(kFullMask, incl, 31);
+    if (o < here) {
+      const int src = __ffs(__ballot_sync(kFullMask, incl > o)) - 1;
+      *z = __shfl_sync(kFullMask, above + o - (incl - e), src);
+      *s = 32 * k + src;
+      return true;
+    }
+    o -= here;
+  }
+  if (lane == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);  // unreachable when the counts agree
+  return false;
+}
+
 template <int G>
 __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     pa_prefill_kernel(const __grid_constant__ CUtensorMap q_map,
@@ -136,8 +212,9 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   auto k_s = [&](int st) { return smem_u32(sm + Cfg::kStage0 + st * 2 * Cfg::kKVBytes); };
   auto v_s = [&](int st) { return k_s(st) + Cfg::kKVBytes; };
 
-  // grid (sequence, KV head, pair of query tiles counted from the end)
-  const int s = blockIdx.x, h = blockIdx.y;
+  // one-dimensional grid: KV head fastest, then the work index
+  const int h = static_cast<int>(blockIdx.x % static_cast<unsigned>(p.num_kv_heads));
+  const int jw = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.num_kv_heads));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bs = p.block_size, lg = p.log2_block_size;
   // every lane polls; the warp proceeds only if all saw the phase complete
@@ -148,19 +225,34 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   pdl_wait();  // inputs may come from the previous kernel in the stream
   pdl_launch_dependents();
 
+  constexpr int CTOK = Cfg::kQT * TOK;  // tokens per CTA
+  const int S = p.num_seqs;
+  int s, z;
+  if (S <= kOrderMaxSeqs) {
+    bool bad = false, found;
+    if (S <= 32) found = work_item<1, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+    else if (S <= 64) found = work_item<2, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+    else if (S <= 128) found = work_item<4, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+    else found = work_item<8, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+    // a sequence with unusable arguments (among them n above the host bound,
+    // whose rows would lie outside the grid) gets no items: flagged once
+    if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+    if (!found) return;
+  } else {
+    s = jw % S;
+    z = jw / S;
+  }
   const int q0 = __ldg(p.query_start + s), q1 = __ldg(p.query_start + s + 1);
   const int L = __ldg(p.context_lens + s);
   const int n = q1 - q0;
-  // n above the host bound would leave rows outside the grid: flag, never drop silently
-  if (q0 < 0 || q1 > p.total_q || n < 0 || n > p.max_query_len || L < n ||
-      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
-    if (threadIdx.x == 0 && h == 0 && blockIdx.z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+  if (!prefill_order::chunk_ok(q0, q1, L, p.total_q, p.max_query_len,
+                               static_cast<int64_t>(p.max_blocks_per_seq) * bs)) {
+    if (threadIdx.x == 0 && h == 0 && z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
     return;
   }
-  constexpr int CTOK = Cfg::kQT * TOK;  // tokens per CTA
-  const int npairs = (n + CTOK - 1) / CTOK;
-  if (static_cast<int>(blockIdx.z) >= npairs) return;  // no rows of this sequence here
-  const int tq0 = (npairs - 1 - static_cast<int>(blockIdx.z)) * CTOK;
+  const int npairs = prefill_order::num_items(n, CTOK);
+  if (z >= npairs) return;  // no rows of this sequence here
+  const int tq0 = (npairs - 1 - z) * CTOK;
   const int ntok_all = min(CTOK, n - tq0);
   const int pos_last = L - n + tq0 + ntok_all - 1;  // <= L - 1
   const int nt = pos_last / KEYN + 1;                // key tiles to visit
@@ -499,9 +591,14 @@ cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, con
       cudaSuccess)
     return e;
   constexpr int kCtaTok = Cfg::kQT * Cfg::kTok;
-  const unsigned tiles = static_cast<unsigned>((sh.max_query_len + kCtaTok - 1) / kCtaTok);
+  // work indices: every sequence could have max_query_len rows; those past
+  // the last item exit at once (they are dispatched last)
+  const int64_t items = static_cast<int64_t>(sh.num_seqs) *
+                        ((sh.max_query_len + kCtaTok - 1) / kCtaTok);
+  const int64_t ctas = items * sh.num_kv_heads;
+  if (ctas > 0x7fffffff) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(sh.num_seqs), static_cast<unsigned>(sh.num_kv_heads), tiles);
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = stream;
@@ -535,6 +632,7 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
   p.log2_block_size = lg;
   p.num_blocks = sh.num_blocks;
   p.max_blocks_per_seq = sh.max_blocks_per_seq;
+  p.num_seqs = sh.num_seqs;
   p.total_q = sh.total_q;
   p.max_query_len = sh.max_query_len;
   p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)

@@ -55,7 +55,9 @@ def _run(before, chunks, hq=32, hkv=8, bs=16, free_order=None, poisoned=False, s
     q = np.concatenate([_queries(s, c, hq) for s, c in enumerate(chunks)])
     kc = dev(np.concatenate([r[0][b:] for r, b in zip(rows, before)]))
     vc = dev(np.concatenate([r[1][b:] for r, b in zip(rows, before)]))
-    out = cache.prefill(dev(q), kc, vc, seqs, list(chunks), 1 / np.sqrt(D))
+    qd = dev(q)
+    out = torch.full_like(qd, float("nan"))     # a row the kernel skips stays NaN
+    out = cache.prefill(qd, kc, vc, seqs, list(chunks), 1 / np.sqrt(D), out=out)
     torch.cuda.synchronize()
     assert pa.pa_device_errors() == 0
     return out.float().cpu().numpy(), q, rows, lens
@@ -93,6 +95,24 @@ def test_prefill_group_sizes(hq, hkv):
     before, chunks = [0, 200, 3], [300, 129, 1]
     got, q, rows, lens = _run(before, chunks, hq=hq, hkv=hkv)
     gh.assert_close(got, _expected(q, rows, lens, chunks, hq), "bf16", f"prefill {hq}/{hkv}")
+
+
+@pytest.mark.parametrize("S,hq,hkv,seed", [(5, 2, 2, 1), (33, 16, 2, 2), (70, 8, 2, 3),
+                                         (200, 4, 2, 4), (300, 8, 2, 5)])
+def test_prefill_work_order_covers_every_row(S, hq, hkv, seed):
+    """Batches of 5 to 300 sequences with mixed lengths and empty chunks: CTAs
+    take their work items longest first (up to 256 sequences, the per-lane
+    layouts of 1, 2, 4 and 8 sequences per lane) or pair by pair past that;
+    every row must be computed exactly once."""
+    rng = np.random.default_rng(seed)
+    total = rng.integers(0, 300 if S <= 70 else 40, S)
+    chunks = [0 if rng.random() < 0.2 else int(rng.integers(0, L + 1)) for L in total]
+    before = [int(L) - c for L, c in zip(total, chunks)]
+    got, q, rows, lens = _run(before, chunks, hq=hq, hkv=hkv)
+    keep = [s for s, c in enumerate(chunks) if c]
+    ref = _expected(q, [rows[s] for s in keep], [lens[s] for s in keep],
+                    [chunks[s] for s in keep], hq)
+    gh.assert_close(got, ref, "bf16", f"prefill order S={S}")
 
 
 def test_prefill_is_bitwise_invariant_to_block_size_and_placement():
