@@ -20,6 +20,7 @@ Entry points (same names as the C ABI):
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -169,6 +170,23 @@ def _stream(stream, device):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _on_device(tensors, stream):
+    """(device guard, stream pointer) for one call. Its CUDA tensors must all be
+    on one device (a kernel given another GPU's pointer would read outside its
+    own memory), an explicit stream must belong to that device, and the call
+    runs with that device current. CPU tensors (pinned host pools) are skipped."""
+    torch = _torch()
+    devs = {t.device for t in tensors if t is not None and t.is_cuda}
+    if len(devs) > 1:
+        raise ValueError("tensors of one call are on several devices: " +
+                         ", ".join(sorted(str(d) for d in devs)))
+    dev = devs.pop() if devs else None
+    if dev is not None and stream is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
+    guard = torch.cuda.device(dev) if dev is not None else contextlib.nullcontext()
+    return guard, _stream(stream, dev)
+
+
 # ---------------------------------------------------------------- kernels
 
 def pa_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> None:
@@ -180,11 +198,13 @@ def pa_kv_append(k_new, v_new, slot_mapping, k_cache, v_cache, stream=None) -> N
     if v_cache.shape != k_cache.shape or slot_mapping.shape != (k_new.shape[0],):
         raise ValueError("cache or slot_mapping shape mismatch")
     dt = k_cache.dtype
-    _check(_lib.pa_kv_append(
-        _dev_ptr(k_new, "k_new", dt), _dev_ptr(v_new, "v_new", dt),
-        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
-        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", dt), nb, bs, hkv, d,
-        _dtype_code(k_cache), _stream(stream, k_cache.device)))
+    guard, st = _on_device((k_new, v_new, slot_mapping, k_cache, v_cache), stream)
+    with guard:
+        _check(_lib.pa_kv_append(
+            _dev_ptr(k_new, "k_new", dt), _dev_ptr(v_new, "v_new", dt),
+            _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
+            _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", dt), nb, bs, hkv, d,
+            _dtype_code(k_cache), st))
 
 
 def pa_kv_append_fp8(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale,
@@ -202,12 +222,15 @@ def pa_kv_append_fp8(k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_sc
         raise TypeError("caches must hold E4M3 codes (uint8 or float8_e4m3fn)")
     if k_scale.shape != (hkv,) or v_scale.shape != (hkv,):
         raise ValueError("k_scale/v_scale must be [num_kv_heads]")
-    _check(_lib.pa_kv_append_fp8(
-        _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
-        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
-        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
-        _dev_ptr(k_scale, "k_scale", torch.float32), _dev_ptr(v_scale, "v_scale", torch.float32),
-        nb, bs, hkv, d, _stream(stream, k_cache.device)))
+    guard, st = _on_device((k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale),
+                           stream)
+    with guard:
+        _check(_lib.pa_kv_append_fp8(
+            _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
+            _dev_ptr(slot_mapping, "slot_mapping", torch.int64), k_new.shape[0],
+            _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+            _dev_ptr(k_scale, "k_scale", torch.float32),
+            _dev_ptr(v_scale, "v_scale", torch.float32), nb, bs, hkv, d, st))
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
@@ -216,10 +239,12 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
     nb, bs, hkv, d = k_cache.shape
     if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
         raise ValueError("block_mapping must be [num_pairs, 2]")
-    _check(_lib.pa_copy_blocks(
-        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", k_cache.dtype),
-        _dev_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], nb, bs,
-        hkv, d, _dtype_code(k_cache), _stream(stream, k_cache.device)))
+    guard, st = _on_device((k_cache, v_cache, block_mapping), stream)
+    with guard:
+        _check(_lib.pa_copy_blocks(
+            _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", k_cache.dtype),
+            _dev_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], nb,
+            bs, hkv, d, _dtype_code(k_cache), st))
 
 
 def _mapped_ptr(t, name, dtype=None):
@@ -246,12 +271,13 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None) -> No
     if block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
         raise ValueError("block_mapping must be [num_pairs, 2]")
     dt = src_k.dtype
-    dev = dst_k.device if dst_k.is_cuda else (src_k.device if src_k.is_cuda else None)
-    _check(_lib.pa_swap_blocks(
-        _mapped_ptr(dst_k, "dst_k", dt), _mapped_ptr(dst_v, "dst_v", dt), dnb,
-        _mapped_ptr(src_k, "src_k", dt), _mapped_ptr(src_v, "src_v", dt), snb,
-        _mapped_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0], bs, hkv,
-        d, _dtype_code(src_k), _stream(stream, dev)))
+    guard, st = _on_device((dst_k, dst_v, src_k, src_v, block_mapping), stream)
+    with guard:
+        _check(_lib.pa_swap_blocks(
+            _mapped_ptr(dst_k, "dst_k", dt), _mapped_ptr(dst_v, "dst_v", dt), dnb,
+            _mapped_ptr(src_k, "src_k", dt), _mapped_ptr(src_v, "src_v", dt), snb,
+            _mapped_ptr(block_mapping, "block_mapping", torch.int64), block_mapping.shape[0],
+            bs, hkv, d, _dtype_code(src_k), st))
 
 
 def pa_decode_partition_size(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:
@@ -284,12 +310,15 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
     if workspace is not None:
         ws_ptr = _dev_ptr(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(_lib.pa_decode(
-        _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
-        _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
-        block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,
-        ws_bytes, _dtype_code(k_cache), _stream(stream, q.device)))
+    guard, st = _on_device((out, q, k_cache, v_cache, block_tables, context_lens, workspace),
+                           stream)
+    with guard:
+        _check(_lib.pa_decode(
+            _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
+            block_tables.shape[1], int(max_context_len), float(scale), int(partition_size),
+            ws_ptr, ws_bytes, _dtype_code(k_cache), st))
 
 
 def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
@@ -311,13 +340,16 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, conte
     if workspace is not None:
         ws_ptr = _dev_ptr(workspace, "workspace")
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(_lib.pa_decode_append(
-        _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_new, "k_new", dt),
-        _dev_ptr(v_new, "v_new", dt), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
-        _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
-        block_tables.shape[1], int(max_context_len), float(scale), int(partition_size), ws_ptr,
-        ws_bytes, _dtype_code(k_cache), _stream(stream, q.device)))
+    guard, st = _on_device((out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                            workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_append(
+            _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), _dev_ptr(k_new, "k_new", dt),
+            _dev_ptr(v_new, "v_new", dt), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache", dt), _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
+            block_tables.shape[1], int(max_context_len), float(scale), int(partition_size),
+            ws_ptr, ws_bytes, _dtype_code(k_cache), st))
 
 
 def _fp8_decode_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
@@ -354,11 +386,13 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cont
     torch = _torch()
     a = _fp8_decode_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                          workspace)
-    _check(_lib.pa_decode_fp8(
-        _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16), a["k_cache"],
-        a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"], *a["sizes"],
-        int(max_context_len), float(scale), int(partition_size), *a["ws"],
-        _stream(stream, q.device)))
+    guard, st = _on_device((out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                            context_lens, workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_fp8(
+            _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16), a["k_cache"],
+            a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"], *a["sizes"],
+            int(max_context_len), float(scale), int(partition_size), *a["ws"], st))
 
 
 def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale, block_tables,
@@ -372,12 +406,14 @@ def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scal
     s, _, hkv, d = a["sizes"][:4]
     if k_new.shape != (s, hkv, d) or v_new.shape != k_new.shape:
         raise ValueError("k_new/v_new must be [S, num_kv_heads, head_dim]")
-    _check(_lib.pa_decode_append_fp8(
-        _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16),
-        _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
-        a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"],
-        *a["sizes"], int(max_context_len), float(scale), int(partition_size), *a["ws"],
-        _stream(stream, q.device)))
+    guard, st = _on_device((out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale,
+                            block_tables, context_lens, workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_append_fp8(
+            _dev_ptr(out, "out", torch.bfloat16), _dev_ptr(q, "q", torch.bfloat16),
+            _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
+            a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"],
+            *a["sizes"], int(max_context_len), float(scale), int(partition_size), *a["ws"], st))
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
@@ -397,13 +433,15 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start
     if block_tables.dim() != 2 or block_tables.shape[0] != s or query_start.shape != (s + 1,):
         raise ValueError("block_tables must be [S, max_blocks], query_start [S + 1]")
     bf = torch.bfloat16
-    _check(_lib.pa_prefill(
-        _dev_ptr(out, "out", bf), _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf),
-        _dev_ptr(v_cache, "v_cache", bf), _dev_ptr(block_tables, "block_tables", torch.int32),
-        _dev_ptr(context_lens, "context_lens", torch.int32),
-        _dev_ptr(query_start, "query_start", torch.int32), s, total_q, hq, hkv, d, bs, nb,
-        block_tables.shape[1], int(max_query_len), float(scale), PA_BF16,
-        _stream(stream, q.device)))
+    guard, st = _on_device((out, q, k_cache, v_cache, block_tables, context_lens, query_start),
+                           stream)
+    with guard:
+        _check(_lib.pa_prefill(
+            _dev_ptr(out, "out", bf), _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf),
+            _dev_ptr(v_cache, "v_cache", bf), _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(context_lens, "context_lens", torch.int32),
+            _dev_ptr(query_start, "query_start", torch.int32), s, total_q, hq, hkv, d, bs, nb,
+            block_tables.shape[1], int(max_query_len), float(scale), PA_BF16, st))
 
 
 def pa_device_errors(stream=None) -> int:
