@@ -28,6 +28,8 @@ finished requests return their blocks to the free list.
 
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 import torch
 
@@ -36,6 +38,17 @@ from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_dec
                pa_kv_append_fp8, pa_prefill)
 
 _TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}
+
+
+def _on_stream(method):
+    """Run the method with the cache's stream current (when it has one), so the
+    tables' host-to-device copies and the buffers it allocates are ordered with
+    the kernels it launches on that stream."""
+    @functools.wraps(method)
+    def run(self, *args, **kwargs):
+        with torch.cuda.stream(self.stream):
+            return method(self, *args, **kwargs)
+    return run
 
 
 class PagedKVCache:
@@ -82,6 +95,7 @@ class PagedKVCache:
         return torch.from_numpy(np.ascontiguousarray(a)).pin_memory().to(self.device,
                                                                           non_blocking=True)
 
+    @_on_stream
     def write(self, seq_ids, counts, k_rows, v_rows):
         """Append counts[i] tokens to seq_ids[i]; k_rows/v_rows are [sum(counts), Hkv, d]
         device tensors in sequence order. Returns the host slot mapping."""
@@ -98,6 +112,7 @@ class PagedKVCache:
         return slots
 
     # -------------------------------------------------------------- prefill
+    @_on_stream
     def prefill(self, q, k_rows, v_rows, seq_ids, counts, scale: float | None = None, out=None):
         """Append counts[i] tokens to seq_ids[i] and attend them causally: q, k_rows,
         v_rows are [sum(counts), H, d] device tensors in sequence order."""
@@ -113,12 +128,14 @@ class PagedKVCache:
         return out
 
     # --------------------------------------------------------------- decode
+    @_on_stream
     def tables(self, seq_ids, max_blocks_per_seq: int | None = None):
         """(block_tables, context_lens) of the sequences, as device int32 tensors."""
         mbps = max_blocks_per_seq or max(1, max(self.bm.seq_num_blocks(s) for s in seq_ids))
         tables, lens = self.bm.block_tables(seq_ids, mbps)
         return self._to_device(tables), self._to_device(lens), int(lens.max(initial=0))
 
+    @_on_stream
     def workspace(self, num_seqs, num_heads, max_context_len, partition_size=0):
         need = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_dim,
                                          max_context_len, partition_size)
@@ -126,6 +143,7 @@ class PagedKVCache:
             self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
         return self._workspace if need > 0 else None
 
+    @_on_stream
     def decode(self, q, seq_ids, scale: float | None = None, partition_size: int = 0, out=None):
         num_seqs, num_heads, _ = q.shape
         block_tables, context_lens, max_len = self.tables(seq_ids)
@@ -143,6 +161,7 @@ class PagedKVCache:
                       scale, partition_size, ws, stream=self.stream)
         return out
 
+    @_on_stream
     def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
                     out=None, fused: bool = True):
         if not fused:
