@@ -101,7 +101,8 @@ def block_permutation(num_blocks: int, seed: int) -> np.ndarray:
 
 def e4m3_scales(num_kv_heads: int):
     """Per-KV-head scales of an E4M3 cache for rows drawn from N(0, 1): around
-    1/32, so |x| / scale reaches ~150 of the format's 448, and not powers of two
-    (the quantising division then rounds). Returns float32 (k_scale, v_scale)."""
+    1/32, so |x| / scale reaches ~150 of the format's 448. K head 0 is exactly
+    1/32 (the quantising division is exact there); every other scale is not a
+    power of two, so the division rounds. Returns float32 (k_scale, v_scale)."""
     h = np.arange(num_kv_heads, dtype=np.float64)
     return ((1.0 + 0.37 * h) / 32.0).astype(np.float32), ((1.3 + 0.29 * h) / 32.0).astype(np.float32)
