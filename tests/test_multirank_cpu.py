@@ -110,3 +110,23 @@ def test_reference_arm_sample_is_bounded_and_valid():
         assert small.shared_prefix == 0 and small.ghost_lens == ()
         assert small.num_blocks >= sum(-(-(n + 1) // small.block_size) for n in small.context_lens)
         assert str(small.num_seqs) in note
+
+
+def test_decode_step_bytes_are_the_oracles_per_token_bytes():
+    """bench.py's algorithmic bytes per decode step (the roofline's numerator):
+    every attended token (context plus the appended one) costs one layer's K
+    and V rows, the oracle's per-token figure pinned to the pages' 128 KiB for
+    32 layers."""
+    from oracle import blocks as oblk
+    from workloads import configs
+
+    bench = _bench()
+    wl = configs.llama3_8b_layer()
+    tokens = sum(n + 1 for n in wl.context_lens)
+    assert tokens == 10_586
+    assert bench.kv_bytes(wl) == tokens * oblk.kv_bytes_per_token(1, 8, 128, 2) == 43_360_256
+    fp8 = configs.Workload(**{**wl.__dict__, "kv_dtype": "fp8_e4m3"})
+    assert bench.kv_bytes(fp8) * 2 == bench.kv_bytes(wl)
+    tiny = configs.tiny()
+    assert bench.kv_bytes(tiny) == sum(n + 1 for n in tiny.context_lens) * \
+        oblk.kv_bytes_per_token(1, 2, 64, 4)
