@@ -319,6 +319,14 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
  * [8, 256]. The result does not depend on block_size or on the physical
  * placement of the blocks. Work is handed to CTAs longest first (an order
  * over all sequences' items found in the kernel); this affects speed only.
+ * The grid has one CTA per KV head and work item of 256 / (num_heads /
+ * num_kv_heads) query rows, sized for max_query_len rows per sequence: if
+ * num_seqs * ceil(max_query_len / that) * num_kv_heads exceeds 2^31 - 1 the
+ * call returns PA_ERR_UNSUPPORTED. num_seqs, total_q or max_query_len 0 is a
+ * no-op; a negative one, a null pointer, a misaligned pointer (16 bytes for
+ * out, q and the caches, 4 for the int32 arrays), max_query_len > total_q or
+ * a scale that is not finite and > 0 returns PA_ERR_INVALID; launch failures
+ * return PA_ERR_CUDA.
  */
 int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                const int32_t* block_tables, const int32_t* context_lens,

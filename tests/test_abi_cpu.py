@@ -99,6 +99,43 @@ def test_append_and_copy_reject_on_host():
         pa.PA_ERR_INVALID
 
 
+def _prefill(**over):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, qs=FAKE, S=2, tq=300, Hq=32,
+             Hkv=8, D=128, bs=16, nb=64, mbps=8, maxq=200, scale=0.1, dt=pa.PA_BF16)
+    a.update(over)
+    st = pa._lib.pa_prefill(a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["qs"], a["S"],
+                            a["tq"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["nb"], a["mbps"],
+                            a["maxq"], a["scale"], a["dt"], None)
+    return st, pa._lib.pa_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status,words", [
+    (dict(dt=pa.PA_F32), pa.PA_ERR_UNSUPPORTED, "dtype"),
+    (dict(D=64), pa.PA_ERR_UNSUPPORTED, "head_dim"),
+    (dict(Hq=24), pa.PA_ERR_UNSUPPORTED, "group"),
+    (dict(Hq=30), pa.PA_ERR_INVALID, "multiple"),
+    (dict(bs=4), pa.PA_ERR_UNSUPPORTED, "block_size"),
+    (dict(bs=24), pa.PA_ERR_UNSUPPORTED, "block_size"),
+    (dict(maxq=301), pa.PA_ERR_INVALID, "max_query_len"),
+    (dict(scale=0.0), pa.PA_ERR_INVALID, "scale"),
+    (dict(scale=float("nan")), pa.PA_ERR_INVALID, "scale"),
+    (dict(S=-1), pa.PA_ERR_INVALID, "negative"),
+    (dict(k=None), pa.PA_ERR_INVALID, "null"),
+    # one CTA per KV head and work item: 65,535 sequences of up to 2^20 rows
+    # would need more than 2^31 - 1 CTAs
+    (dict(S=65535, tq=1 << 20, maxq=1 << 20), pa.PA_ERR_UNSUPPORTED, "grid"),
+    (dict(qs=ctypes.c_void_p(0x10002)), pa.PA_ERR_INVALID, "misaligned"),
+])
+def test_prefill_rejects_on_host(over, status, words):
+    st, msg = _prefill(**over)
+    assert st == status and words in msg, msg
+
+
+def test_prefill_empty_batch_is_a_no_op():
+    for over in (dict(S=0), dict(tq=0, maxq=0), dict(maxq=0)):
+        assert _prefill(**over)[0] == pa.PA_OK
+
+
 def test_partition_size_and_workspace():
     for s, h, n in [(8, 8, 4101), (256, 8, 4096), (1, 1, 7), (16, 8, 32768), (64, 8, 3054)]:
         p = pa.pa_decode_partition_size(s, h, n)
