@@ -99,6 +99,45 @@ def test_append_and_copy_reject_on_host():
         pa.PA_ERR_INVALID
 
 
+def test_e4m3_swap_and_fused_step_reject_on_host():
+    lib, F, E = pa._lib, FAKE, pa.PA_FP8_E4M3
+    err = lambda: lib.pa_last_error().decode()  # noqa: E731
+    # E4M3 caches go through the _fp8 entry points
+    assert lib.pa_kv_append(F, F, F, 3, F, F, 4, 4, 2, 128, E, None) == pa.PA_ERR_UNSUPPORTED
+    assert "pa_kv_append_fp8" in err()
+    assert _decode(dt=E)[0] == pa.PA_ERR_UNSUPPORTED
+    # pa_kv_append_fp8: scales present and aligned, head_dim a multiple of 16
+    assert lib.pa_kv_append_fp8(F, F, F, 3, F, F, None, F, 4, 4, 2, 128, None) == \
+        pa.PA_ERR_INVALID
+    assert lib.pa_kv_append_fp8(F, F, F, 3, F, F, F, F, 4, 4, 2, 40, None) == \
+        pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_kv_append_fp8(F, F, F, 3, F, F, ctypes.c_void_p(0x10002), F, 4, 4, 2, 128,
+                                None) == pa.PA_ERR_INVALID
+    assert lib.pa_kv_append_fp8(F, F, F, 0, F, F, F, F, 4, 4, 2, 128, None) == pa.PA_OK
+    # pa_decode_fp8: head_dim 128 only, scales required
+    fp8 = lambda **o: lib.pa_decode_fp8(  # noqa: E731
+        F, F, F, F, o.get("ks", F), F, F, F, 2, 32, 8, o.get("D", 128), 16, 64, 8, 100, 0.1, 0,
+        None, 0, None)
+    assert fp8(D=64) == pa.PA_ERR_UNSUPPORTED and "head_dim" in err()
+    assert fp8(ks=None) == pa.PA_ERR_INVALID and "scale" in err()
+    # fused steps need the new rows
+    assert lib.pa_decode_append(F, F, None, F, F, F, F, F, 2, 32, 8, 128, 16, 64, 8, 100, 0.1, 0,
+                                None, 0, pa.PA_BF16, None) == pa.PA_ERR_INVALID
+    assert lib.pa_decode_append_fp8(F, F, F, ctypes.c_void_p(0x10008), F, F, F, F, F, F, 2, 32, 8,
+                                    128, 16, 64, 8, 100, 0.1, 0, None, 0, None) == \
+        pa.PA_ERR_INVALID
+    # pa_swap_blocks: pointers, pair count, block bytes
+    swap = lambda **o: lib.pa_swap_blocks(  # noqa: E731
+        o.get("dk", F), F, 4, F, F, 4, o.get("m", F), o.get("n", 2), o.get("bs", 4), 2,
+        o.get("D", 64), o.get("dt", pa.PA_BF16), None)
+    assert swap(n=0) == pa.PA_OK
+    assert swap(n=-1) == pa.PA_ERR_INVALID
+    assert swap(dk=None) == pa.PA_ERR_INVALID
+    assert swap(m=ctypes.c_void_p(0x10004)) == pa.PA_ERR_INVALID
+    assert swap(bs=1, D=2, dt=E) == pa.PA_ERR_UNSUPPORTED            # 4-byte blocks
+    assert swap(dt=9) == pa.PA_ERR_UNSUPPORTED
+
+
 def _prefill(**over):
     a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, qs=FAKE, S=2, tq=300, Hq=32,
              Hkv=8, D=128, bs=16, nb=64, mbps=8, maxq=200, scale=0.1, dt=pa.PA_BF16)
