@@ -73,6 +73,13 @@ def test_reference_arm_under_two_ranks_prints_once():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "e2e",
+                "cpu_baseline"):
+        assert key in line, key
+    assert line["n_gpus"] == 2 and line["steps"] == 1 and line["value"] > 0
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"]["value"] == line["value"] and line["config"]["workload"]
 
 
 def test_prefill_flop_count_is_the_causal_pair_count():
