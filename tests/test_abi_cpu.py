@@ -201,10 +201,15 @@ def _snapshot_oracle(ob, seqs):
     return [list(ob.tables[s]) for s in seqs], [ob.lengths[s] for s in seqs], ob.num_free()
 
 
-def test_block_manager_matches_oracle_on_random_operations():
-    rng = np.random.default_rng(12)
-    nb, bs = 300, 4
+@pytest.mark.parametrize("seed,nb,bs", [(12, 300, 4), (13, 64, 1), (14, 500, 16), (15, 40, 3),
+                                         (16, 120, 8)])
+def test_block_manager_matches_oracle_on_random_operations(seed, nb, bs):
+    """Random add / fork / free / multi-sequence appends, native against oracle
+    after every operation; small pools run out often, block size 1 and a block
+    size that is not a power of two included."""
+    rng = np.random.default_rng(seed)
     order = rng.permutation(nb).astype(np.int32)
+    seen = {"cow": 0, "exhausted": 0}
     nat = pa.BlockManager(nb, bs)
     nat.allocator.set_free_order(order)
     ob = oblk.BlockManager(nb, bs)
@@ -232,6 +237,8 @@ def test_block_manager_matches_oracle_on_random_operations():
                 with pytest.raises(pa.PagedAttentionError) as ei:
                     nat.append_slots([live_n[i] for i in idx], counts)
                 assert ei.value.status == pa.PA_ERR_NO_BLOCKS
+                seen["exhausted"] += 1
+                assert _snapshot_native(nat, live_n) == _snapshot_oracle(ob, live_o)
                 continue
             slots_n, cows_n = nat.append_slots([live_n[i] for i in idx], counts)
             slots_o, cows_o = [], []
@@ -241,9 +248,13 @@ def test_block_manager_matches_oracle_on_random_operations():
                 cows_o += cw
             assert slots_n.tolist() == slots_o
             assert [tuple(x) for x in cows_n.tolist()] == cows_o
+            seen["cow"] += len(cows_o)
         assert _snapshot_native(nat, live_n) == _snapshot_oracle(ob, live_o)
         for b in range(0, nb, 7):
             assert nat.allocator.refcount(b) == ob.refcount[b]
+    # one token per block: a shared tail is always full, so nothing is ever copied
+    assert (seen["cow"] == 0) if bs == 1 else (seen["cow"] > 0)
+    assert seen["exhausted"] > 0 or nb >= 300
 
 
 def test_block_manager_worked_example_and_exhaustion(golden):
