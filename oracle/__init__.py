@@ -9,8 +9,10 @@ path computes, written from three pages:
 
 `blocks` covers the block arithmetic and a reference block manager (free list,
 reference counts, copy-on-write). `attention` covers the cache writes (append,
-block copy) and decode attention in float64 over the logically contiguous
-context that the block table describes.
+block copy, block swap) and decode and causal (chunked) prefill attention in
+float64 over the logically contiguous context that the block table describes.
+`quant` covers the 8-bit E4M3 cache format (encode with round-to-nearest-even
+and saturation, exact decode, per-head scales).
 
 Only the test suite, the smoke check and the benchmark's CPU-baseline leg may
 import this package. It shares no code with the CUDA library and the library
