@@ -79,16 +79,6 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, block_
     return out
 
 
-def decode_one(q_vec, k_cache, v_cache, block_table, length: int, scale: float, block_size: int,
-               kv_head: int):
-    """One (sequence, query head) output, gathering only that KV head: [d] float64."""
-    if length == 0:
-        return np.zeros(q_vec.shape[-1], dtype=np.float64)
-    keys = gather_context(k_cache[:, :, kv_head:kv_head + 1], block_table, length, block_size)
-    values = gather_context(v_cache[:, :, kv_head:kv_head + 1], block_table, length, block_size)
-    return softmax_attention(q_vec, keys[:, 0, :], values[:, 0, :], scale)
-
-
 def kv_append(k_cache, v_cache, k_new, v_new, slot_mapping, block_size: int):
     """Copies of the caches with row i of k_new/v_new written at slot_mapping[i].
 

@@ -371,25 +371,6 @@ def check_swap_roundtrip():
     assert not back_k[0].any() and not back_v[4].any()
 
 
-def check_swap_roundtrip():
-    """Swapping blocks out to another pool and back restores them exactly and
-    touches nothing else."""
-    rng = np.random.default_rng(13)
-    dev_k = rng.standard_normal((6, 4, 2, 3))
-    dev_v = rng.standard_normal((6, 4, 2, 3))
-    host_k = np.zeros((4, 4, 2, 3))
-    host_v = np.zeros((4, 4, 2, 3))
-    out_pairs = np.array([[5, 0], [1, 3], [2, 1]])
-    hk, hv = oatt.swap_blocks(host_k, host_v, dev_k, dev_v, out_pairs)
-    assert np.array_equal(hk[0], dev_k[5]) and np.array_equal(hv[3], dev_v[1])
-    assert np.array_equal(hk[2], host_k[2])
-    back_k, back_v = oatt.swap_blocks(np.zeros_like(dev_k), np.zeros_like(dev_v), hk, hv,
-                                      out_pairs[:, ::-1])
-    for src, _ in out_pairs:
-        assert np.array_equal(back_k[src], dev_k[src]) and np.array_equal(back_v[src], dev_v[src])
-    assert not back_k[0].any() and not back_v[4].any()
-
-
 
 # ---------------------------------------------------------------- E4M3 codes
 
@@ -428,6 +409,39 @@ def check_e4m3_roundtrip():
     assert np.array_equal(oq.e4m3_encode(oq.e4m3_decode(codes).astype(np.float32)), codes)
     vals = oq.e4m3_decode(codes)
     assert np.nanmax(vals) == 448.0 and np.nanmin(vals) == -448.0
+
+
+def check_e4m3_scale():
+    """The per-head scale: the stored code is that of value / scale, the cache
+    value is decode(code) * scale ("What is paged attention in vLLM, and why
+    does it matter?", Trade-offs and edge cases, fourth point: narrower cache
+    values; the scale convention is the E4M3 reading)."""
+    # 3 / 0.5 = 6 = 1.5 * 2^2: exponent field 2 + 7 = 9, mantissa 4 -> 0x4C
+    assert int(oq.quantize(np.float32(3.0), np.float32(0.5))) == 0x4C
+    # and back: 6 * 0.5 = 3
+    assert float(oq.dequantize(np.uint8(0x4C), 0.5)) == 3.0
+    # decode(0x3A) = 1.25; times a scale that is not a power of two
+    assert float(oq.dequantize(np.uint8(0x3A), np.float32(0.3))) == 1.25 * float(np.float32(0.3))
+    # a power-of-two scale divides exactly: quantise(x, 1/32) is the code of 32 x
+    rng = np.random.default_rng(23)
+    x = (rng.standard_normal(512) * 4).astype(np.float32)
+    assert np.array_equal(oq.quantize(x, np.float32(1 / 32)), oq.e4m3_encode(32 * x))
+    # The division is float32 and its rounding can decide the code. With
+    # x = 2.375 - 2^-22 (= 9961471 * 2^-22) and s = 2 - 2^-23 (= 16777215 * 2^-23)
+    # the exact quotient is 19922942 / 16777215 = 1.1875 - 0.8125 / 16777215,
+    # 4.84e-8 below 1.1875; the float32 spacing there is 2^-23 = 1.19e-7, so the
+    # float32 quotient is 1.1875 exactly, the midpoint between the E4M3 values
+    # 1.125 (0x39) and 1.25 (0x3A), and ties-to-even gives 0x3A (even mantissa
+    # 2). Dividing in float64 instead would keep the quotient below the
+    # midpoint and give 0x39.
+    xs = np.float32(9961471 * 2.0 ** -22)
+    ss = np.float32(16777215 * 2.0 ** -23)
+    assert float(xs) == 2.375 - 2.0 ** -22 and float(ss) == 2.0 - 2.0 ** -23
+    assert int(oq.quantize(xs, ss)) == 0x3A
+    # scales broadcast per KV head: column h uses scale[h]
+    rows = np.array([[3.0, 3.0], [-1.5, 0.75]], dtype=np.float32)
+    sc = np.array([0.5, 0.25], dtype=np.float32)
+    assert oq.quantize(rows, sc).tolist() == [[0x4C, 0x54], [0xC4, 0x44]]
 
 
 # ------------------------------------------------------------------ prefill
@@ -532,6 +546,7 @@ ATTENTION_CHECKS = [
     check_brute_force_tiny, check_sdpa_identity_table, check_closed_forms,
     check_placement_and_sharing_invariance, check_append_and_copy_roundtrip,
     check_swap_roundtrip, check_e4m3_against_torch, check_e4m3_hand_values, check_e4m3_roundtrip,
+    check_e4m3_scale,
     check_prefill_single_query_is_decode, check_prefill_full_matches_causal_sdpa,
     check_prefill_first_row_and_chunks, check_prefill_brute_force,
 ]

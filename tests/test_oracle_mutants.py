@@ -73,7 +73,33 @@ def _swap_wrong_index(dk, dv, sk, sv, mapping):
     return k, v
 
 
+def _quantize_times_scale(x, scale):
+    return _ORIG_E4M3(np.asarray(x, np.float32) * np.asarray(scale, np.float32))
+
+
+def _quantize_float64(x, scale):
+    # divides in float64 and picks the nearest E4M3 value of that quotient with
+    # no rounding to float32 in between (nearest finite code by magnitude)
+    q = np.asarray(x, np.float32).astype(np.float64) / np.asarray(scale, np.float64)
+    codes = np.arange(0x7F, dtype=np.uint8)
+    mags = oq.e4m3_decode(codes)
+    near = codes[np.argmin(np.abs(np.abs(q)[..., None] - mags), axis=-1)]
+    return (near | (np.signbit(q).astype(np.uint8) << 7)).astype(np.uint8)
+
+
+def _dequantize_divides(codes, scale):
+    return oq.e4m3_decode(codes) / np.asarray(scale, np.float64)
+
+
+def _quantize_first_scale_only(x, scale):
+    return _ORIG_E4M3(np.asarray(x, np.float32) / np.asarray(scale, np.float32).ravel()[0])
+
+
 MUTANTS = {
+    "quantize_multiplies_by_scale": (oq, "quantize", _quantize_times_scale),
+    "quantize_divides_in_float64": (oq, "quantize", _quantize_float64),
+    "quantize_ignores_head_scales": (oq, "quantize", _quantize_first_scale_only),
+    "dequantize_divides_by_scale": (oq, "dequantize", _dequantize_divides),
     "prefill_diagonal_hidden": (oatt, "causal_visible",
                                 lambda L, pos: np.arange(L)[None, :] < np.asarray(pos)[:, None]),
     "prefill_unmasked": (oatt, "causal_visible",
