@@ -647,7 +647,8 @@ def run_b200(args, wl, rank, world, local_rank):
             c.step()
         torch.cuda.synchronize(device)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
+        early = 0 if os.environ.get("PA_BENCH_NO_EARLY") else pa.PA_DECODE_EARLY_CACHE_READS
+        with torch.cuda.graph(graph, stream=stream), pa.decode_options(early):
             for c in layer_calls:
                 c.step()
         for _ in range(3):

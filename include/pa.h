@@ -172,6 +172,30 @@ int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
 int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len);
 
 /*
+ * pa_set_decode_options — options of the decode calls (pa_decode,
+ * pa_decode_append, their _fp8 forms and pa_decode_noalloc) made later by the
+ * calling host thread, until changed; returns the previous options. A CUDA
+ * graph keeps the options its calls were captured with. Not from the pages:
+ * a launch-scheduling option of this library.
+ *
+ *   PA_DECODE_EARLY_CACHE_READS  The decode kernels are launched with
+ *     programmatic dependent launch, so they may start while the previous
+ *     kernel on the stream drains. Normally they wait for it before reading
+ *     anything. With this option they read the context lengths, the block
+ *     tables and the cached K/V at once, filling their load pipelines in the
+ *     previous kernel's tail, and wait only before reading q (and k_new /
+ *     v_new) and before writing anything. Set it only when no kernel that can
+ *     still be running when a decode call starts writes that call's cache
+ *     blocks, block tables or context lengths: the usual case of a layer loop,
+ *     where the kernel before attention produces q and the new K/V rows, and
+ *     tables, lengths and copy-on-write copies were set up before the step's
+ *     first layer. With the option and a kernel that does write them, the
+ *     results are undefined.
+ */
+#define PA_DECODE_EARLY_CACHE_READS 0x1u
+unsigned int pa_set_decode_options(unsigned int options);
+
+/*
  * pa_decode_workspace_bytes — bytes of workspace pa_decode needs for these
  * sizes (0 when no sequence can span more than one partition).
  * partition_size = 0 means the automatic choice.
@@ -206,10 +230,13 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
  *                  pa_decode_partition_size(). A sequence longer than one
  *                  partition is split; partial results (max, sum, unnormalised
  *                  output) go to the workspace and a second kernel combines
- *                  them with a log-sum-exp rescale.
+ *                  them with a log-sum-exp rescale, in partition order.
  *   workspace      device scratch of at least pa_decode_workspace_bytes(...)
  *                  bytes (may be NULL when that is 0). Contents on entry are
- *                  ignored; calls sharing one workspace must not overlap.
+ *                  ignored: it needs no clearing, before the first call or
+ *                  between calls of any shape (every value the merge reads is
+ *                  written by the same call first). Calls sharing one
+ *                  workspace must not overlap on the GPU.
  * Supported: dtype PA_F32 or PA_BF16; head_dim 64 or 128; num_heads /
  * num_kv_heads in {1, 2, 4, 8}; block_size a power of two in [1, 256].
  * The result for a sequence depends only on its logical tokens and on
@@ -351,9 +378,13 @@ int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cach
  *   - A call whose pa_decode_workspace_bytes(...) exceeds that size returns
  *     PA_ERR_INVALID before launching anything (raise partition_size, split
  *     the batch, or use pa_decode with your own workspace).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture. Later calls do no set-up.
+ *   - The first call in each CUDA context (normally: on each device) looks
+ *     up the array's device address (cudaGetSymbolAddress) and caches it for
+ *     that context; make that first call before any stream capture. Later
+ *     calls in the context do no set-up. A context created later on the same
+ *     device (after cudaDeviceReset) gets its own lookup.
+ *   - Arguments are checked exactly as pa_decode checks them, before the size
+ *     check below: a bad argument is reported as such.
  *   - Nothing here allocates: no cudaMalloc, cudaFree or allocating library
  *     routine.
  *   - All calls on a device share the one array and it keeps the last call's

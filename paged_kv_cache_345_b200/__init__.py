@@ -35,6 +35,7 @@ __all__ = [
     "pa_prefill",
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
+    "pa_set_decode_options", "PA_DECODE_EARLY_CACHE_READS", "decode_options",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
@@ -68,6 +69,7 @@ _sig("pa_kv_append_fp8", _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i
 _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
+_sig("pa_set_decode_options", ctypes.c_uint, ctypes.c_uint)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _f32, _i32, _vp, _sz, _i32, _vp)
@@ -109,7 +111,8 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 
 EXPORTED = (
     "pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_swap_blocks",
-    "pa_decode_partition_size", "pa_decode_workspace_bytes", "pa_decode", "pa_decode_append",
+    "pa_decode_partition_size", "pa_set_decode_options", "pa_decode_workspace_bytes",
+    "pa_decode", "pa_decode_append",
     "pa_decode_fp8", "pa_decode_append_fp8", "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
@@ -282,6 +285,31 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None) -> No
 
 def pa_decode_partition_size(num_seqs: int, num_kv_heads: int, max_context_len: int) -> int:
     return int(_lib.pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len))
+
+
+PA_DECODE_EARLY_CACHE_READS = 0x1
+
+
+def pa_set_decode_options(options: int) -> int:
+    """Options of this host thread's later decode calls (PA_DECODE_EARLY_CACHE_READS);
+    returns the previous options. See include/pa.h for when the option is safe."""
+    return int(_lib.pa_set_decode_options(options))
+
+
+class decode_options:
+    """Context manager: `with decode_options(PA_DECODE_EARLY_CACHE_READS): ...`
+    sets this thread's decode options and restores the previous ones on exit."""
+
+    def __init__(self, options: int):
+        self.options = options
+
+    def __enter__(self):
+        self.previous = pa_set_decode_options(self.options)
+        return self
+
+    def __exit__(self, *exc):
+        pa_set_decode_options(self.previous)
+        return False
 
 
 def pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,

@@ -14,6 +14,7 @@
 #include <new>
 #include <string>
 #include <utility>
+#include <unordered_map>
 #include <vector>
 
 #include "pa.h"
@@ -62,14 +63,6 @@ struct pa_bm {
     }
     seqs.emplace_back();
     return static_cast<int32_t>(seqs.size() - 1);
-  }
-  // Fresh blocks `count` more tokens of `s` will take (a copied shared tail included).
-  int64_t blocks_needed(const Seq& s, int64_t count) const {
-    if (count <= 0) return 0;
-    int64_t extra = ceil_div(s.length + count, block_size) - ceil_div(s.length, block_size);
-    int64_t off = s.length % block_size;
-    if (off != 0 && pool->refcount[s.blocks[s.length / block_size]] > 1) extra += 1;
-    return extra;
   }
 };
 
@@ -264,15 +257,32 @@ int pa_bm_append_slots(pa_bm* bm, const int32_t* seq_ids, const int32_t* counts,
   if (std::adjacent_find(sorted.begin(), sorted.end()) != sorted.end())
     return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: a sequence id appears twice");
   const int bs = bm->block_size;
-  for (int i = 0; i < n; ++i) {
-    const Seq* s = bm->get(seq_ids[i]);
-    if (!s) return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: unknown sequence %d", seq_ids[i]);
-    if (counts[i] < 0) return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: negative count");
-    need += bm->blocks_needed(*s, counts[i]);
-    total += counts[i];
-    if (counts[i] > 0 && s->length % bs != 0 &&
-        bm->pool->refcount[s->blocks[s->length / bs]] > 1)
-      cows += 1;
+  // The apply loop below works sequence by sequence: once one sharer of a
+  // partly filled tail has copied it, the tail has one holder fewer, and the
+  // last holder writes in place. Count the same way: `dropped` holds, per
+  // shared tail, the holders that earlier sequences of this batch took away.
+  std::unordered_map<int32_t, int32_t> dropped;
+  try {
+    for (int i = 0; i < n; ++i) {
+      const Seq* s = bm->get(seq_ids[i]);
+      if (!s)
+        return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: unknown sequence %d", seq_ids[i]);
+      if (counts[i] < 0) return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: negative count");
+      if (counts[i] == 0) continue;
+      need += ceil_div(s->length + counts[i], bs) - ceil_div(s->length, bs);
+      total += counts[i];
+      if (s->length % bs != 0) {
+        const int32_t tail = s->blocks[s->length / bs];
+        int32_t& gone = dropped[tail];
+        if (bm->pool->refcount[tail] - gone > 1) {  // still shared when this sequence writes
+          cows += 1;
+          need += 1;
+          gone += 1;
+        }
+      }
+    }
+  } catch (...) {
+    return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: out of host memory");
   }
   if (total > 0 && !slot_mapping)
     return pa_fail(PA_ERR_INVALID, "pa_bm_append_slots: slot_mapping is null");

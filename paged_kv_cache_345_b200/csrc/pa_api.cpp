@@ -11,6 +11,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local unsigned int g_decode_options = 0;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -181,6 +182,12 @@ int pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, int dst_num_blocks,
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_swap_blocks launch", e);
 }
 
+unsigned int pa_set_decode_options(unsigned int options) {
+  const unsigned int old = g_decode_options;
+  g_decode_options = options & PA_DECODE_EARLY_CACHE_READS;
+  return old;
+}
+
 int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
   // The bf16 kernel runs one CTA per (group of up to 4 KV heads, partition,
   // sequence), two per SM. Aim for about three CTAs per SM if every sequence
@@ -215,15 +222,18 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads, 
   return pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, np).total;
 }
 
-static int decode_common(void* out, const void* q, const void* k_cache, const void* v_cache,
-                         const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
-                         int num_heads, int num_kv_heads, int head_dim, int block_size,
-                         int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
-                         int partition_size, void* workspace, size_t workspace_bytes,
-                         pa_dtype dtype, const void* k_new, const void* v_new,
-                         const float* k_scale, const float* v_scale, pa_stream_t stream) {
+// (C++ linkage inside the extern "C" block: an internal helper, also used by
+// pa_decode_noalloc)
+extern "C++" {
+namespace pa {
+
+int check_decode_args(const void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, const void* workspace, pa_dtype dtype,
+                      const float* k_scale, const float* v_scale, DecodeShape* shape) {
   if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode: num_seqs < 0");
-  if (num_seqs == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return pa_fail(PA_ERR_INVALID, "pa_decode: null pointer");
   const bool fp8 = dtype == PA_FP8_E4M3;
@@ -255,10 +265,10 @@ static int decode_common(void* out, const void* q, const void* k_cache, const vo
                    max_context_len,
                    static_cast<long long>(max_blocks_per_seq) * block_size);
   if (!std::isfinite(scale)) return pa_fail(PA_ERR_INVALID, "pa_decode: scale not finite");
-  if (partition_size < 0 || partition_size % pa::kChunkTokens != 0 ||
-      partition_size > pa::kMaxPartitionSize)
+  if (partition_size < 0 || partition_size % kChunkTokens != 0 ||
+      partition_size > kMaxPartitionSize)
     return pa_fail(PA_ERR_INVALID, "pa_decode: partition_size %d not a multiple of %d in [0, %d]",
-                   partition_size, pa::kChunkTokens, pa::kMaxPartitionSize);
+                   partition_size, kChunkTokens, kMaxPartitionSize);
   if (num_seqs > 65535) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: num_seqs > 65535");
   if (num_kv_heads > 65535) return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: num_kv_heads > 65535");
   if (static_cast<int64_t>(num_blocks) * block_size * num_kv_heads * head_dim *
@@ -269,7 +279,8 @@ static int decode_common(void* out, const void* q, const void* k_cache, const vo
       (workspace && !aligned(workspace, 16)))
     return pa_fail(PA_ERR_INVALID, "pa_decode: misaligned pointer");
 
-  pa::DecodeShape sh{};
+  DecodeShape& sh = *shape;
+  sh = DecodeShape{};
   sh.num_seqs = num_seqs;
   sh.num_heads = num_heads;
   sh.num_kv_heads = num_kv_heads;
@@ -284,9 +295,30 @@ static int decode_common(void* out, const void* q, const void* k_cache, const vo
   sh.num_partitions = resolve_partitions(max_context_len, &sh.partition_size);
   sh.scale = scale;
   sh.dtype = dtype;
-  if (sh.num_partitions > pa::kMaxPartitions)
+  sh.early_reads = (g_decode_options & PA_DECODE_EARLY_CACHE_READS) != 0;
+  if (sh.num_partitions > kMaxPartitions)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode: %d partitions > %d", sh.num_partitions,
-                   pa::kMaxPartitions);
+                   kMaxPartitions);
+  return PA_OK;
+}
+
+}  // namespace pa
+}  // extern "C++"
+
+static int decode_common(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                         int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void* workspace, size_t workspace_bytes,
+                         pa_dtype dtype, const void* k_new, const void* v_new,
+                         const float* k_scale, const float* v_scale, pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  pa::DecodeShape sh;
+  const int st = pa::check_decode_args(out, q, k_cache, v_cache, block_tables, context_lens,
+                                       num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                       num_blocks, max_blocks_per_seq, max_context_len, scale,
+                                       partition_size, workspace, dtype, k_scale, v_scale, &sh);
+  if (st != PA_OK) return st;
   const size_t need =
       pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, sh.num_partitions).total;
   if (need > 0 && (!workspace || workspace_bytes < need))

@@ -61,6 +61,10 @@ struct DecodeParams {
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks;
   int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
   float q_scale;  // scale * log2(e)
+  // PA_DECODE_EARLY_CACHE_READS: the caller vouches that no kernel still
+  // running when this call starts writes the cache, the block tables or the
+  // context lengths, so they may be read before the dependent-launch wait.
+  int early_reads;
 };
 
 
@@ -447,14 +451,19 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = static_cast<int>(r / p.num_heads);
   // The context length is read before the dependent-launch wait: the kernel
-  // before this one is the decode kernel of the same call, which itself waited
-  // for all earlier work before letting this kernel start, and neither writes it.
+  // before this one is the decode kernel of the same call, which waited for all
+  // earlier work before letting this kernel start (or, under
+  // PA_DECODE_EARLY_CACHE_READS, the caller vouches that nothing still running
+  // writes it), and neither kernel writes it.
   const int L = __ldg(p.context_lens + s);
   if (L < 0 || L > p.max_context_len ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size)
     return;  // flagged and zero-filled by the decode kernel
   const int np = (L + p.partition_size - 1) / p.partition_size;
   if (np <= 1) return;  // written directly by the decode kernel
+  // The next kernel may start its launch now: whatever it reads before its
+  // own wait is, by the same contract, not written here.
+  pdl_launch_dependents();
   pdl_wait();  // the partials are the decode kernel's output
   const int64_t row = r * p.num_partitions;
   const float* a = p.ws_acc + row * D + lane * E;

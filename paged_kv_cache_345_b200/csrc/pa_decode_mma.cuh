@@ -123,7 +123,14 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     prefetch_tensormap(&k_map);
     prefetch_tensormap(&v_map);
   }
-  pdl_wait();  // inputs may come from the previous kernel in the stream
+  // Inputs may come from the previous kernel in the stream. Normally every
+  // thread waits for it here. Under PA_DECODE_EARLY_CACHE_READS the context
+  // length, the block table and the cached K/V are read at once and the first
+  // ring stages fill while that kernel drains; the waits then come right
+  // before q (consumers), before the fused append reads k_new / v_new
+  // (producer), and before any write.
+  const bool early = p.early_reads != 0;
+  if (!early) pdl_wait();
   pdl_launch_dependents();
 
   // Independent loads first so their latencies overlap: the context length,
@@ -141,6 +148,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   const int64_t out_row = static_cast<int64_t>(s) * p.num_heads + kvh * G;
   uint32_t qa[D / 16][2];  // Q as the B operand (column = head of the group), 16-bit pairs
   if (warp < HB) {
+    if (early) pdl_wait();
     const uint32_t* qp = reinterpret_cast<const uint32_t*>(
         static_cast<const __nv_bfloat16*>(p.q) + (out_row + (real_row ? qr : 0)) * D);
     if constexpr (!FP8) {
@@ -176,6 +184,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 
   if (L == 0) {  // empty context: zeros for every query head of the group
+    if (early) pdl_wait();
     if (part == 0) {
       const int64_t first = static_cast<int64_t>(s) * p.num_heads + hg * HB * G;
       for (int e = threadIdx.x; e < HB * G * D; e += blockDim.x)
@@ -209,6 +218,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
         // this CTA holds the sequence's newest token: write it before reading it
         const int tn = L - 1;
         const int bn = __shfl_sync(kFullMask, ent, (tn >> lg) - base);
+        if (early) pdl_wait();  // k_new / v_new come from the previous kernel
         if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks)) {
           if constexpr (FP8)
             append_newest_rows_fp8(p, s, bn, tn & (bs - 1), hg * HB, HB, D, lane);

@@ -15,11 +15,10 @@
 // library holds these kScratchBytes, used or not. Its size caps what one call
 // may ask for; a call that would need more is rejected before any launch.
 // Host code cannot pass the array's name to a kernel (on the host that name
-// is only a stand-in, not a device address), so the first call on each
-// device looks its device address up with cudaGetSymbolAddress and keeps it.
-#include <atomic>
-#include <mutex>
-
+// is only a stand-in, not a device address), so the first call in each CUDA
+// context looks its device address up with cudaGetSymbolAddress and keeps it
+// for that context; a context made later (after cudaDeviceReset, say) loads
+// the device code again and gets its own lookup.
 #include "pa.h"
 #include "pa_internal.h"
 
@@ -31,27 +30,13 @@ static_assert(kScratchBytes == PA_DECODE_NOALLOC_SCRATCH_BYTES, "header and libr
 // Split-K partial maxima, sums and accumulators of pa_decode_noalloc calls.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device, looked up once.
-int scratch_for_current_device(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return pa_fail(PA_ERR_CUDA, "pa_decode_noalloc: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices)
-    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_noalloc: device %d beyond %d", dev, kMaxDevices);
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    if (e != cudaSuccess || !ptr)
-      return pa_fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress failed: %s",
-                     cudaGetErrorString(e));
-    g_scratch_ptr[dev] = ptr;
-  }
-  *out = g_scratch_ptr[dev];
+// Device address of g_decode_scratch in the current context, looked up once per context.
+int scratch_for_current_context(void** out) {
+  static pa::SymbolAddressCache cache;
+  const cudaError_t e = cache.get(&g_decode_scratch, out);
+  if (e != cudaSuccess)
+    return pa_fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress failed: %s",
+                   cudaGetErrorString(e));
   return PA_OK;
 }
 
@@ -65,10 +50,21 @@ extern "C" int pa_decode_noalloc(void* out, const void* q, const void* k_cache,
                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
                                  int max_blocks_per_seq, int max_context_len, float scale,
                                  int partition_size, pa_dtype dtype, pa_stream_t stream) {
-  // Size the scratch this call needs exactly as pa_decode would, and refuse
-  // before touching the device if it does not fit.
-  const size_t need = pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
-                                                max_context_len, partition_size);
+  if (num_seqs == 0) return PA_OK;
+  if (dtype == PA_FP8_E4M3)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_noalloc: E4M3 caches decode through pa_decode_fp8");
+  // pa_decode's own argument checks first, so that a bad argument is reported
+  // as such and not as a scratch shortfall; then the scratch this call needs,
+  // sized exactly as pa_decode sizes a workspace, refused before any launch if
+  // it does not fit.
+  pa::DecodeShape sh;
+  const int checked = pa::check_decode_args(
+      out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_heads, num_kv_heads,
+      head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+      partition_size, nullptr, dtype, nullptr, nullptr, &sh);
+  if (checked != PA_OK) return checked;
+  const size_t need = pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim,
+                                           sh.num_partitions).total;
   if (need > kScratchBytes)
     return pa_fail(PA_ERR_INVALID,
                    "pa_decode_noalloc: this call needs %zu bytes of split-K scratch, the limit is "
@@ -77,7 +73,7 @@ extern "C" int pa_decode_noalloc(void* out, const void* q, const void* k_cache,
                    need, kScratchBytes);
   void* scratch = nullptr;
   if (need > 0) {
-    const int st = scratch_for_current_device(&scratch);
+    const int st = scratch_for_current_context(&scratch);
     if (st != PA_OK) return st;
   }
   // Same checks, kernels and launch as pa_decode; only the workspace differs.

@@ -26,6 +26,7 @@ struct DecodeShape {
   int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
   float scale;
   pa_dtype dtype;
+  bool early_reads;  // PA_DECODE_EARLY_CACHE_READS for this call
 };
 
 // Byte offsets of the split-K workspace regions.
@@ -34,6 +35,16 @@ struct WorkspaceLayout {
 };
 WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int num_kv_heads, int head_dim,
                                  int num_partitions);
+
+// Every host-side check of a decode call except the workspace size; fills the
+// shape (partition size resolved) and returns PA_OK, or the status a call
+// would return (with the last-error text set). num_seqs must be > 0.
+int check_decode_args(const void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, const void* workspace, pa_dtype dtype,
+                      const float* k_scale, const float* v_scale, DecodeShape* shape);
 
 // Launchers (pa_kernels.cu). Return cudaSuccess or the launch error.
 cudaError_t launch_kv_append(const void* k_new, const void* v_new, const int64_t* slot_mapping,
@@ -72,5 +83,24 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
                            cudaStream_t stream);
 // Device error word of the current device (address in device memory).
 cudaError_t device_error_word(unsigned int** ptr);
+
+// Device address of a __device__ variable of this library in the current CUDA
+// context, looked up with cudaGetSymbolAddress once per context and cached.
+// The key is the context's unique id (cuCtxGetId), not the device ordinal: a
+// context created later on the same device (after cudaDeviceReset, say) loads
+// the library's device code again, possibly elsewhere, and gets its own lookup.
+class SymbolAddressCache {
+ public:
+  cudaError_t get(const void* symbol, void** out);
+
+ private:
+  static constexpr int kEntries = 64;
+  struct Entry {
+    unsigned long long ctx_id;
+    void* ptr;
+  };
+  Entry entries_[kEntries] = {};
+  int next_ = 0;
+};
 
 }  // namespace pa

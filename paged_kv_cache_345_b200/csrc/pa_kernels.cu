@@ -18,25 +18,65 @@ namespace pa {
 // reads and clears it.
 __device__ unsigned int g_error_word = 0;
 
-cudaError_t device_error_word(unsigned int** ptr) {
-  constexpr int kMaxDevices = 64;
-  static std::atomic<unsigned int*> cache[kMaxDevices];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < kMaxDevices) {
-    unsigned int* c = cache[dev].load(std::memory_order_acquire);
-    if (c) {
-      *ptr = c;
-      return cudaSuccess;
-    }
+namespace {
+
+// Unique id of the current context (0 when no context is current yet).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(ptr);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+std::mutex g_symbol_mutex;
+
+}  // namespace
+
+cudaError_t SymbolAddressCache::get(const void* symbol, void** out) {
+  unsigned long long id = current_context_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_symbol_mutex);
+    for (const Entry& e : entries_)
+      if (e.ctx_id == id && e.ptr) {
+        *out = e.ptr;
+        return cudaSuccess;
+      }
   }
-  void* addr = nullptr;
-  e = cudaGetSymbolAddress(&addr, g_error_word);
+  void* ptr = nullptr;
+  // (makes the device's primary context current if none was)
+  cudaError_t e = cudaGetSymbolAddress(&ptr, symbol);
   if (e != cudaSuccess) return e;
-  *ptr = static_cast<unsigned int*>(addr);
-  if (dev < kMaxDevices) cache[dev].store(*ptr, std::memory_order_release);
+  if (!ptr) return cudaErrorInvalidSymbol;
+  id = current_context_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(g_symbol_mutex);
+    entries_[next_] = Entry{id, ptr};
+    next_ = (next_ + 1) % kEntries;
+  }
+  *out = ptr;
   return cudaSuccess;
+}
+
+cudaError_t device_error_word(unsigned int** ptr) {
+  static SymbolAddressCache cache;
+  void* addr = nullptr;
+  cudaError_t e = cache.get(&g_error_word, &addr);
+  if (e == cudaSuccess) *ptr = static_cast<unsigned int*>(addr);
+  return e;
 }
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -470,6 +510,7 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   p.partition_size = sh.partition_size;
   p.num_partitions = sh.num_partitions;
   p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
+  p.early_reads = sh.early_reads ? 1 : 0;
   switch (sh.head_dim) {
     case 64: return dispatch_group<64>(sh, p, k_cache, v_cache, stream);
     case 128: return dispatch_group<128>(sh, p, k_cache, v_cache, stream);

