@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="llama3_8b_layer",
                     choices=["llama3_8b_layer", "large_batch", "shared_prefix", "long_context",
-                             "swap", "prefill", "chunked_prefill"])
+                             "swap", "prefill", "chunked_prefill", "layout_sweep"])
     ap.add_argument("--placement", choices=["random", "identity"], default="random",
                     help="physical block order: a seeded permutation (default) or identity "
                          "(each sequence's blocks contiguous in memory)")
@@ -61,6 +61,10 @@ def parse_args():
                     help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-back-to-back", action="store_true")
+    ap.add_argument("--no-side-workloads", action="store_true",
+                    help="skip the large-batch, long-context and shared-prefix lines")
+    ap.add_argument("--no-early-reads", action="store_true",
+                    help="decode without PA_DECODE_EARLY_CACHE_READS")
     ap.add_argument("--layers", type=int, default=32,
                     help="cache replicas of the back-to-back figure (one per model layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -92,6 +96,17 @@ def kv_bytes(wl) -> int:
     """K and V bytes the decode step reads: every attended token, every KV head."""
     return (sum(n + 1 for n in wl.context_lens) * wl.num_kv_heads * 2 * wl.head_dim *
             wl.cache_elem_bytes)
+
+
+def kv_bytes_unique(wl) -> int:
+    """K and V bytes of the distinct physical rows the step reads: a prefix held
+    in shared blocks is stored once however many sequences attend it ("PagedAttention
+    — AI Glossary", How it works, step 4: sharers point at the same blocks). Only the
+    whole blocks of the prefix stay shared; a partly filled shared tail is copied
+    before the first divergent write, so every sequence reads its own copy of it."""
+    shared = (wl.shared_prefix // wl.block_size) * wl.block_size
+    tokens = shared + sum(n + 1 - shared for n in wl.context_lens)
+    return tokens * wl.num_kv_heads * 2 * wl.head_dim * wl.cache_elem_bytes
 
 
 # ------------------------------------------------------------- rank plumbing
@@ -226,6 +241,11 @@ class StepCalls:
         import paged_kv_cache_345_b200 as pa
 
         self.lib = pa._lib
+        # the calls below hold raw pointers only: keep every tensor they point
+        # into alive for as long as this object (a cache copy made for one
+        # layer would otherwise be freed while a captured graph still uses it)
+        self._keep = (cache.k_cache, cache.v_cache, getattr(cache, "k_scale", None),
+                      getattr(cache, "v_scale", None), dict(dev))
         s, hq, d = dev["q"].shape
         nb, bs, hkv, _ = cache.k_cache.shape
         self.fp8 = cache.k_cache.dtype == torch.uint8
@@ -524,6 +544,326 @@ def load_traffic(kernel_key: str, files=DECODE_SOURCES):
         return None
 
 
+def load_peak(key="hbm_gbs", fallback=FALLBACK_HBM_GBS):
+    """(peak, source): the measured figure from MEASURED_PEAKS.json, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))[key]), "measured"
+    return fallback, "fallback"
+
+
+class L2Flush:
+    """Between timed steps: write a buffer larger than L2, then read another one,
+    so a step starts with L2 holding clean, unrelated lines (a write alone would
+    leave the step paying for the write-back of dirty lines)."""
+
+    def __init__(self, device):
+        import torch
+
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.w = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
+        self.r = torch.ones((2 * l2 + (64 << 20)) // 4, dtype=torch.float32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+    def describe(self):
+        return (f"flushed between steps ({self.w.numel() >> 20} MiB written, then "
+                f"{(self.r.numel() * 4) >> 20} MiB of another buffer read; outside the timed "
+                "events)")
+
+
+def cold_steps(step, flush, steps, warmup, stream, barrier=None):
+    """Per-step device times (ms): each step bracketed by CUDA events on the
+    launching stream, L2 flushed before it, outside the events."""
+    import torch
+
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    if barrier:
+        barrier()
+    for i in range(steps):
+        flush()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def host_allocator_metrics(steps: int = 10):
+    """The host block manager's decode step on the large batch (256 lognormal
+    sequences in a fragmented 80,000-block pool): append_slots (next slot, a new
+    block when a tail is full, copy-on-write when it is shared) + block_tables,
+    through the Python binding, for `steps` steps; and cache utilisation
+    (tokens / allocated slots) of the worked example's batch, before and after
+    one decode step, beside the slab figure of the same batch ("What is paged
+    attention in vLLM...", Worked example: 99.4 % vs 16.1 %)."""
+    import paged_kv_cache_345_b200 as pa
+    from workloads import configs, synth
+
+    wl = configs.large_batch(steps=steps)
+    bm = pa.BlockManager(wl.num_blocks, wl.block_size)
+    bm.allocator.set_free_order(synth.block_permutation(wl.num_blocks, wl.placement_seed))
+    ghosts = [bm.add_seq() for _ in wl.ghost_lens]
+    bm.append_slots(ghosts, list(wl.ghost_lens))
+    for i in range(0, len(ghosts), 2):
+        bm.free_seq(ghosts[i])
+    seqs = [bm.add_seq() for _ in wl.context_lens]
+    bm.append_slots(seqs, list(wl.context_lens))
+    mb = -(-(max(wl.context_lens) + steps) // wl.block_size)
+    free0 = bm.allocator.num_free()
+    times = []
+    ones = [1] * len(seqs)
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        slots, cows = bm.append_slots(seqs, ones)
+        tables, lens = bm.block_tables(seqs, mb)
+        times.append(time.perf_counter() - t0)
+    # the same step called through the C ABI with preallocated buffers (what a
+    # native caller pays): 10 more steps
+    ids = np.asarray(seqs, dtype=np.int32)
+    cnt = np.ones(len(seqs), dtype=np.int32)
+    mb2 = mb + steps // wl.block_size + 1
+    slot_buf = np.empty(len(seqs), dtype=np.int64)
+    cow_buf = np.empty((len(seqs), 2), dtype=np.int64)
+    tab_buf = np.empty((len(seqs), mb2), dtype=np.int32)
+    len_buf = np.empty(len(seqs), dtype=np.int32)
+    ncow = ctypes.c_int(0)
+    i32p, i64p = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+    args_a = (bm._h, ids.ctypes.data_as(i32p), cnt.ctypes.data_as(i32p), len(seqs),
+              slot_buf.ctypes.data_as(i64p), cow_buf.ctypes.data_as(i64p), len(seqs),
+              ctypes.byref(ncow))
+    args_t = (bm._h, ids.ctypes.data_as(i32p), len(seqs), tab_buf.ctypes.data_as(i32p), mb2,
+              len_buf.ctypes.data_as(i32p))
+    c_times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        if pa._lib.pa_bm_append_slots(*args_a) or pa._lib.pa_bm_block_tables(*args_t):
+            raise RuntimeError(pa._lib.pa_last_error().decode())
+        c_times.append(time.perf_counter() - t0)
+    new_blocks = free0 - bm.allocator.num_free()
+    held = sum(bm.seq_num_blocks(s) for s in seqs)
+    tokens = sum(bm.seq_len(s) for s in seqs)
+
+    ex = configs.llama3_8b_layer()
+    wb = pa.BlockManager(ex.num_blocks, ex.block_size)
+    wseqs = [wb.add_seq() for _ in ex.context_lens]
+    wb.append_slots(wseqs, list(ex.context_lens))
+
+    def util(b, ss):
+        t = sum(b.seq_len(x) for x in ss)
+        slots_ = sum(b.seq_num_blocks(x) for x in ss) * b.block_size
+        return t, slots_
+
+    t_pre, s_pre = util(wb, wseqs)
+    wb.append_slots(wseqs, [1] * len(wseqs))
+    t_post, s_post = util(wb, wseqs)
+    max_positions = 8192   # Llama-3-8B context length: the slab a contiguous cache reserves
+    return {
+        "allocator_step": {
+            "us_per_step_mean": 1e6 * statistics.mean(times),
+            "us_per_step_p50": 1e6 * statistics.median(times),
+            "us_per_step_c_abi_p50": 1e6 * statistics.median(c_times),
+            "sequences": len(seqs), "steps": 2 * steps, "new_blocks": int(new_blocks),
+            "what": "pa_bm_append_slots (slot, new block when the tail is full, copy-on-write "
+                    "check) + pa_bm_block_tables: the first figures through the Python binding "
+                    "(10 steps), the c_abi one through ctypes with preallocated buffers (10 "
+                    "more steps)",
+            "utilisation_after": tokens / (held * wl.block_size)},
+        "cache_utilisation": {
+            "workload": "worked example (8 requests, block 16)",
+            "paged_before_step": t_pre / s_pre, "paged_after_step": t_post / s_post,
+            "tokens_before_step": t_pre, "slots_before_step": s_pre,
+            "slab": t_pre / (len(wseqs) * max_positions),
+            "slab_slots": len(wseqs) * max_positions},
+    }
+
+
+def cpu_baseline_line(wl, bytes_step, budget_s):
+    """The oracle on the host cores (all of them, then one), bounded samples."""
+    try:
+        times, cores = cpu_oracle_run(wl, budget_s)
+    except ValueError as exc:
+        return {"value": None, "unit": "GB/s", "cores": 0, "kind": "oracle",
+                "sample": f"not run: {exc}"}
+    line = {"value": bytes_step * len(times) / sum(times) / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{len(times)} whole decode steps of the {wl.num_seqs}-sequence batch in "
+                      f"{sum(times):.1f} s (float64 NumPy)"}
+    try:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            t1, _ = cpu_oracle_run(wl, budget_s / 2)
+        line["one_core"] = {"value": bytes_step * len(t1) / sum(t1) / 1e9, "unit": "GB/s",
+                            "cores": 1,
+                            "sample": f"{len(t1)} whole decode steps in {sum(t1):.1f} s, BLAS "
+                                      "limited to one thread"}
+    except Exception as exc:  # noqa: BLE001
+        line["one_core"] = {"value": None, "sample": f"not run: {exc}"}
+    return line
+
+
+def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
+    """One more workload in the same process: the fused decode step, cold (L2
+    flushed), its rate against the HBM peak, with its own clock record."""
+    import torch
+
+    wl2 = make_workload(name, 16)
+    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl2, device)
+    ps = TUNED_PARTITION[wl2.name.split("_bs")[0]]
+    calls = StepCalls(cache, dev, max_len, wl2.scale, ps, stream)
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    ms = cold_steps(calls.step, flush, steps, warmup, stream)
+    clk = clocks.stop()
+    mean_s = statistics.mean(ms) * 1e-3
+    logical, unique = kv_bytes(wl2), kv_bytes_unique(wl2)
+    res = {"us_per_step": 1e3 * statistics.mean(ms),
+           "step_us_p10_p50_p90": [1e3 * float(np.percentile(ms, p)) for p in (10, 50, 90)],
+           "kv_bytes_per_step": unique, "GB_per_s": unique / mean_s / 1e9,
+           "frac": unique / mean_s / 1e9 / peak,
+           "attended_tokens_per_s": sum(n + 1 for n in wl2.context_lens) / mean_s,
+           "num_seqs": wl2.num_seqs, "block_size": wl2.block_size,
+           "partition_size": calls.partition_size, "steps": steps, "clocks": clk}
+    if unique != logical:
+        res["kv_bytes_logical"] = logical
+        res["GB_per_s_logical"] = logical / mean_s / 1e9
+        res["copy_on_write_pairs"] = cow_pairs
+    pa_device_errors_or_raise()
+    del calls, cache, dev, host
+    torch.cuda.empty_cache()
+    return res
+
+
+def pa_device_errors_or_raise():
+    import paged_kv_cache_345_b200 as pa
+
+    if pa.pa_device_errors() != 0:
+        raise RuntimeError("device error word set")
+
+
+def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp8=False):
+    """StepCalls over `layers` copies of the cache (one per model layer)."""
+    import paged_kv_cache_345_b200 as pa  # noqa: F401
+
+    out = []
+    for _ in range(layers):
+        view = type("CacheView", (), {})()
+        view.k_cache, view.v_cache = cache.k_cache.clone(), cache.v_cache.clone()
+        if fp8:
+            view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
+        out.append(StepCalls(view, dev, max_len, scale, ps, stream, fused=fused))
+    return out
+
+
+def back_to_back(layer_calls, stream, reps, early):
+    """One CUDA graph of the step over every layer's cache (together far larger
+    than L2, so no flush), replayed: mean time per layer (ms)."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+
+    for c in layer_calls:   # warm-up, eager
+        c.step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream), pa.decode_options(early):
+        for c in layer_calls:
+            c.step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for i in range(reps):
+        gev[i][0].record(stream)
+        graph.replay()
+        gev[i][1].record(stream)
+    torch.cuda.synchronize()
+    per_layer = statistics.mean(e[0].elapsed_time(e[1]) for e in gev) / len(layer_calls)
+    del graph
+    return per_layer
+
+
+def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early, fp8=False):
+    """End to end through the C ABI with the host copies pipelined: two pinned
+    host packs and two device packs; for step i the inputs go host -> device on
+    an upload stream (pack i % 2, once step i - 2 has finished reading it), the
+    step runs on the compute stream, its output goes device -> host on a
+    download stream, so step i + 1's input copy and step i - 1's output copy
+    overlap step i's kernels. Steps rotate over per-layer cache copies (no flush);
+    the whole pipeline of `layers` steps is one CUDA graph. Returns ms per step."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+
+    device = cache.k_cache.device
+    packs = [pack_step_inputs({k: v for k, v in host.items() if k != "_pack"}, device)
+             for _ in range(2)]
+    calls = []
+    for i in range(layers):
+        view = type("CacheView", (), {})()
+        view.k_cache, view.v_cache = cache.k_cache.clone(), cache.v_cache.clone()
+        if fp8:
+            view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
+        calls.append(StepCalls(view, packs[i % 2][1], max_len, scale, ps, stream))
+    outs_host = [torch.empty(calls[0].out.shape, dtype=calls[0].out.dtype).pin_memory()
+                 for _ in range(2)]
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    for c in calls:
+        c.step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    done = [None, None]
+    with torch.cuda.graph(graph, stream=stream), pa.decode_options(early):
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        for i, c in enumerate(calls):
+            b = i % 2
+            if done[b] is not None:
+                up.wait_event(done[b])
+            with torch.cuda.stream(up):
+                packs[b][1]["_pack"].copy_(packs[b][0]["_pack"], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(up)
+            stream.wait_event(ready)
+            c.step()
+            fin = torch.cuda.Event()
+            fin.record(stream)
+            done[b] = fin
+            down.wait_event(fin)
+            with torch.cuda.stream(down):
+                outs_host[b].copy_(c.out, non_blocking=True)
+        stream.wait_stream(up)
+        stream.wait_stream(down)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    for i in range(reps):
+        gev[i][0].record(stream)
+        graph.replay()
+        gev[i][1].record(stream)
+    torch.cuda.synchronize()
+    per_step = statistics.mean(e[0].elapsed_time(e[1]) for e in gev) / layers
+    h2d = packs[0][0]["_pack"].numel()
+    d2h = outs_host[0].numel() * outs_host[0].element_size()
+    del graph, calls
+    torch.cuda.empty_cache()
+    return per_step, h2d, d2h
+
+
+# workloads measured beside the headline one, in the same process
+SIDE_WORKLOADS = ("large_batch", "long_context", "shared_prefix")
+
+
 def run_b200(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -537,68 +877,40 @@ def run_b200(args, wl, rank, world, local_rank):
     # a stream of our own (CUDA graphs cannot be captured on the default stream)
     stream = torch.cuda.Stream(device)
     torch.cuda.set_stream(stream)
+    peak, peak_src = load_peak()
+    early = 0 if args.no_early_reads else pa.PA_DECODE_EARLY_CACHE_READS
 
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device, args.placement)
     ps = TUNED_PARTITION[wl.name.split("_bs")[0]] if args.partition_size < 0 else args.partition_size
     calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused)
-    bytes_step = kv_bytes(wl)
+    launches_per_step, part_size = calls.launches_per_step, calls.partition_size
+    num_partitions = calls.num_partitions
+    bytes_step = kv_bytes_unique(wl)
+    bytes_logical = kv_bytes(wl)
     tokens_step = sum(n + 1 for n in wl.context_lens)
-
-    # L2 flush between steps: write a buffer larger than L2, then read another
-    # one, so the timed step starts with L2 holding clean, unrelated lines (a
-    # write alone would leave the step paying for the write-back of its dirty
-    # lines).
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush_w = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
-    flush_r = torch.ones((2 * l2 + (64 << 20)) // 4, dtype=torch.float32, device=device)
-
-    class _Flush:
-        def zero_(self):
-            flush_w.zero_()
-            flush_r.sum()
-
-        def numel(self):
-            return flush_w.numel() + flush_r.numel() * 4
-
-    flush = _Flush()
+    flush = L2Flush(device)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local_rank])
         torch.cuda.synchronize(device)
 
-    # ---- device-resident steps
-    for _ in range(args.warmup):
-        flush.zero_()
-        calls.step()
-    torch.cuda.synchronize(device)
-    if pa.pa_device_errors() != 0:
-        raise RuntimeError("device error word set during warm-up")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # ---- device-resident steps (the headline): cold, L2 flushed before each
     clocks = ClockSampler(local_rank)
     clocks.start()
-    barrier()
     t_wall = time.perf_counter()
-    for i in range(args.steps):
-        flush.zero_()
-        ev[i][0].record(stream)
-        calls.step()
-        ev[i][1].record(stream)
-    barrier()
+    with pa.decode_options(early):
+        step_ms = cold_steps(calls.step, flush, args.steps, args.warmup, stream, barrier)
     wall = time.perf_counter() - t_wall
     clk = clocks.stop()
-    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    decode_ms = step_ms  # the step's kernels: (append +) decode + split-K merge
+    pa_device_errors_or_raise()
     total_ms = max_over_ranks(sum(step_ms), world, device)
-    if pa.pa_device_errors() != 0:
-        raise RuntimeError("device error word set during the timed steps")
 
     # ---- end to end: pinned host inputs -> device -> kernels -> host output
     e2e = None
     if not args.no_e2e:
         out_host = torch.empty(calls.out.shape, dtype=calls.out.dtype).pin_memory()
-        # q, new K/V rows, slot mapping, tables and lengths: one packed copy
-        h2d = host["_pack"].numel()
+        h2d = host["_pack"].numel()     # q, new K/V rows, slot mapping, tables, lengths
         d2h = out_host.numel() * out_host.element_size()
 
         def e2e_step():
@@ -606,94 +918,67 @@ def run_b200(args, wl, rank, world, local_rank):
             calls.step()
             out_host.copy_(calls.out, non_blocking=True)
 
-        for _ in range(args.warmup):
-            flush.zero_()
-            e2e_step()
-        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-        barrier()
-        for i in range(args.steps):
-            flush.zero_()
-            ee[i][0].record(stream)
-            e2e_step()
-            ee[i][1].record(stream)
-        barrier()
-        e2e_ms = max_over_ranks(sum(ee[i][0].elapsed_time(ee[i][1]) for i in range(args.steps)),
-                                world, device)
-        e2e = {"value": whole_job_rate(bytes_step, args.steps, world, e2e_ms) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / args.steps}
+        with pa.decode_options(early):
+            e_ms = cold_steps(e2e_step, flush, args.steps, args.warmup, stream, barrier)
+        e2e_ms = max_over_ranks(sum(e_ms), world, device)
+        e2e = {"value": whole_job_rate(bytes_step, args.steps, world, e2e_ms) / 1e9,
+               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.steps,
+               "how": "serial: one packed host->device copy, the step, the output copy back, "
+                      "per step, L2 flushed between steps"}
+        if world == 1 and not args.no_back_to_back:
+            ov_ms, oh2d, od2h = e2e_overlapped(cache, host, max_len, wl.scale,
+                                               calls.partition_size, stream, args.layers,
+                                               max(5, min(50, args.steps // args.layers)), early,
+                                               calls.fp8)
+            pa_device_errors_or_raise()
+            e2e["overlapped"] = {
+                "value": bytes_step / (ov_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_step": ov_ms, "h2d_bytes_per_step": oh2d, "d2h_bytes_per_step": od2h,
+                "how": f"two host/device packs, uploads and downloads on two more streams "
+                       f"overlapping the neighbouring steps, {args.layers} steps over per-layer cache copies in "
+                       "one CUDA graph (no flush)"}
 
-    # ---- back to back: the same step over `layers` different cache replicas
-    # (one per model layer, together far larger than L2, so no flush), all
-    # layers captured in one CUDA graph and replayed. Consecutive layers
-    # overlap launch and start-up through programmatic dependent launch.
+    # ---- back to back: the same step over `layers` cache copies in one graph
     b2b = None
     if not args.no_back_to_back and world == 1:
-        reps = []
-        for _ in range(args.layers):
-            kc = cache.k_cache.clone()
-            vc = cache.v_cache.clone()
-            reps.append((kc, vc))
-        del kc, vc
-        layer_calls = []
-        for kc, vc in reps:
-            view = type("CacheView", (), {})()
-            view.k_cache, view.v_cache = kc, vc
-            if calls.fp8:
-                view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
-            layer_calls.append(StepCalls(view, dev, max_len, wl.scale, calls.partition_size,
-                                         stream, fused=calls.fused))
-        for c in layer_calls:   # warm-up, eager
-            c.step()
-        torch.cuda.synchronize(device)
-        graph = torch.cuda.CUDAGraph()
-        early = 0 if os.environ.get("PA_BENCH_NO_EARLY") else pa.PA_DECODE_EARLY_CACHE_READS
-        with torch.cuda.graph(graph, stream=stream), pa.decode_options(early):
-            for c in layer_calls:
-                c.step()
-        for _ in range(3):
-            graph.replay()
-        torch.cuda.synchronize(device)
-        reps_n = max(5, min(50, args.steps // args.layers))
-        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps_n)]
-        for i in range(reps_n):
-            gev[i][0].record(stream)
-            graph.replay()
-            gev[i][1].record(stream)
-        torch.cuda.synchronize(device)
-        per_layer_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in gev) / args.layers
-        if pa.pa_device_errors() != 0:
-            raise RuntimeError("device error word set during the back-to-back replay")
+        layer_calls = replica_calls(cache, dev, max_len, wl.scale, calls.partition_size, stream,
+                                    args.layers, fused=calls.fused, fp8=calls.fp8)
+        reps = max(5, min(50, args.steps // args.layers))
+        per_layer_ms = back_to_back(layer_calls, stream, reps, early)
+        pa_device_errors_or_raise()
         b2b = {"layers": args.layers, "us_per_layer": 1e3 * per_layer_ms,
                "kv_GB_per_s": bytes_step / (per_layer_ms * 1e-3) / 1e9,
-               "how": "one CUDA graph of the step over per-layer cache replicas, no L2 flush"}
-        del graph, layer_calls, reps
+               "frac_of_peak": bytes_step / (per_layer_ms * 1e-3) / 1e9 / peak,
+               "early_cache_reads": bool(early),
+               "how": "one CUDA graph of the step over per-layer cache copies (together larger "
+                      "than L2), no flush; consecutive layers overlap through programmatic "
+                      "dependent launch"}
+        del layer_calls
         torch.cuda.empty_cache()
 
-    # ---- roofline of pa_decode (decode kernel + split-K merge kernel)
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(peaks_path):
-        peak, peak_src = float(json.load(open(peaks_path))["hbm_gbs"]), "measured"
-    else:
-        peak, peak_src = FALLBACK_HBM_GBS, "fallback"
-    if b2b is not None:
-        b2b["frac_of_peak"] = b2b["kv_GB_per_s"] / peak
-    dec_s = statistics.mean(decode_ms) * 1e-3
-    achieved = bytes_step / dec_s / 1e9
-    traffic = load_traffic(f"pa_decode_{wl.name}" + ("_fp8" if calls.fp8 else ""))
+    # ---- the other workloads, same process (one GPU, default workload only)
+    side = None
+    if world == 1 and wl.name == "llama3_8b_layer" and not args.no_side_workloads:
+        del calls
+        torch.cuda.empty_cache()
+        side = {}
+        with pa.decode_options(early):
+            for name in SIDE_WORKLOADS:
+                side[name] = measure_workload(name, args, device, stream, flush, peak,
+                                              steps=max(10, min(args.steps, 100)))
+        calls = None
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, one GPU only)
+    # ---- roofline of the headline step
+    dec_s = statistics.mean(step_ms) * 1e-3
+    achieved = bytes_step / dec_s / 1e9
+    traffic = load_traffic(f"pa_decode_{wl.name}" + ("_fp8" if wl.cache_dtype != "bf16" else ""))
+
+    # ---- host side and CPU baseline (rank 0, one GPU only)
+    host_side = host_allocator_metrics() if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        try:
-            times, cores = cpu_oracle_run(wl, args.cpu_budget_s)
-            cpu = {"value": bytes_step * len(times) / sum(times) / 1e9, "unit": "GB/s",
-                   "cores": cores, "kind": "oracle",
-                   "sample": f"{len(times)} whole decode steps of the {wl.num_seqs}-sequence "
-                             f"batch in {sum(times):.1f} s (float64 NumPy)"}
-        except ValueError as exc:
-            cpu = {"value": None, "unit": "GB/s", "cores": 0, "kind": "oracle",
-                   "sample": f"not run: {exc}"}
+        cpu = cpu_baseline_line(wl, bytes_logical, args.cpu_budget_s)
 
     value = whole_job_rate(bytes_step, args.steps, world, total_ms) / 1e9
     line = {
@@ -704,26 +989,27 @@ def run_b200(args, wl, rank, world, local_rank):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "block_size": wl.block_size, "num_blocks": wl.num_blocks,
                    "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
-                   "partition_size": calls.partition_size,
-                   "num_partitions": calls.num_partitions, "copy_on_write_pairs": cow_pairs,
+                   "kv_bytes_logical_per_step": bytes_logical,
+                   "partition_size": part_size, "num_partitions": num_partitions,
+                   "copy_on_write_pairs": cow_pairs,
                    "placement": args.placement, "kv_cache": wl.cache_dtype,
-                   "l2": f"flushed between steps ({flush_w.numel() >> 20} MiB written, then "
-                         f"{(flush_r.numel() * 4) >> 20} MiB of another buffer read; outside the "
-                         "timed events)",
-                   "parallelism": f"replicas x{world}"},
+                   "early_cache_reads": bool(early),
+                   "l2": flush.describe(), "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": whole_job_rate(tokens_step, args.steps, world, total_ms),
         "us_per_step": 1e3 * total_ms / args.steps,
-        "step_us_p10_p50_p90": [1e3 * float(np.percentile(decode_ms, p)) for p in (10, 50, 90)],
+        "step_us_p10_p50_p90": [1e3 * float(np.percentile(step_ms, p)) for p in (10, 50, 90)],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": ("pa_decode_append (fused append + decode kernel, split-K "
-                                "merge kernel)" if calls.fused else
+                                "merge kernel)" if not args.unfused else
                                 "pa_kv_append + pa_decode (decode + split-K merge kernels)"),
                      "peak_source": f"{peak_src} hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "back_to_back": b2b,
-        "gpu_launches": calls.launches_per_step * args.steps,
+        "workloads": side,
+        "host": host_side,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "wall_s_timed_region": wall,
     }
@@ -732,6 +1018,115 @@ def run_b200(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier(device_ids=[local_rank])
         dist.destroy_process_group()
+
+
+LAYOUT_METRIC = "decode attention over paged vs contiguous caches: us per call and KV-read GB/s"
+
+
+def run_layout_sweep(args, rank, world, local_rank):
+    """The cost of paging on this GPU ("What is paged attention in vLLM, and why
+    does it matter?", Trade-offs and edge cases, first point: table reads,
+    extra branches and irregular accesses made the 2023 paged kernel 20-26 %
+    slower than a kernel over contiguous caches; "Paged Attention" glossary,
+    FAQ: small blocks mean more lookups). The same tokens are decoded
+    (pa_decode, no append) from paged caches at block sizes 8..128 with a
+    random and an in-order (identity) physical placement, and from one
+    contiguous slab per sequence (pa_decode_contiguous: no table at all), on the
+    Llama-3-8B-shaped batch and on the long-context batch. Each call is timed
+    cold (L2 flushed before it); every paged output is checked bit for bit
+    against the contiguous one."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+    from workloads import configs, synth
+
+    if rank != 0:
+        return
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
+    peak, peak_src = load_peak()
+    flush = L2Flush(device)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    table = {}
+    for name, steps in (("llama3_8b_layer", min(args.steps, 200)),
+                        ("long_context", min(args.steps, 40))):
+        wl = make_workload(name, 16)
+        lens = [n + 1 for n in wl.context_lens]          # the step's attended tokens
+        S, hkv, d = wl.num_seqs, wl.num_kv_heads, wl.head_dim
+        slab_len = -(-max(lens) // 16) * 16
+        ks = torch.zeros((S, slab_len, hkv, d), dtype=torch.bfloat16, device=device)
+        vs = torch.zeros_like(ks)
+        for s, n in enumerate(lens):
+            k, v = synth.kv_rows(wl.value_seed, s, n, hkv, d)
+            ks[s, :n] = torch.from_numpy(k).to(device).to(torch.bfloat16)
+            vs[s, :n] = torch.from_numpy(v).to(device).to(torch.bfloat16)
+        q = torch.from_numpy(synth.queries(wl.value_seed, 0, S, wl.num_heads, d)).to(
+            device).to(torch.bfloat16)
+        lens_d = torch.tensor(lens, dtype=torch.int32, device=device)
+        max_len = max(lens)
+        ps = wl.partition_size or pa.pa_decode_partition_size(S, hkv, max_len)
+        ws = torch.empty(max(16, pa.pa_decode_workspace_bytes(S, wl.num_heads, hkv, d, max_len,
+                                                               ps)),
+                         dtype=torch.uint8, device=device)
+        bytes_call = sum(lens) * hkv * 2 * d * 2
+        out_c = torch.empty_like(q)
+
+        def contig():
+            pa.pa_decode_contiguous(out_c, q, ks, vs, lens_d, max_len, wl.scale, ps, ws)
+
+        ms = cold_steps(contig, flush, steps, 3, stream)
+        rows = {"contiguous": {"us_per_call": 1e3 * statistics.median(ms),
+                               "GB_per_s": bytes_call / (statistics.median(ms) * 1e-3) / 1e9}}
+        for bs in (8, 16, 32, 64, 128):
+            for placement in ("random", "identity"):
+                nb = sum(-(-n // bs) for n in lens) + 16
+                bm = pa.BlockManager(nb, bs)
+                order = synth.block_permutation(nb, wl.placement_seed + bs) \
+                    if placement == "random" else np.arange(nb, dtype=np.int32)
+                bm.allocator.set_free_order(order)
+                seqs = [bm.add_seq() for _ in lens]
+                kc = torch.empty((nb, bs, hkv, d), dtype=torch.bfloat16, device=device)
+                vc = torch.empty_like(kc)
+                for s, n in enumerate(lens):
+                    slots, _ = bm.append_slots([seqs[s]], [n])
+                    pa.pa_kv_append(ks[s, :n], vs[s, :n], torch.from_numpy(slots).to(device),
+                                    kc, vc)
+                mb = -(-max_len // bs)
+                tables, lens_bm = bm.block_tables(seqs, mb)
+                tables = torch.from_numpy(tables).to(device)
+                out_p = torch.empty_like(q)
+
+                def paged():
+                    pa.pa_decode(out_p, q, kc, vc, tables, lens_d, max_len, wl.scale, ps, ws)
+
+                ms = cold_steps(paged, flush, steps, 3, stream)
+                pa_device_errors_or_raise()
+                med = statistics.median(ms)
+                rows[f"bs{bs}_{placement}"] = {
+                    "us_per_call": 1e3 * med, "GB_per_s": bytes_call / (med * 1e-3) / 1e9,
+                    "vs_contiguous": med / (rows["contiguous"]["us_per_call"] * 1e-3),
+                    "bit_identical_to_contiguous": bool(torch.equal(out_p, out_c))}
+                del kc, vc, tables, bm
+                torch.cuda.empty_cache()
+        table[name] = {"num_seqs": S, "attended_tokens": sum(lens), "kv_bytes_per_call":
+                       bytes_call, "partition_size": ps, "slab_len": slab_len, "steps": steps,
+                       "results": rows}
+        del ks, vs, ws
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    ref = table["llama3_8b_layer"]["results"]["contiguous"]
+    print(json.dumps({
+        "metric": LAYOUT_METRIC, "value": ref["GB_per_s"], "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": 3, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "layout_sweep: llama3_8b_layer and long_context, block sizes "
+                               "8-128, random / identity placement, contiguous slabs",
+                   "l2": flush.describe()},
+        "peak": peak, "peak_source": f"{peak_src} hbm_gbs", "layouts": table, "clocks": clk,
+        "gpu_launches": None}), flush=True)
 
 
 def run_swap(args, rank, world, local_rank):
@@ -962,6 +1357,14 @@ def main():
     rank, world, local_rank = dist_env()
     if args.workload in ("prefill", "chunked_prefill"):
         run_prefill(args, rank, world, local_rank)
+        return
+    if args.workload == "layout_sweep":
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the oracle has no kernels whose memory layout could be compared"}))
+            return
+        run_layout_sweep(args, rank, world, local_rank)
         return
     if args.workload == "swap":
         if args.impl == "reference":

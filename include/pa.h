@@ -317,6 +317,31 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                          pa_stream_t stream);
 
 /*
+ * pa_decode_contiguous — the same decode attention over a contiguous cache,
+ * with no block table: the baseline that paging is measured against, not part
+ * of the paged method. "What is paged attention in vLLM, and why does it
+ * matter?", Trade-offs and edge cases, first point: the paged kernel pays for
+ * its table reads and irregular accesses with higher attention-kernel latency
+ * than a kernel over contiguous per-request caches; Steps 1-2 and
+ * "PagedAttention — AI Glossary", Example: such caches reserve one slab per
+ * request. Here every sequence owns one slab of slab_len token rows:
+ *
+ *   k, v           device, [num_seqs][slab_len][num_kv_heads][head_dim], bf16;
+ *                  token t of sequence s is row t of slab s.
+ *   context_lens   device, int32 [num_seqs]: tokens to attend, <= slab_len.
+ *   slab_len       tokens per slab, >= 16.
+ * Every other argument as pa_decode (bf16 only: dtype must be PA_BF16). The
+ * kernel is pa_decode's tensor-core kernel with the table read removed and one
+ * TMA box per 16 tokens; chunks and reduction order are the same, so on the
+ * same tokens the output equals pa_decode's bit for bit.
+ */
+int pa_decode_contiguous(void* out, const void* q, const void* k, const void* v,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int slab_len, int max_context_len,
+                         float scale, int partition_size, void* workspace,
+                         size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_prefill — causal attention of each sequence's newest chunk of query rows
  * over its paged context (prompt prefill, or chunked prefill on top of an
  * already-cached prefix). "Paged Attention" (klaylearn.com glossary),

@@ -36,6 +36,7 @@ __all__ = [
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
     "pa_set_decode_options", "PA_DECODE_EARLY_CACHE_READS", "decode_options",
+    "pa_decode_contiguous",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
@@ -70,6 +71,8 @@ _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, 
 _sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
 _sig("pa_set_decode_options", ctypes.c_uint, ctypes.c_uint)
+_sig("pa_decode_contiguous", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+     _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
 _sig("pa_decode", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _f32, _i32, _vp, _sz, _i32, _vp)
@@ -112,7 +115,7 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 EXPORTED = (
     "pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_swap_blocks",
     "pa_decode_partition_size", "pa_set_decode_options", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_decode_append",
+    "pa_decode", "pa_decode_append", "pa_decode_contiguous",
     "pa_decode_fp8", "pa_decode_append_fp8", "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
@@ -347,6 +350,30 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
             _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
             block_tables.shape[1], int(max_context_len), float(scale), int(partition_size),
             ws_ptr, ws_bytes, _dtype_code(k_cache), st))
+
+
+def pa_decode_contiguous(out, q, k, v, context_lens, max_context_len: int, scale: float,
+                         partition_size: int = 0, workspace=None, stream=None) -> None:
+    """Decode attention over a contiguous cache (no block table); see
+    pa_decode_contiguous in include/pa.h. k, v: [S, slab_len, Hkv, d] bf16."""
+    torch = _torch()
+    s, slab, hkv, d = k.shape
+    _, hq, dq = q.shape
+    if q.shape[0] != s or dq != d or out.shape != q.shape or v.shape != k.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if context_lens.shape != (s,):
+        raise ValueError("context_lens must be [S]")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    guard, st = _on_device((out, q, k, v, context_lens, workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_contiguous(
+            _dev_ptr(out, "out", k.dtype), _dev_ptr(q, "q", k.dtype), _dev_ptr(k, "k"),
+            _dev_ptr(v, "v", k.dtype), _dev_ptr(context_lens, "context_lens", torch.int32), s, hq,
+            hkv, d, slab, int(max_context_len), float(scale), int(partition_size), ws_ptr,
+            ws_bytes, _dtype_code(k), st))
 
 
 def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,

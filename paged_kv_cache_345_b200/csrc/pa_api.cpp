@@ -394,6 +394,81 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                        PA_FP8_E4M3, k_new, v_new, k_scale, v_scale, stream);
 }
 
+int pa_decode_contiguous(void* out, const void* q, const void* k, const void* v,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int slab_len, int max_context_len,
+                         float scale, int partition_size, void* workspace,
+                         size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: num_seqs < 0");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k || !v || !context_lens)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: null pointer");
+  if (dtype != PA_BF16)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: dtype %d (built: bf16)", dtype);
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa_fail(PA_ERR_INVALID,
+                   "pa_decode_contiguous: num_heads %d not a multiple of num_kv_heads %d",
+                   num_heads, num_kv_heads);
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: group size %d (built: 1, 2, 4, 8)",
+                   group);
+  if (head_dim != 64 && head_dim != 128)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: head_dim %d (built: 64, 128)",
+                   head_dim);
+  if (slab_len < 16 || slab_len > (1 << 24))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: slab_len %d outside [16, 2^24]",
+                   slab_len);
+  if (max_context_len < 0 || max_context_len > slab_len)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: max_context_len %d outside [0, %d]",
+                   max_context_len, slab_len);
+  if (!std::isfinite(scale)) return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: scale not finite");
+  if (partition_size < 0 || partition_size % pa::kChunkTokens != 0 ||
+      partition_size > pa::kMaxPartitionSize)
+    return pa_fail(PA_ERR_INVALID,
+                   "pa_decode_contiguous: partition_size %d not a multiple of %d in [0, %d]",
+                   partition_size, pa::kChunkTokens, pa::kMaxPartitionSize);
+  if (num_seqs > 65535 || num_kv_heads > 65535)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: num_seqs or num_kv_heads > 65535");
+  if (static_cast<int64_t>(num_seqs) * slab_len * num_kv_heads * head_dim * 2 / 16 >
+      (int64_t(1) << 36))
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: cache larger than 1 TiB");
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+      !aligned(context_lens, 4) || (workspace && !aligned(workspace, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: misaligned pointer");
+  pa::DecodeShape sh{};
+  sh.num_seqs = num_seqs;
+  sh.num_heads = num_heads;
+  sh.num_kv_heads = num_kv_heads;
+  sh.head_dim = head_dim;
+  sh.block_size = slab_len;   // one "block" per sequence: its slab
+  sh.num_blocks = num_seqs;
+  sh.max_blocks_per_seq = 1;
+  sh.max_context_len = max_context_len;
+  sh.partition_size = partition_size == 0
+                          ? pa_decode_partition_size(num_seqs, num_kv_heads, max_context_len)
+                          : partition_size;
+  sh.num_partitions = resolve_partitions(max_context_len, &sh.partition_size);
+  sh.scale = scale;
+  sh.dtype = dtype;
+  sh.early_reads = (g_decode_options & PA_DECODE_EARLY_CACHE_READS) != 0;
+  sh.contiguous = true;
+  if (sh.num_partitions > pa::kMaxPartitions)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: %d partitions > %d",
+                   sh.num_partitions, pa::kMaxPartitions);
+  const size_t need =
+      pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, sh.num_partitions).total;
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_contiguous: workspace %zu B < %zu B needed",
+                   workspace ? workspace_bytes : size_t(0), need);
+  cudaError_t e = pa::launch_decode(sh, out, q, k, v, nullptr, context_lens, workspace, nullptr,
+                                    nullptr, nullptr, nullptr,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_contiguous: no kernel for this shape");
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode_contiguous launch", e);
+}
+
 int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                const int32_t* block_tables, const int32_t* context_lens,
                const int32_t* query_start, int num_seqs, int total_q, int num_heads,

@@ -94,7 +94,12 @@ __host__ __device__ constexpr int box_stride_bytes(int hb, int rows_per_box, int
   return (hb * rows_per_box * rs + 127) & ~127;
 }
 
-template <int D, int G, int HB, int NS, bool FP8>
+// TABLE = false: the table-free variant over a contiguous cache
+// [num_seqs][slab_len][num_kv_heads][head_dim] (each sequence's K/V in one
+// slab, token t at row t): the same pipeline and arithmetic, but no block-table
+// read, and every chunk of 16 tokens is one box at (token t, sequence s). The
+// tensor map describes the slab as a "block" of slab_len tokens per sequence.
+template <int D, int G, int HB, int NS, bool FP8, bool TABLE = true>
 __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     pa_decode_mma_kernel(const __grid_constant__ CUtensorMap k_map,
                          const __grid_constant__ CUtensorMap v_map, const DecodeParams p) {
@@ -109,7 +114,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   const int hg = blockIdx.x, part = blockIdx.y, s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = p.partition_size, bs = p.block_size, lg = p.log2_block_size;
-  const int rows_per_box = bs < C ? bs : C;
+  const int rows_per_box = (!TABLE || bs >= C) ? C : bs;
   const int box_stride = box_stride_bytes(HB, rows_per_box, RS);
 
   if (threadIdx.x == 0) {
@@ -134,21 +139,20 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   pdl_launch_dependents();
 
   // Independent loads first so their latencies overlap: the context length,
-  // the first 32 block-table entries of this partition (producer warp) and the
-  // query fragments (consumer warps).
+  // the first 32 block-table entries of this partition (producer warp) and
+  // (without early reads) the query fragments (consumer warps).
   int L = __ldg(p.context_lens + s);
   const int t0 = part * P;
   const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
   int base = t0 >> lg, ent = 0;
-  if (warp == HB && base + lane < p.max_blocks_per_seq) ent = __ldg(trow + base + lane);
+  if (TABLE && warp == HB && base + lane < p.max_blocks_per_seq) ent = __ldg(trow + base + lane);
   const int kvh = hg * HB + (warp < HB ? warp : 0);  // this consumer warp's KV head
   const int qr = lane >> 2;  // fragment row: query head of the group (rows >= G are padding)
   const int qc = lane & 3;   // fragment column pair
   const bool real_row = qr < G;
   const int64_t out_row = static_cast<int64_t>(s) * p.num_heads + kvh * G;
   uint32_t qa[D / 16][2];  // Q as the B operand (column = head of the group), 16-bit pairs
-  if (warp < HB) {
-    if (early) pdl_wait();
+  auto load_q = [&]() {
     const uint32_t* qp = reinterpret_cast<const uint32_t*>(
         static_cast<const __nv_bfloat16*>(p.q) + (out_row + (real_row ? qr : 0)) * D);
     if constexpr (!FP8) {
@@ -173,7 +177,12 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
         }
       }
     }
-  }
+  };
+  // q may be the previous kernel's output: loaded here when everyone has
+  // waited; under early reads only after the CTA barrier below, so that the
+  // producer, which does not wait before its first loads, is never held back
+  // by consumers that do
+  if (warp < HB && !early) load_q();
 
   if (L < 0 || L > p.max_context_len ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
@@ -196,6 +205,10 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   const int t1 = min(t0 + P, L);
   const int nchunks = (t1 - t0 + C - 1) / C;
   __syncthreads();
+  if (warp < HB && early) {
+    pdl_wait();
+    load_q();
+  }
 
   if (warp == HB) {
     // ------------------------------------------------------------- producer
@@ -209,6 +222,17 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
       }
       const int t = t0 + c * C;
       const int nvalid = min(C, t1 - t);
+      if constexpr (!TABLE) {
+        // table-free: one box of 16 token rows of this sequence's slab
+        const uint32_t full_bar = smem_u32(bars + st);
+        const uint32_t kdst = smem_u32(smem + st * Cfg::kStageBytes);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(full_bar, 2u * HB * C * RS);
+          tma_load_4d(kdst, &k_map, 0, t, hg * HB, s, full_bar);
+          tma_load_4d(kdst + TB, &v_map, 0, t, hg * HB, s, full_bar);
+        }
+        continue;
+      }
       const int lb_lo = t >> lg, lb_hi = (t + nvalid - 1) >> lg;
       if (lb_hi - base >= 32) {  // refill: the next 32 table entries, one per lane
         base = lb_lo;
@@ -265,7 +289,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
 
   // byte offset of (token r of the chunk, 16-byte column c) of this warp's head
   const int head_off = warp * rows_per_box * RS;
-  const int lgb = lg < 4 ? lg : 4;  // log2(rows_per_box)
+  const int lgb = (!TABLE || lg >= 4) ? 4 : lg;  // log2(rows_per_box)
   auto at = [&](int r, int c) -> uint32_t {
     const int b = r >> lgb;
     return b * box_stride + head_off + (r - (b << lgb)) * RS + c * 16;

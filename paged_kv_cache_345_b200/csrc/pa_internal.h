@@ -27,6 +27,9 @@ struct DecodeShape {
   float scale;
   pa_dtype dtype;
   bool early_reads;  // PA_DECODE_EARLY_CACHE_READS for this call
+  // pa_decode_contiguous: a slab of block_size (= slab length) tokens per
+  // sequence, num_blocks = num_seqs, no block table
+  bool contiguous;
 };
 
 // Byte offsets of the split-K workspace regions.

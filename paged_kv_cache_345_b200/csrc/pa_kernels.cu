@@ -411,12 +411,15 @@ cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
   constexpr int kNSfit = (FP8 ? 65536 : 114688) / kStage;
   constexpr int NS = kNSfit < 2 ? 2 : (kNSfit > 4 ? 4 : kNSfit);
   using Cfg = GroupConfig<D, G, HB, NS, FP8>;
-  auto kernel = pa_decode_mma_kernel<D, G, HB, NS, FP8>;
-  static std::atomic<unsigned long long> configured{0};
-  cudaError_t e = ensure_smem(kernel, Cfg::kSmemBytes, configured);
+  auto kernel = pa_decode_mma_kernel<D, G, HB, NS, FP8, true>;
+  if constexpr (!FP8) {
+    if (sh.contiguous) kernel = pa_decode_mma_kernel<D, G, HB, NS, false, false>;
+  }
+  static std::atomic<unsigned long long> configured[2] = {{0}, {0}};
+  cudaError_t e = ensure_smem(kernel, Cfg::kSmemBytes, configured[sh.contiguous ? 1 : 0]);
   if (e != cudaSuccess) return e;
   CUtensorMap kmap, vmap;
-  const int rows = sh.block_size < Cfg::kC ? sh.block_size : Cfg::kC;
+  const int rows = (sh.contiguous || sh.block_size >= Cfg::kC) ? Cfg::kC : sh.block_size;
   if ((e = encode_group_map(&kmap, k_cache, sh, rows, HB)) != cudaSuccess) return e;
   if ((e = encode_group_map(&vmap, v_cache, sh, rows, HB)) != cudaSuccess) return e;
   dim3 grid(sh.num_kv_heads / HB, sh.num_partitions, sh.num_seqs);

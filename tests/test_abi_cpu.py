@@ -90,6 +90,42 @@ def test_decode_zero_sequences_is_a_no_op():
     assert _decode(S=0)[0] == pa.PA_OK
 
 
+def _contig(**over):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, cl=FAKE, S=2, Hq=32, Hkv=8, D=128, slab=4112,
+             maxlen=4101, scale=0.1, P=0, ws=FAKE, wsb=1 << 30, dt=pa.PA_BF16)
+    a.update(over)
+    st = pa._lib.pa_decode_contiguous(a["out"], a["q"], a["k"], a["v"], a["cl"], a["S"], a["Hq"],
+                                      a["Hkv"], a["D"], a["slab"], a["maxlen"], a["scale"],
+                                      a["P"], a["ws"], a["wsb"], a["dt"], None)
+    return st, pa._lib.pa_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dt=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),        # bf16 only
+    (dict(dt=pa.PA_FP8_E4M3), pa.PA_ERR_UNSUPPORTED),
+    (dict(Hq=24), pa.PA_ERR_UNSUPPORTED),               # group 3
+    (dict(Hq=30), pa.PA_ERR_INVALID),
+    (dict(D=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(slab=8, maxlen=8), pa.PA_ERR_INVALID),        # slabs of at least 16 tokens
+    (dict(maxlen=4113), pa.PA_ERR_INVALID),             # longer than a slab
+    (dict(maxlen=-1), pa.PA_ERR_INVALID),
+    (dict(P=24), pa.PA_ERR_INVALID),
+    (dict(scale=float("inf")), pa.PA_ERR_INVALID),
+    (dict(k=None), pa.PA_ERR_INVALID),
+    (dict(v=ctypes.c_void_p(0x10004)), pa.PA_ERR_INVALID),   # misaligned
+    (dict(ws=None, wsb=0), pa.PA_ERR_INVALID),          # split sequences need a workspace
+    (dict(S=-1), pa.PA_ERR_INVALID),
+])
+def test_contiguous_decode_rejects_on_host(over, status):
+    st, msg = _contig(**over)
+    assert st == status, msg
+    assert msg
+
+
+def test_contiguous_decode_zero_sequences_is_a_no_op():
+    assert _contig(S=0)[0] == pa.PA_OK
+
+
 def test_append_and_copy_reject_on_host():
     lib = pa._lib
     assert lib.pa_kv_append(FAKE, FAKE, FAKE, -1, FAKE, FAKE, 4, 4, 2, 64, 0, None) == \

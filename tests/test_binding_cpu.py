@@ -67,6 +67,18 @@ def test_cache_writes_and_block_copies(calls):
                                             "block_mapping", 3, 8, 2, 16, pa.PA_BF16, "stream"))
 
 
+def test_contiguous_decode_call(calls):
+    s, hq, hkv, d, slab = 3, 8, 2, 128, 64
+    k, v = z(s, slab, hkv, d), z(s, slab, hkv, d)
+    q, out, lens, ws = z(s, hq, d), z(s, hq, d), z(s, dtype=I32), z(1024, dtype=U8)
+    pa.pa_decode_contiguous(out, q, k, v, lens, 50, 0.125, 32, ws)
+    name, a = calls[-1]
+    assert name == "pa_decode_contiguous"
+    assert a[:5] == ("out", "q", "k", "v", "context_lens")
+    assert a[5:13] == (s, hq, hkv, d, slab, 50, pytest.approx(0.125), 32)
+    assert a[13:] == ("workspace", 1024, pa.PA_BF16, "stream")
+
+
 def test_decode_calls(calls):
     s, hq, hkv, d, nb, bs, mb = 3, 8, 2, 128, 10, 16, 4
     kc, vc = z(nb, bs, hkv, d), z(nb, bs, hkv, d)

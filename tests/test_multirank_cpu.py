@@ -137,3 +137,21 @@ def test_decode_step_bytes_are_the_oracles_per_token_bytes():
     tiny = configs.tiny()
     assert bench.kv_bytes(tiny) == sum(n + 1 for n in tiny.context_lens) * \
         oblk.kv_bytes_per_token(1, 2, 64, 4)
+
+
+def test_host_metrics_reproduce_the_worked_example():
+    """bench.py's host figures: the worked example's cache utilisation through
+    the native block manager is the page's 99.4 % (10,578 tokens in 10,640
+    slots), the slab figure its 16.1 %; the allocator step covers 256 sequences."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    m = bench.host_allocator_metrics(steps=4)
+    cu = m["cache_utilisation"]
+    assert (cu["tokens_before_step"], cu["slots_before_step"]) == (10_578, 10_640)
+    assert round(100 * cu["paged_before_step"], 1) == 99.4
+    assert round(100 * cu["slab"], 1) == 16.1
+    assert cu["paged_after_step"] == 10_586 / 10_656
+    a = m["allocator_step"]
+    assert a["sequences"] == 256 and a["us_per_step_p50"] > 0 and a["us_per_step_c_abi_p50"] > 0
+    assert 0.9 < a["utilisation_after"] <= 1.0
