@@ -61,6 +61,9 @@ def parse_args():
                     help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-back-to-back", action="store_true")
+    ap.add_argument("--compact-pool", action="store_true",
+                    help="a pool just large enough for the batch, no ghost sequences (a small "
+                         "case of the same step for profilers)")
     ap.add_argument("--no-side-workloads", action="store_true",
                     help="skip the large-batch, long-context and shared-prefix lines")
     ap.add_argument("--no-early-reads", action="store_true",
@@ -881,7 +884,8 @@ def run_b200(args, wl, rank, world, local_rank):
     early = 0 if args.no_early_reads else pa.PA_DECODE_EARLY_CACHE_READS
 
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device, args.placement)
-    ps = TUNED_PARTITION[wl.name.split("_bs")[0]] if args.partition_size < 0 else args.partition_size
+    ps = TUNED_PARTITION[wl.name.split("_bs")[0].replace("_compact", "")] \
+        if args.partition_size < 0 else args.partition_size
     calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused)
     launches_per_step, part_size = calls.launches_per_step, calls.partition_size
     num_partitions = calls.num_partitions
@@ -1377,6 +1381,10 @@ def main():
     wl = make_workload(args.workload, args.block_size)
     if args.kv_dtype != "bf16":
         wl = dataclasses.replace(wl, kv_dtype=args.kv_dtype)
+    if args.compact_pool:
+        need = sum(-(-(n + 2) // wl.block_size) for n in wl.context_lens) + 64
+        wl = dataclasses.replace(wl, num_blocks=need, ghost_lens=(),
+                                 name=wl.name + "_compact")
     if args.impl == "reference":
         run_reference(args, wl, rank)
         return

@@ -31,7 +31,8 @@
 //  * Stages form a ring of NS; a stage is released once all HB warps read it.
 //  * Consumer warp per chunk: S = Q K^T with m16n8k16 (A = Q rows of the
 //    group, B = K rows via ldmatrix), online softmax in base 2 on the
-//    accumulator fragments (row max / sum over the 4-lane quad), P converted to
+//    accumulator fragments (row max / sum over the 4-lane quad; the reference
+//    maximum moves only when a chunk exceeds it by 2^8), P converted to
 //    bfloat16 in registers becomes the A operand of O += P V (B = V rows via
 //    ldmatrix.trans). m, l and O stay in registers.
 //  * End: a single-partition sequence writes `out`; otherwise (m, l, O) go to
@@ -376,21 +377,32 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
       cm0 = fmaxf(cm0, __shfl_xor_sync(kFullMask, cm0, off));
       cm1 = fmaxf(cm1, __shfl_xor_sync(kFullMask, cm1, off));
     }
-    const float mn0 = fmaxf(m[0], cm0), mn1 = fmaxf(m[1], cm1);
-    const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);
-    m[0] = mn0;
-    m[1] = mn1;
-    const float p0 = exp2f(x[0] - mn0), p1 = exp2f(x[1] - mn1);
-    const float p2 = exp2f(x[2] - mn0), p3 = exp2f(x[3] - mn1);
-    l_part[0] = fmaf(l_part[0], al0, p0 + p2);
-    l_part[1] = fmaf(l_part[1], al1, p1 + p3);
+    // The reference maximum m moves only when a chunk's maximum exceeds it by
+    // more than 2^8 (logits are base 2): the exponentials stay at most 2^8, far
+    // from overflowing the fp32 sums or the 16-bit P, and O and l are rescaled
+    // on few chunks instead of every one. Numerator and denominator share m,
+    // so the softmax is the same whatever m is. The vote keeps the branch
+    // warp-uniform (lanes with the same t hold the same heads' m).
+    constexpr float kSlack = 8.0f;
+    if (__any_sync(kFullMask, cm0 > m[0] + kSlack || cm1 > m[1] + kSlack)) {
+      const float mn0 = fmaxf(m[0], cm0), mn1 = fmaxf(m[1], cm1);
+      const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);  // 0 on the first chunk
+      m[0] = mn0;
+      m[1] = mn1;
+      l_part[0] *= al0;
+      l_part[1] *= al1;
 #pragma unroll
-    for (int i = 0; i < D / 16; ++i) {
-      o[i][0] *= al0;
-      o[i][1] *= al1;
-      o[i][2] *= al0;
-      o[i][3] *= al1;
+      for (int i = 0; i < D / 16; ++i) {
+        o[i][0] *= al0;
+        o[i][1] *= al1;
+        o[i][2] *= al0;
+        o[i][3] *= al1;
+      }
     }
+    const float p0 = exp2f(x[0] - m[0]), p1 = exp2f(x[1] - m[1]);
+    const float p2 = exp2f(x[2] - m[0]), p3 = exp2f(x[3] - m[1]);
+    l_part[0] += p0 + p2;
+    l_part[1] += p1 + p3;
     if constexpr (!FP8) {
       // P^T as B: (token 2t, 2t+1 (+8), head g) = transpose of the (token g, head 2t..) pairs
       const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
