@@ -338,11 +338,12 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
 #pragma unroll
         for (int kq = 0; kq < D / 64; ++kq) kr[h][kq] = lds128(ks_u32 + at(g + 8 * h, 2 * t + kq));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 4; ++i) vr[i] = lds128(vs_u32 + at(2 * t + (i & 1) + 8 * (i >> 1), g));
+      if (nvalid < C) {  // (warp-uniform) the last chunk of a context
         // rows past the context hold stale bytes (possibly NaN codes): use zeros
-        const int r = 2 * t + (i & 1) + 8 * (i >> 1);
-        const uint4 x = lds128(vs_u32 + at(r, g));
-        vr[i] = r < nvalid ? x : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (2 * t + (i & 1) + 8 * (i >> 1) >= nvalid) vr[i] = make_uint4(0, 0, 0, 0);
       }
       // every operand byte is in registers: hand the stage back to the producer
       __syncwarp();
@@ -366,9 +367,11 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     // x[0], x[1]: token g, heads 2t, 2t+1; x[2], x[3]: token g + 8
     float x[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tok = g + (i >> 1) * 8;
-      x[i] = tok < nvalid ? (s0[i] + s1[i]) * qscale : -INFINITY;
+    for (int i = 0; i < 4; ++i) x[i] = (s0[i] + s1[i]) * qscale;
+    if (nvalid < C) {  // (warp-uniform) keys past the context take no weight
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (g + (i >> 1) * 8 >= nvalid) x[i] = -INFINITY;
     }
     // per-head (column) max over the 16 tokens: over the lane's 2 rows, then over g
     float cm0 = fmaxf(x[0], x[2]), cm1 = fmaxf(x[1], x[3]);
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     constexpr float kSlack = 8.0f;
     if (__any_sync(kFullMask, cm0 > m[0] + kSlack || cm1 > m[1] + kSlack)) {
       const float mn0 = fmaxf(m[0], cm0), mn1 = fmaxf(m[1], cm1);
-      const float al0 = exp2f(m[0] - mn0), al1 = exp2f(m[1] - mn1);  // 0 on the first chunk
+      const float al0 = exp2_fast(m[0] - mn0), al1 = exp2_fast(m[1] - mn1);  // 0 on the 1st chunk
       m[0] = mn0;
       m[1] = mn1;
       l_part[0] *= al0;
@@ -399,8 +402,8 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
         o[i][3] *= al1;
       }
     }
-    const float p0 = exp2f(x[0] - m[0]), p1 = exp2f(x[1] - m[1]);
-    const float p2 = exp2f(x[2] - m[0]), p3 = exp2f(x[3] - m[1]);
+    const float p0 = exp2_fast(x[0] - m[0]), p1 = exp2_fast(x[1] - m[1]);
+    const float p2 = exp2_fast(x[2] - m[0]), p3 = exp2_fast(x[3] - m[1]);
     l_part[0] += p0 + p2;
     l_part[1] += p1 + p3;
     if constexpr (!FP8) {

@@ -180,6 +180,15 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 2^x on the MUFU unit (ex2.approx: relative error ~2^-22, results below
+// 2^-126 flush to 0, -inf gives 0): the softmax weights of the decode kernel,
+// which are rounded to 16 bits before they are used.
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Two floats to a float16 pair (round to nearest even); `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;

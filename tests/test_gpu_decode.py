@@ -250,3 +250,19 @@ def test_fused_step_equals_append_then_decode(bs, dtype):
     assert torch.equal(a.cache.v_cache, b.cache.v_cache)
     gh.assert_close(gh.gpu_out(a), gh.expected_all(a), dtype, f"fused bs={bs}")
     assert pa.pa_device_errors() == 0
+
+
+def test_a_thousand_short_sequences():
+    """1,100 and 1,000 short sequences (empty and exact-multiple lengths
+    included) at partitions of 16 tokens: a wide grid of mostly single-chunk
+    CTAs, against the oracle."""
+    rng = np.random.default_rng(77)
+    lens = [int(x) for x in rng.integers(0, 60, size=1100)]
+    lens[:4] = [0, 15, 47, 48]
+    wl = _custom(8, 2, 128, "bf16", 16, lens, seed=11)
+    case = gh.build_case(wl, partition_size=16)
+    gh.assert_close(gh.gpu_out(case), gh.expected_all(case), "bf16", "S=1100")
+    small = _custom(8, 2, 128, "bf16", 16, lens[:1000], seed=11)
+    case2 = gh.build_case(small, partition_size=16)
+    gh.assert_close(gh.gpu_out(case2), gh.expected_all(case2), "bf16", "S=1000")
+    assert pa.pa_device_errors() == 0
