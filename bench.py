@@ -236,9 +236,12 @@ class StepCalls:
     """The C-ABI calls of one decode step with their arguments marshalled once.
 
     fused: the step is one pa_decode_append call (append each newest token, then
-    attend); otherwise pa_kv_append followed by pa_decode (same result)."""
+    attend); otherwise pa_kv_append followed by pa_decode (same result).
+    prefix_len > 0: the step is one pa_decode_shared_prefix call with the append
+    (every sequence's first prefix_len tokens in the same blocks)."""
 
-    def __init__(self, cache, dev, max_len, scale, partition_size, stream, fused=True):
+    def __init__(self, cache, dev, max_len, scale, partition_size, stream, fused=True,
+                 prefix_len=0):
         import torch
 
         import paged_kv_cache_345_b200 as pa
@@ -288,6 +291,22 @@ class StepCalls:
             self.fns = (self.lib.pa_kv_append, self.lib.pa_decode, self.lib.pa_decode_append)
         self.fused = fused
         self.launches_per_step = (1 if fused else 2) + (1 if self.num_partitions > 1 else 0)
+        self.prefix_len = prefix_len
+        if prefix_len:
+            # the cascade step: shared prefix on the tensor cores, each sequence's
+            # own tokens (with the append) by the decode kernel, then the merge
+            if self.fp8 or dt != pa.PA_BF16:
+                raise ValueError("the shared-prefix step runs on a bf16 cache")
+            need = pa.pa_decode_shared_prefix_workspace_bytes(s, hq, hkv, d, prefix_len, max_len,
+                                                              partition_size)
+            self.prefix_workspace = torch.empty(need, dtype=torch.uint8, device=dev["q"].device)
+            self.step_args = (p(self.out), p(dev["q"]), p(dev["k_new"]), p(dev["v_new"]),
+                              p(cache.k_cache), p(cache.v_cache), p(dev["tables"]),
+                              p(dev["lens"]), s, hq, hkv, d, bs, nb, mbps, prefix_len, max_len,
+                              scale, partition_size, p(self.prefix_workspace), need, dt, st)
+            self.fns = (self.fns[0], self.fns[1], self.lib.pa_decode_shared_prefix)
+            self.fused = True
+            self.launches_per_step = 3
 
     def _call(self, fn, args):
         st = fn(*args)
@@ -740,6 +759,24 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
         res["kv_bytes_logical"] = logical
         res["GB_per_s_logical"] = logical / mean_s / 1e9
         res["copy_on_write_pairs"] = cow_pairs
+    if wl2.shared_prefix:
+        # the same step through the cascade entry point: the shared blocks read
+        # once for the whole batch
+        prefix = (wl2.shared_prefix // wl2.block_size) * wl2.block_size
+        cascade = StepCalls(cache, dev, max_len, wl2.scale, 0, stream, prefix_len=prefix)
+        clocks = ClockSampler(device.index or 0)
+        clocks.start()
+        cms = cold_steps(cascade.step, flush, steps, warmup, stream)
+        cclk = clocks.stop()
+        cmean = statistics.mean(cms) * 1e-3
+        res["shared_prefix_step"] = {
+            "entry": "pa_decode_shared_prefix", "prefix_len": prefix,
+            "us_per_step": 1e3 * statistics.mean(cms),
+            "step_us_p10_p50_p90": [1e3 * float(np.percentile(cms, p)) for p in (10, 50, 90)],
+            "GB_per_s": unique / cmean / 1e9, "frac": unique / cmean / 1e9 / peak,
+            "attended_tokens_per_s": sum(n + 1 for n in wl2.context_lens) / cmean,
+            "launches_per_step": cascade.launches_per_step, "clocks": cclk}
+        del cascade
     pa_device_errors_or_raise()
     del calls, cache, dev, host
     torch.cuda.empty_cache()

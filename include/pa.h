@@ -317,6 +317,48 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                          pa_stream_t stream);
 
 /*
+ * pa_decode_shared_prefix — decode attention (optionally with the step's
+ * append, as pa_decode_append) for a batch whose sequences all begin with the
+ * same prefix_len tokens held in the same physical blocks: block_tables[s][0
+ * .. prefix_len / block_size) are equal for every s (sequences forked from a
+ * common parent, parallel sampling). "PagedAttention — AI Glossary", How it
+ * works, step 4: sharers point at the same blocks; "What is paged attention in
+ * vLLM...", Trade-offs and edge cases: prefix sharing. The result is the same
+ * softmax attention over each sequence's whole context; only the work is
+ * split:
+ *   - the prefix: every sequence's query rows of a KV head against the shared
+ *     keys at once, on the tcgen05 tensor cores (a dense contraction of
+ *     num_seqs * group rows), each prefix block read once per call instead of
+ *     once per sequence;
+ *   - each sequence's own tokens [prefix_len, context_lens[s]) with the decode
+ *     kernel (appending each newest token there when k_new / v_new are given);
+ *   - the partial results of both combined per row with a log-sum-exp rescale.
+ *
+ *   k_new, v_new   NULL (attend only) or each sequence's newest K/V row
+ *                  [num_seqs][num_kv_heads][head_dim], written at position
+ *                  context_lens[s] - 1, which must lie past the prefix.
+ *   prefix_len     tokens shared by every sequence, a positive multiple of
+ *                  block_size, <= every context_lens[s].
+ *   workspace      at least pa_decode_shared_prefix_workspace_bytes(...) bytes;
+ *                  contents on entry ignored.
+ * Every other argument as pa_decode_append / pa_decode. Supported: bf16,
+ * head_dim 128, num_heads / num_kv_heads in {1, 2, 4, 8}, block_size a power
+ * of two in [8, 256], scale > 0. A context shorter than prefix_len sets
+ * PA_DEVERR_CONTEXT. Within the bf16 tolerance of pa_decode on the same
+ * tokens (the order of the sums differs), not bit-identical.
+ */
+size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                               int head_dim, int prefix_len, int max_context_len,
+                                               int partition_size);
+int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            int max_blocks_per_seq, int prefix_len, int max_context_len,
+                            float scale, int partition_size, void* workspace,
+                            size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_decode_contiguous — the same decode attention over a contiguous cache,
  * with no block table: the baseline that paging is measured against, not part
  * of the paged method. "What is paged attention in vLLM, and why does it

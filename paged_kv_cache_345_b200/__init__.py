@@ -36,7 +36,7 @@ __all__ = [
     "pa_decode_workspace_bytes",
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
     "pa_set_decode_options", "PA_DECODE_EARLY_CACHE_READS", "decode_options",
-    "pa_decode_contiguous",
+    "pa_decode_contiguous", "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
@@ -71,6 +71,9 @@ _sig("pa_copy_blocks", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, 
 _sig("pa_swap_blocks", _i32, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _vp)
 _sig("pa_decode_partition_size", _i32, _i32, _i32, _i32)
 _sig("pa_set_decode_options", ctypes.c_uint, ctypes.c_uint)
+_sig("pa_decode_shared_prefix_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
+_sig("pa_decode_shared_prefix", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_decode_contiguous", _i32, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
      _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_decode_workspace_bytes", _sz, _i32, _i32, _i32, _i32, _i32, _i32)
@@ -115,7 +118,8 @@ _sig("pa_bm_block_tables", _i32, _vp, _i32p, _i32, _i32p, _i32, _i32p)
 EXPORTED = (
     "pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_swap_blocks",
     "pa_decode_partition_size", "pa_set_decode_options", "pa_decode_workspace_bytes",
-    "pa_decode", "pa_decode_append", "pa_decode_contiguous",
+    "pa_decode", "pa_decode_append", "pa_decode_contiguous", "pa_decode_shared_prefix",
+    "pa_decode_shared_prefix_workspace_bytes",
     "pa_decode_fp8", "pa_decode_append_fp8", "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
@@ -350,6 +354,48 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
             _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
             block_tables.shape[1], int(max_context_len), float(scale), int(partition_size),
             ws_ptr, ws_bytes, _dtype_code(k_cache), st))
+
+
+def pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                            prefix_len, max_context_len,
+                                            partition_size=0) -> int:
+    return int(_lib.pa_decode_shared_prefix_workspace_bytes(
+        num_seqs, num_heads, num_kv_heads, head_dim, prefix_len, max_context_len, partition_size))
+
+
+def pa_decode_shared_prefix(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                            prefix_len: int, max_context_len: int, scale: float,
+                            partition_size: int = 0, workspace=None, stream=None) -> None:
+    """Decode (with the step's append when k_new / v_new are given) for sequences
+    that all begin with the same prefix_len tokens in the same blocks; see
+    pa_decode_shared_prefix in include/pa.h."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    s, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None and (k_new.shape != (s, hkv, d) or v_new.shape != k_new.shape):
+        raise ValueError("k_new/v_new must be [S, num_kv_heads, head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    if workspace is None:
+        raise ValueError("pa_decode_shared_prefix needs a workspace")
+    dt = k_cache.dtype
+    guard, st = _on_device((out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens,
+                            workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_shared_prefix(
+            _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt),
+            None if k_new is None else _dev_ptr(k_new, "k_new", dt),
+            None if v_new is None else _dev_ptr(v_new, "v_new", dt),
+            _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache", dt),
+            _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(context_lens, "context_lens", torch.int32), s, hq, hkv, d, bs, nb,
+            block_tables.shape[1], int(prefix_len), int(max_context_len), float(scale),
+            int(partition_size), _dev_ptr(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _dtype_code(k_cache), st))
 
 
 def pa_decode_contiguous(out, q, k, v, context_lens, max_context_len: int, scale: float,

@@ -394,6 +394,104 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                        PA_FP8_E4M3, k_new, v_new, k_scale, v_scale, stream);
 }
 
+// Sizes of a shared-prefix call: suffix partition size, suffix partitions,
+// prefix partition size (keys) and prefix partitions.
+namespace {
+struct PrefixPlan {
+  int suffix_part, suffix_parts, prefix_part, prefix_parts;
+};
+PrefixPlan plan_shared_prefix(int num_seqs, int num_heads, int num_kv_heads, int prefix_len,
+                              int max_context_len, int partition_size) {
+  PrefixPlan pl{};
+  const int rest = max_context_len - prefix_len;
+  pl.suffix_part = partition_size == 0
+                       ? pa_decode_partition_size(num_seqs, num_kv_heads, rest > 0 ? rest : 0)
+                       : partition_size;
+  pl.suffix_parts = rest <= 0 ? 1 : (rest + pl.suffix_part - 1) / pl.suffix_part;
+  pl.prefix_part = pa::prefix_partition_keys(num_seqs, num_heads, num_kv_heads, prefix_len);
+  pl.prefix_parts = (prefix_len + pl.prefix_part - 1) / pl.prefix_part;
+  return pl;
+}
+}  // namespace
+
+size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int num_kv_heads,
+                                               int head_dim, int prefix_len, int max_context_len,
+                                               int partition_size) {
+  if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || prefix_len <= 0 ||
+      max_context_len < prefix_len || partition_size < 0 || num_heads % num_kv_heads != 0)
+    return 0;
+  const PrefixPlan pl = plan_shared_prefix(num_seqs, num_heads, num_kv_heads, prefix_len,
+                                           max_context_len, partition_size);
+  return pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim,
+                              pl.prefix_parts + pl.suffix_parts)
+      .total;
+}
+
+int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int num_seqs, int num_heads,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            int max_blocks_per_seq, int prefix_len, int max_context_len,
+                            float scale, int partition_size, void* workspace,
+                            size_t workspace_bytes, pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  pa::DecodeShape sh;
+  int st = pa::check_decode_args(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                                 num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                 max_blocks_per_seq, max_context_len, scale, partition_size,
+                                 workspace, dtype, nullptr, nullptr, &sh);
+  if (st != PA_OK) return st;
+  if (dtype != PA_BF16 || head_dim != 128)
+    return pa_fail(PA_ERR_UNSUPPORTED,
+                   "pa_decode_shared_prefix: dtype %d, head_dim %d (built: bf16, 128)", dtype,
+                   head_dim);
+  if (block_size < 8)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix: block_size %d (built: 8..256)",
+                   block_size);
+  if (!std::isfinite(scale) || scale <= 0.0f)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_shared_prefix: scale must be finite and > 0");
+  if (prefix_len <= 0 || prefix_len % block_size != 0 || prefix_len > max_context_len)
+    return pa_fail(PA_ERR_INVALID,
+                   "pa_decode_shared_prefix: prefix_len %d not a positive multiple of block_size "
+                   "%d within max_context_len %d",
+                   prefix_len, block_size, max_context_len);
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_shared_prefix: k_new and v_new go together");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_shared_prefix: misaligned k_new or v_new");
+  const PrefixPlan pl = plan_shared_prefix(num_seqs, num_heads, num_kv_heads, prefix_len,
+                                           max_context_len, partition_size);
+  sh.partition_size = pl.suffix_part;
+  sh.prefix_slots = pl.prefix_parts;
+  sh.num_partitions = pl.prefix_parts + pl.suffix_parts;
+  sh.first_token = prefix_len;
+  if (sh.num_partitions > pa::kMaxPartitions)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix: %d partitions > %d",
+                   sh.num_partitions, pa::kMaxPartitions);
+  const pa::WorkspaceLayout wl =
+      pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, sh.num_partitions);
+  if (!workspace || workspace_bytes < wl.total)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_shared_prefix: workspace %zu B < %zu B needed",
+                   workspace ? workspace_bytes : size_t(0), wl.total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  // 1: every sequence's query against the shared prefix, once per KV head
+  cudaError_t e = pa::launch_prefix_attention(
+      num_seqs, num_heads, num_kv_heads, block_size, num_blocks, max_blocks_per_seq, prefix_len,
+      pl.prefix_part, scale, q, k_cache, v_cache, block_tables,
+      reinterpret_cast<float*>(ws + wl.m_off), reinterpret_cast<float*>(ws + wl.l_off),
+      reinterpret_cast<float*>(ws + wl.acc_off), sh.num_partitions, cs);
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix: no prefix kernel for this shape");
+  if (e != cudaSuccess) return cuda_fail("pa_decode_shared_prefix prefix launch", e);
+  // 2, 3: each sequence's own tokens (appending its newest first), then the merge
+  e = pa::launch_decode(sh, out, q, k_cache, v_cache, block_tables, context_lens, workspace,
+                        k_new, v_new, nullptr, nullptr, cs);
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_shared_prefix: no kernel for this shape");
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode_shared_prefix launch", e);
+}
+
 int pa_decode_contiguous(void* out, const void* q, const void* k, const void* v,
                          const int32_t* context_lens, int num_seqs, int num_heads,
                          int num_kv_heads, int head_dim, int slab_len, int max_context_len,

@@ -65,6 +65,13 @@ struct DecodeParams {
   // running when this call starts writes the cache, the block tables or the
   // context lengths, so they may be read before the dependent-launch wait.
   int early_reads;
+  // Shared-prefix decode (pa_decode_shared_prefix): this kernel attends only
+  // tokens [first_token, context_lens[s]) (first_token a multiple of the block
+  // size; the table is read from block first_token / block_size on), and
+  // leaves every row to the merge: its partition p goes to workspace slot
+  // prefix_slots + p, slots 0 .. prefix_slots - 1 holding the prefix's
+  // partial results. Both 0 for the other calls.
+  int first_token, prefix_slots;
 };
 
 
@@ -457,10 +464,12 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
   // writes it), and neither kernel writes it.
   const int L = __ldg(p.context_lens + s);
   if (L < 0 || L > p.max_context_len ||
-      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size)
-    return;  // flagged and zero-filled by the decode kernel
-  const int np = (L + p.partition_size - 1) / p.partition_size;
-  if (np <= 1) return;  // written directly by the decode kernel
+      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size ||
+      L < p.first_token)
+    return;  // flagged (and, without a prefix, zero-filled) by the decode kernel
+  // partial results: the prefix's slots, then this row's own partitions
+  const int np = p.prefix_slots + (L - p.first_token + p.partition_size - 1) / p.partition_size;
+  if (np <= 1 && p.prefix_slots == 0) return;  // written directly by the decode kernel
   // The next kernel may start its launch now: whatever it reads before its
   // own wait is, by the same contract, not written here.
   pdl_launch_dependents();

@@ -144,9 +144,12 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   // (without early reads) the query fragments (consumer warps).
   int L = __ldg(p.context_lens + s);
   const int t0 = part * P;
-  const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
+  // (shared-prefix decode: the table from the first block after the prefix)
+  const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq +
+                        (p.first_token >> lg);
   int base = t0 >> lg, ent = 0;
-  if (TABLE && warp == HB && base + lane < p.max_blocks_per_seq) ent = __ldg(trow + base + lane);
+  if (TABLE && warp == HB && base + lane < p.max_blocks_per_seq - (p.first_token >> lg))
+    ent = __ldg(trow + base + lane);
   const int kvh = hg * HB + (warp < HB ? warp : 0);  // this consumer warp's KV head
   const int qr = lane >> 2;  // fragment row: query head of the group (rows >= G are padding)
   const int qc = lane & 3;   // fragment column pair
@@ -186,14 +189,25 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   if (warp < HB && !early) load_q();
 
   if (L < 0 || L > p.max_context_len ||
-      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs) {
+      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs ||
+      L < p.first_token) {
     if (threadIdx.x == 0 && hg == 0 && part == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
-    L = 0;
+    L = p.first_token;
   }
+  L -= p.first_token;  // the tokens this kernel attends (all of them without a prefix)
   const int n_part_s = (L + P - 1) / P;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  const bool to_merge = p.prefix_slots > 0;  // every row is left to the merge
 
   if (L == 0) {  // empty context: zeros for every query head of the group
+    if (to_merge) {  // the prefix's partial results are the whole row
+      // (a newest token to append would lie inside the shared prefix)
+      if (p.k_new != nullptr && threadIdx.x == 0 && hg == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+      // the merge waits for this grid only: this grid must not end before the
+      // prefix kernel ahead of it, even when no CTA of it has tokens to attend
+      if (early) pdl_wait();
+      return;
+    }
     if (early) pdl_wait();
     if (part == 0) {
       const int64_t first = static_cast<int64_t>(s) * p.num_heads + hg * HB * G;
@@ -454,7 +468,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   if constexpr (FP8) {
     // lane (g, t) holds head_dim 16g .. 16g+15 of heads 2t and 2t+1:
     // o[dt][0] / o[dt][1] at 16g + 2dt, o[dt][2] / o[dt][3] at 16g + 2dt + 1
-    if (n_part_s == 1) {
+    if (n_part_s == 1 && !to_merge) {
       const float i0 = l0 > 0.0f ? vscale / l0 : 0.0f, i1 = l1 > 0.0f ? vscale / l1 : 0.0f;
       uint32_t w0[8], w1[8];
 #pragma unroll
@@ -474,7 +488,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
       }
       return;
     }
-    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + part;
+    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + p.prefix_slots + part;
     const int64_t w1 = w0 + p.num_partitions;
     float4* a0 = reinterpret_cast<float4*>(p.ws_acc + w0 * D + 16 * g);
     float4* a1 = reinterpret_cast<float4*>(p.ws_acc + w1 * D + 16 * g);
@@ -500,7 +514,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     return;
   }
 
-  if (n_part_s == 1) {
+  if (n_part_s == 1 && !to_merge) {
     const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
     __nv_bfloat16* o0 = out + (out_row + 2 * t) * D + g;
     __nv_bfloat16* o1 = o0 + D;
@@ -520,7 +534,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
 
   // split-K: this partition's (m, l, O) to the workspace
   {
-    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + part;
+    const int64_t w0 = (out_row + 2 * t) * p.num_partitions + p.prefix_slots + part;
     const int64_t w1 = w0 + p.num_partitions;
     float* a0 = p.ws_acc + w0 * D + g;
     float* a1 = p.ws_acc + w1 * D + g;

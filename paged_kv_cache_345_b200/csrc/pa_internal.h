@@ -30,6 +30,10 @@ struct DecodeShape {
   // pa_decode_contiguous: a slab of block_size (= slab length) tokens per
   // sequence, num_blocks = num_seqs, no block table
   bool contiguous;
+  // pa_decode_shared_prefix's suffix pass: attend tokens from first_token on;
+  // num_partitions counts the prefix_slots workspace slots before this
+  // call's own partitions, and every row goes through the merge
+  int first_token, prefix_slots;
 };
 
 // Byte offsets of the split-K workspace regions.
@@ -84,6 +88,19 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
                            const void* v_cache, const int32_t* block_tables,
                            const int32_t* context_lens, const int32_t* query_start,
                            cudaStream_t stream);
+// Shared-prefix decode, prefix pass (pa_prefill.cu): the num_seqs decode
+// queries q [num_seqs][num_heads][128] (bf16) attend keys [0, prefix_len) read
+// through the first row of block_tables, on the tcgen05 tensor cores, in
+// partitions of prefix_part keys (a multiple of 64); partition k of row r is
+// written to the decode workspace as slot k (ws_slots slots per row).
+int prefix_partition_keys(int num_seqs, int num_heads, int num_kv_heads, int prefix_len);
+cudaError_t launch_prefix_attention(int num_seqs, int num_heads, int num_kv_heads, int block_size,
+                                    int num_blocks, int max_blocks_per_seq, int prefix_len,
+                                    int prefix_part, float scale, const void* q,
+                                    const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, float* ws_m, float* ws_l,
+                                    float* ws_acc, int ws_slots, cudaStream_t stream);
+
 // Device error word of the current device (address in device memory).
 cudaError_t device_error_word(unsigned int** ptr);
 

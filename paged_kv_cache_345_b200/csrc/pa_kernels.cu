@@ -348,7 +348,7 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<unsigned long long
 
 template <typename T, int D>
 cudaError_t launch_merge(const DecodeShape& sh, const DecodeParams& p, cudaStream_t stream) {
-  if (sh.num_partitions <= 1) return cudaSuccess;
+  if (sh.num_partitions <= 1 && sh.prefix_slots == 0) return cudaSuccess;
   const unsigned rows = static_cast<unsigned>(sh.num_seqs) * sh.num_heads;
   return launch_pdl(pa_merge_kernel<T, D>, dim3(rows), dim3(128), 0, stream, p);
 }
@@ -422,7 +422,8 @@ cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
   const int rows = (sh.contiguous || sh.block_size >= Cfg::kC) ? Cfg::kC : sh.block_size;
   if ((e = encode_group_map(&kmap, k_cache, sh, rows, HB)) != cudaSuccess) return e;
   if ((e = encode_group_map(&vmap, v_cache, sh, rows, HB)) != cudaSuccess) return e;
-  dim3 grid(sh.num_kv_heads / HB, sh.num_partitions, sh.num_seqs);
+  // (a shared-prefix call's own partitions follow the prefix's slots)
+  dim3 grid(sh.num_kv_heads / HB, sh.num_partitions - sh.prefix_slots, sh.num_seqs);
   e = launch_pdl(kernel, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, kmap, vmap, p);
   if (e != cudaSuccess) return e;
   return launch_merge<__nv_bfloat16, D>(sh, p, stream);
@@ -514,6 +515,8 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   p.num_partitions = sh.num_partitions;
   p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
   p.early_reads = sh.early_reads ? 1 : 0;
+  p.first_token = sh.first_token;
+  p.prefix_slots = sh.prefix_slots;
   switch (sh.head_dim) {
     case 64: return dispatch_group<64>(sh, p, k_cache, v_cache, stream);
     case 128: return dispatch_group<128>(sh, p, k_cache, v_cache, stream);

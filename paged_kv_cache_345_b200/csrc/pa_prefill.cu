@@ -65,6 +65,17 @@ struct PrefillParams {
   int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks, max_blocks_per_seq;
   int num_seqs, total_q, max_query_len;
   float q_scale;  // scale * log2(e)
+  // Shared-prefix mode (PREFIX kernels, pa_decode_shared_prefix): the
+  // total_q decode queries ([total_q][Hq][128], one "token" per sequence)
+  // attend keys [0, prefix_keys) through the first table row (every sequence
+  // shares those blocks), split into prefix_parts partitions of prefix_part
+  // keys (a multiple of 64), no causal mask; each CTA writes fp32 partial
+  // results (reference maximum m, sum l, unnormalised O) of its rows to the
+  // decode split-K workspace at slot = its partition (ws_slots per row).
+  int prefix_keys, prefix_part, prefix_parts, ws_slots;
+  float* ws_m;
+  float* ws_l;
+  float* ws_acc;
 };
 
 template <int G>
@@ -194,7 +205,7 @@ __device__ __forceinline__ bool work_item(const PrefillParams& p, int S, int j, 
   return false;
 }
 
-template <int G>
+template <int G, bool PREFIX = false>
 __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     pa_prefill_kernel(const __grid_constant__ CUtensorMap q_map,
                       const __grid_constant__ CUtensorMap k_map,
@@ -227,40 +238,57 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
 
   constexpr int CTOK = Cfg::kQT * TOK;  // tokens per CTA
   const int S = p.num_seqs;
-  int s, z;
-  if (S <= kOrderMaxSeqs) {
-    bool bad = false, found;
-    if (S <= 32) found = work_item<1, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
-    else if (S <= 64) found = work_item<2, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
-    else if (S <= 128) found = work_item<4, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
-    else found = work_item<8, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
-    // a sequence with unusable arguments (among them n above the host bound,
-    // whose rows would lie outside the grid) gets no items: flagged once
-    if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
-    if (!found) return;
+  // this CTA's query rows (tokens tq0 .. of the chunk [q0, q0 + n)) and keys
+  // [key_lo, L), of which the last visible to any row is pos_last
+  int s = 0, z = 0, q0 = 0, n = 0, L = 0, tq0 = 0, pos_last = 0, nt = 0, key_lo = 0, kpart = 0;
+  const int32_t* trow = p.block_tables;
+  if constexpr (PREFIX) {
+    // grid: KV head fastest, then the key partition, then the pair of query tiles
+    kpart = jw % p.prefix_parts;
+    z = jw / p.prefix_parts;
+    n = p.total_q;
+    tq0 = z * CTOK;
+    key_lo = kpart * p.prefix_part;
+    L = min(key_lo + p.prefix_part, p.prefix_keys);
+    if (tq0 >= n || key_lo >= L) return;
+    pos_last = L - 1;
+    nt = (L - key_lo + KEYN - 1) / KEYN;
   } else {
-    s = jw % S;
-    z = jw / S;
+    if (S <= kOrderMaxSeqs) {
+      bool bad = false, found;
+      if (S <= 32) found = work_item<1, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+      else if (S <= 64) found = work_item<2, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+      else if (S <= 128) found = work_item<4, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+      else found = work_item<8, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
+      // a sequence with unusable arguments (among them n above the host bound,
+      // whose rows would lie outside the grid) gets no items: flagged once
+      if (bad && blockIdx.x == 0 && threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+      if (!found) return;
+    } else {
+      s = jw % S;
+      z = jw / S;
+    }
+    q0 = __ldg(p.query_start + s);
+    const int q1 = __ldg(p.query_start + s + 1);
+    L = __ldg(p.context_lens + s);
+    n = q1 - q0;
+    if (!prefill_order::chunk_ok(q0, q1, L, p.total_q, p.max_query_len,
+                                 static_cast<int64_t>(p.max_blocks_per_seq) * bs)) {
+      if (threadIdx.x == 0 && h == 0 && z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
+      return;
+    }
+    const int npairs = prefill_order::num_items(n, CTOK);
+    if (z >= npairs) return;  // no rows of this sequence here
+    tq0 = (npairs - 1 - z) * CTOK;
+    const int ntok_all = min(CTOK, n - tq0);
+    pos_last = L - n + tq0 + ntok_all - 1;  // <= L - 1
+    nt = pos_last / KEYN + 1;               // key tiles to visit
+    trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
   }
-  const int q0 = __ldg(p.query_start + s), q1 = __ldg(p.query_start + s + 1);
-  const int L = __ldg(p.context_lens + s);
-  const int n = q1 - q0;
-  if (!prefill_order::chunk_ok(q0, q1, L, p.total_q, p.max_query_len,
-                               static_cast<int64_t>(p.max_blocks_per_seq) * bs)) {
-    if (threadIdx.x == 0 && h == 0 && z == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
-    return;
-  }
-  const int npairs = prefill_order::num_items(n, CTOK);
-  if (z >= npairs) return;  // no rows of this sequence here
-  const int tq0 = (npairs - 1 - z) * CTOK;
-  const int ntok_all = min(CTOK, n - tq0);
-  const int pos_last = L - n + tq0 + ntok_all - 1;  // <= L - 1
-  const int nt = pos_last / KEYN + 1;                // key tiles to visit
   if (smem_u32(sm) & 1023) {                         // the swizzled operand layout needs this
     if (threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
     return;
   }
-  const int32_t* trow = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kQFull), 1);
@@ -303,7 +331,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
         if (lane == 0) ok = mbar_wait(bar(kKVEmpty + st), (u - 1) & 1, p.err);
         if (!__shfl_sync(kFullMask, ok, 0)) break;
       }
-      const int key0 = j * KEYN;
+      const int key0 = key_lo + j * KEYN;
       const int nkeys = min(KEYN, L - key0);
       const int nbox = (nkeys + rows - 1) / rows;  // boxes holding this tile's keys (<= 8)
       int blk = 0;
@@ -388,8 +416,10 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     const int tok = r / G, g = r - (r / G) * G;
     const int tx0 = tq0 + x * TOK;                  // first token of this query tile
     const int ntok = max(0, min(TOK, n - tx0));     // valid tokens of this query tile
-    const int pos0 = min(L - n + tx0, pos_last);    // position of its first token
-    const int prow = tok < ntok ? pos0 + tok : pos_last;  // last visible key of this row
+    // position of its first token, and the last key visible to this row (every
+    // row sees the whole key range in the shared-prefix mode)
+    const int pos0 = PREFIX ? pos_last : min(L - n + tx0, pos_last);
+    const int prow = PREFIX ? pos_last : (tok < ntok ? pos0 + tok : pos_last);
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float qs = p.q_scale;
     float m_use = -INFINITY, l_run = 0.0f;
@@ -407,13 +437,14 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       // the row maximum of the raw scores (scale > 0), masking only tiles that
       // reach past some row's position
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (j * KEYN + KEYN - 1 <= pos0) {
+      const int key0 = key_lo + j * KEYN;
+      if (key0 + KEYN - 1 <= pos0) {
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(sv[c][i]));
       } else {
-        const int lim = prow - j * KEYN;  // keys 0 .. lim of this tile are visible
+        const int lim = prow - key0;  // keys 0 .. lim of this tile are visible
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -477,7 +508,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
         // keys past the context in the last tile: stale or unwritten V rows become
         // zeros (their P is 0, but 0 * NaN would not be); both P V of the tile
         // are issued after this warpgroup's P is published
-        const int nkeys = L - j * KEYN;
+        const int nkeys = L - key0;
         if (nkeys < KEYN) {
           const uint32_t vb = v_s(j % NS);
           for (int i = r; i < (KEYN - nkeys) * 16; i += 128) {
@@ -494,7 +525,29 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       tc::fence_before_sync();
       mbar_arrive(bar(kPFull + 2 * x + (j & 1)));
     }
-    if (ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
+    if (PREFIX && ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
+      // the row's partial result over this key partition, for the decode merge
+      tc::fence_after_sync();
+      const int64_t row =
+          (static_cast<int64_t>(tx0 + tok) * p.num_heads + h * G + g) * p.ws_slots + kpart;
+      if (tok < ntok) {
+        p.ws_m[row] = m_use;
+        p.ws_l[row] = l_run;
+      }
+      float* dst = p.ws_acc + row * Cfg::kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tc::ld32(t_o(x) + lane_off + c * 32, ov);
+        tc::wait_ld();
+        if (tok < ntok) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            *reinterpret_cast<uint4*>(dst + c * 32 + v * 4) =
+                make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+        }
+      }
+    } else if (!PREFIX && ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
       __nv_bfloat16* dst = p.out + ((static_cast<int64_t>(q0) + tx0 + tok) * p.num_heads +
@@ -560,9 +613,9 @@ cudaError_t encode_kv_map(CUtensorMap* map, const void* base, int num_blocks, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int G>
-cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, const void* q,
-                             const void* k_cache, const void* v_cache, cudaStream_t stream) {
+template <int G, bool PREFIX>
+cudaError_t launch_prefill_g(const PrefillParams& p, const void* q, const void* k_cache,
+                             const void* v_cache, int64_t ctas, cudaStream_t stream) {
   using Cfg = PrefillConfig<G>;
   static std::atomic<unsigned long long> configured{0};
   int dev = 0;
@@ -570,32 +623,27 @@ cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, con
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev % 64);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(pa_prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::kSmemBytes);
+    e = cudaFuncSetAttribute(pa_prefill_kernel<G, PREFIX>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     // all of the unified L1 / shared storage as shared memory (a per-kernel
     // preference, not a device setting)
-    e = cudaFuncSetAttribute(pa_prefill_kernel<G>,
+    e = cudaFuncSetAttribute(pa_prefill_kernel<G, PREFIX>,
                              cudaFuncAttributePreferredSharedMemoryCarveout,
                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   CUtensorMap qmap, kmap, vmap;
-  const int rows = sh.block_size < Cfg::kKeys ? sh.block_size : Cfg::kKeys;
-  if ((e = encode_q_map(&qmap, q, sh.total_q, sh.num_heads, G, Cfg::kTok)) != cudaSuccess) return e;
-  if ((e = encode_kv_map(&kmap, k_cache, sh.num_blocks, sh.block_size, sh.num_kv_heads, rows)) !=
+  const int rows = p.block_size < Cfg::kKeys ? p.block_size : Cfg::kKeys;
+  if ((e = encode_q_map(&qmap, q, p.total_q, p.num_heads, G, Cfg::kTok)) != cudaSuccess) return e;
+  if ((e = encode_kv_map(&kmap, k_cache, p.num_blocks, p.block_size, p.num_kv_heads, rows)) !=
       cudaSuccess)
     return e;
-  if ((e = encode_kv_map(&vmap, v_cache, sh.num_blocks, sh.block_size, sh.num_kv_heads, rows)) !=
+  if ((e = encode_kv_map(&vmap, v_cache, p.num_blocks, p.block_size, p.num_kv_heads, rows)) !=
       cudaSuccess)
     return e;
-  constexpr int kCtaTok = Cfg::kQT * Cfg::kTok;
-  // work indices: every sequence could have max_query_len rows; those past
-  // the last item exit at once (they are dispatched last)
-  const int64_t items = static_cast<int64_t>(sh.num_seqs) *
-                        ((sh.max_query_len + kCtaTok - 1) / kCtaTok);
-  const int64_t ctas = items * sh.num_kv_heads;
+  if (ctas <= 0) return cudaSuccess;
   if (ctas > 0x7fffffff) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
@@ -607,7 +655,34 @@ cudaError_t launch_prefill_g(const PrefillShape& sh, const PrefillParams& p, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, pa_prefill_kernel<G>, qmap, kmap, vmap, p);
+  return cudaLaunchKernelEx(&cfg, pa_prefill_kernel<G, PREFIX>, qmap, kmap, vmap, p);
+}
+
+template <bool PREFIX>
+cudaError_t dispatch_prefill(const PrefillParams& p, const void* q, const void* k_cache,
+                             const void* v_cache, int64_t ctas, cudaStream_t stream) {
+  switch (p.num_heads / p.num_kv_heads) {
+    case 1: return launch_prefill_g<1, PREFIX>(p, q, k_cache, v_cache, ctas, stream);
+    case 2: return launch_prefill_g<2, PREFIX>(p, q, k_cache, v_cache, ctas, stream);
+    case 4: return launch_prefill_g<4, PREFIX>(p, q, k_cache, v_cache, ctas, stream);
+    case 8: return launch_prefill_g<8, PREFIX>(p, q, k_cache, v_cache, ctas, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+PrefillParams common_params(int num_heads, int num_kv_heads, int block_size, int num_blocks,
+                            int max_blocks_per_seq, float scale) {
+  PrefillParams p{};
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.block_size = block_size;
+  int lg = 0;
+  while ((1 << lg) < block_size) ++lg;
+  p.log2_block_size = lg;
+  p.num_blocks = num_blocks;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.q_scale = scale * 1.4426950408889634f;  // log2(e)
+  return p;
 }
 
 }  // namespace
@@ -617,32 +692,61 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
                            const int32_t* context_lens, const int32_t* query_start,
                            cudaStream_t stream) {
   if (sh.max_query_len <= 0 || sh.num_seqs <= 0) return cudaSuccess;
-  PrefillParams p{};
+  PrefillParams p = common_params(sh.num_heads, sh.num_kv_heads, sh.block_size, sh.num_blocks,
+                                  sh.max_blocks_per_seq, sh.scale);
   p.out = static_cast<__nv_bfloat16*>(out);
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   p.query_start = query_start;
   cudaError_t e = device_error_word(&p.err);
   if (e != cudaSuccess) return e;
-  p.num_heads = sh.num_heads;
-  p.num_kv_heads = sh.num_kv_heads;
-  p.block_size = sh.block_size;
-  int lg = 0;
-  while ((1 << lg) < sh.block_size) ++lg;
-  p.log2_block_size = lg;
-  p.num_blocks = sh.num_blocks;
-  p.max_blocks_per_seq = sh.max_blocks_per_seq;
   p.num_seqs = sh.num_seqs;
   p.total_q = sh.total_q;
   p.max_query_len = sh.max_query_len;
-  p.q_scale = sh.scale * 1.4426950408889634f;  // log2(e)
-  switch (sh.num_heads / sh.num_kv_heads) {
-    case 1: return launch_prefill_g<1>(sh, p, q, k_cache, v_cache, stream);
-    case 2: return launch_prefill_g<2>(sh, p, q, k_cache, v_cache, stream);
-    case 4: return launch_prefill_g<4>(sh, p, q, k_cache, v_cache, stream);
-    case 8: return launch_prefill_g<8>(sh, p, q, k_cache, v_cache, stream);
-    default: return cudaErrorNotSupported;
-  }
+  // work indices: every sequence could have max_query_len rows; those past
+  // the last item exit at once (they are dispatched last)
+  const int tok = 2 * (128 / (sh.num_heads / sh.num_kv_heads));  // query tokens per CTA
+  const int64_t items = static_cast<int64_t>(sh.num_seqs) * ((sh.max_query_len + tok - 1) / tok);
+  return dispatch_prefill<false>(p, q, k_cache, v_cache, items * sh.num_kv_heads, stream);
+}
+
+int prefix_partition_keys(int num_seqs, int num_heads, int num_kv_heads, int prefix_len) {
+  // about one wave of CTAs: (KV heads) x (query-tile pairs) x (key partitions)
+  const int tok = 2 * (128 / (num_heads / num_kv_heads));
+  const int64_t pairs = (static_cast<int64_t>(num_seqs) + tok - 1) / tok;
+  int64_t parts = 148 / (static_cast<int64_t>(num_kv_heads) * pairs);
+  if (parts < 1) parts = 1;
+  int64_t keys = (prefix_len + parts - 1) / parts;
+  keys = (keys + 63) / 64 * 64;
+  return static_cast<int>(keys < 64 ? 64 : keys);
+}
+
+cudaError_t launch_prefix_attention(int num_seqs, int num_heads, int num_kv_heads, int block_size,
+                                    int num_blocks, int max_blocks_per_seq, int prefix_len,
+                                    int prefix_part, float scale, const void* q,
+                                    const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, float* ws_m, float* ws_l,
+                                    float* ws_acc, int ws_slots, cudaStream_t stream) {
+  PrefillParams p = common_params(num_heads, num_kv_heads, block_size, num_blocks,
+                                  max_blocks_per_seq, scale);
+  p.block_tables = block_tables;
+  cudaError_t e = device_error_word(&p.err);
+  if (e != cudaSuccess) return e;
+  p.num_seqs = num_seqs;
+  p.total_q = num_seqs;
+  p.max_query_len = num_seqs;
+  p.prefix_keys = prefix_len;
+  p.prefix_part = prefix_part;
+  p.prefix_parts = (prefix_len + prefix_part - 1) / prefix_part;
+  p.ws_slots = ws_slots;
+  p.ws_m = ws_m;
+  p.ws_l = ws_l;
+  p.ws_acc = ws_acc;
+  const int tok = 2 * (128 / (num_heads / num_kv_heads));
+  const int64_t pairs = (static_cast<int64_t>(num_seqs) + tok - 1) / tok;
+  return dispatch_prefill<true>(p, q, k_cache, v_cache,
+                                static_cast<int64_t>(num_kv_heads) * p.prefix_parts * pairs,
+                                stream);
 }
 
 }  // namespace pa

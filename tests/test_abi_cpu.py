@@ -122,6 +122,48 @@ def test_contiguous_decode_rejects_on_host(over, status):
     assert msg
 
 
+def _shared(**over):
+    a = dict(out=FAKE, q=FAKE, kn=None, vn=None, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, S=64, Hq=32,
+             Hkv=8, D=128, bs=16, nb=8192, mbps=256, prefix=2048, maxlen=3054, scale=0.1, P=0,
+             ws=FAKE, wsb=1 << 30, dt=pa.PA_BF16)
+    a.update(over)
+    st = pa._lib.pa_decode_shared_prefix(
+        a["out"], a["q"], a["kn"], a["vn"], a["k"], a["v"], a["bt"], a["cl"], a["S"], a["Hq"],
+        a["Hkv"], a["D"], a["bs"], a["nb"], a["mbps"], a["prefix"], a["maxlen"], a["scale"],
+        a["P"], a["ws"], a["wsb"], a["dt"], None)
+    return st, pa._lib.pa_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dt=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
+    (dict(D=64), pa.PA_ERR_UNSUPPORTED),
+    (dict(bs=4, mbps=1024), pa.PA_ERR_UNSUPPORTED),      # the prefix kernel's boxes need >= 8
+    (dict(Hq=24), pa.PA_ERR_UNSUPPORTED),                # group 3
+    (dict(prefix=0), pa.PA_ERR_INVALID),
+    (dict(prefix=2050), pa.PA_ERR_INVALID),              # not a multiple of the block size
+    (dict(prefix=3072), pa.PA_ERR_INVALID),              # past max_context_len
+    (dict(scale=-0.1), pa.PA_ERR_INVALID),
+    (dict(kn=FAKE), pa.PA_ERR_INVALID),                  # k_new without v_new
+    (dict(kn=ctypes.c_void_p(0x10008), vn=FAKE), pa.PA_ERR_INVALID),   # misaligned
+    (dict(ws=None, wsb=0), pa.PA_ERR_INVALID),
+    (dict(wsb=1024), pa.PA_ERR_INVALID),                 # workspace too small
+    (dict(P=24), pa.PA_ERR_INVALID),
+])
+def test_shared_prefix_decode_rejects_on_host(over, status):
+    st, msg = _shared(**over)
+    assert st == status, msg
+    assert msg
+
+
+def test_shared_prefix_workspace_holds_both_parts():
+    # the prefix's partitions and the suffix's, more than a plain decode of the suffix
+    both = pa.pa_decode_shared_prefix_workspace_bytes(64, 32, 8, 128, 2048, 3054, 0)
+    rest = pa.pa_decode_workspace_bytes(64, 32, 8, 128, 3054 - 2048, 0)
+    assert both > rest > 0
+    assert pa.pa_decode_shared_prefix_workspace_bytes(64, 32, 8, 128, 0, 3054, 0) == 0
+    assert _shared(S=0)[0] == pa.PA_OK
+
+
 def test_contiguous_decode_zero_sequences_is_a_no_op():
     assert _contig(S=0)[0] == pa.PA_OK
 

@@ -67,6 +67,23 @@ def test_cache_writes_and_block_copies(calls):
                                             "block_mapping", 3, 8, 2, 16, pa.PA_BF16, "stream"))
 
 
+def test_shared_prefix_decode_call(calls):
+    s, hq, hkv, d, nb, bs, mb = 3, 8, 2, 128, 10, 16, 4
+    kc, vc = z(nb, bs, hkv, d), z(nb, bs, hkv, d)
+    q, out = z(s, hq, d), z(s, hq, d)
+    tables, lens, ws = z(s, mb, dtype=I32), z(s, dtype=I32), z(1024, dtype=U8)
+    pa.pa_decode_shared_prefix(out, q, z(s, hkv, d), z(s, hkv, d), kc, vc, tables, lens, 32, 50,
+                               0.125, 16, ws)
+    name, a = calls[-1]
+    assert name == "pa_decode_shared_prefix"
+    assert a[:8] == ("out", "q", "k_new", "v_new", "k_cache", "v_cache", "block_tables",
+                     "context_lens")
+    assert a[8:20] == (s, hq, hkv, d, bs, nb, mb, 32, 50, pytest.approx(0.125), 16, "workspace")
+    assert a[20:] == (1024, pa.PA_BF16, "stream")
+    pa.pa_decode_shared_prefix(out, q, None, None, kc, vc, tables, lens, 32, 50, 0.125, 0, ws)
+    assert calls[-1][1][2:4] == (None, None)
+
+
 def test_contiguous_decode_call(calls):
     s, hq, hkv, d, slab = 3, 8, 2, 128, 64
     k, v = z(s, slab, hkv, d), z(s, slab, hkv, d)

@@ -1,0 +1,123 @@
+"""pa_decode_shared_prefix on the GPU: decode for sequences that share their
+first blocks ("PagedAttention — AI Glossary", How it works, step 4), the shared
+prefix attended once for the whole batch on the tensor cores, each sequence's
+own tokens by the decode kernel, the two merged per row.
+
+The result is attention over each sequence's whole context: it must match the
+float64 oracle (bf16 tolerance) and the plain paged decode of the same tokens;
+with the step's append, the cache rows it writes must equal pa_decode_append's
+bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_harness as gh
+import paged_kv_cache_345_b200 as pa
+from workloads import configs
+
+pytestmark = pytest.mark.gpu
+
+
+def _shared_decode(case, prefix_len, k_new=None, v_new=None, ps=0):
+    tables, lens, max_len = case.cache.tables(case.seqs)
+    q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+    s, hq, d = q.shape
+    need = pa.pa_decode_shared_prefix_workspace_bytes(s, hq, case.cache.num_kv_heads, d,
+                                                      prefix_len, max_len, ps)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)  # contents on entry are ignored
+    out = torch.full_like(q, float("nan"))
+    pa.pa_decode_shared_prefix(out, q, k_new, v_new, case.cache.k_cache, case.cache.v_cache,
+                               tables, lens, prefix_len, max_len, case.scale, ps, ws)
+    torch.cuda.synchronize()
+    return out
+
+
+def test_shared_prefix_workload_matches_oracle_and_paged_decode():
+    """64 sequences forked from a 2,053-token parent (the 128 whole blocks stay
+    shared, the partly filled 129th was copied on write) plus their own
+    suffixes: attended after the step's append."""
+    wl = configs.shared_prefix()
+    case = gh.build_case(wl)
+    prefix = (wl.shared_prefix // wl.block_size) * wl.block_size
+    out = _shared_decode(case, prefix)
+    assert pa.pa_device_errors() == 0
+    got = out.float().cpu().numpy()
+    gh.assert_close(got, gh.expected_all(case), "bf16", "shared prefix vs oracle")
+    gh.assert_close(got, gh.gpu_out(case), "bf16", "shared prefix vs pa_decode_append")
+
+
+def _custom(hq, hkv, bs, prefix, suffixes, seed):
+    lens = tuple(prefix + x for x in suffixes)
+    nb = -(-prefix // bs) + sum(-(-(x + 2) // bs) for x in suffixes) + 16
+    return configs.Workload(f"shared_{hq}_{hkv}_{bs}_{prefix}", hq, hkv, 128, "bf16", bs, nb, lens,
+                            5400 + seed, 6400 + seed, shared_prefix=prefix)
+
+
+@pytest.mark.parametrize("hq,hkv,bs,prefix,nseq", [
+    (8, 8, 16, 144, 5),      # group 1; a prefix that is not a multiple of 64 keys
+    (32, 8, 8, 512, 70),     # group 4, block 8, two pairs of query tiles (64 rows each)
+    (16, 2, 64, 1024, 9),    # group 8, block 64
+])
+def test_ragged_shapes(hq, hkv, bs, prefix, nseq):
+    rng = np.random.default_rng(nseq)
+    suffixes = [0] + [int(x) for x in rng.integers(0, 300, size=nseq - 1)]
+    wl = _custom(hq, hkv, bs, prefix, suffixes, nseq)
+    case = gh.build_case(wl)
+    out = _shared_decode(case, prefix, ps=64)
+    assert pa.pa_device_errors() == 0
+    got = out.float().cpu().numpy()
+    gh.assert_close(got, gh.expected_all(case), "bf16", f"G={hq // hkv} bs={bs}")
+    gh.assert_close(got, gh.gpu_out(case), "bf16", "vs pa_decode_append")
+
+
+def test_fused_append_writes_what_decode_append_writes():
+    """A second decode step, once through pa_decode_append and once through
+    pa_decode_shared_prefix on a copy of the cache: identical cache contents,
+    outputs within tolerance of each other."""
+    wl = _custom(32, 8, 16, 256, [3, 40, 17, 200], 1)
+    case = gh.build_case(wl)
+    s = len(case.seqs)
+    slots, cows = case.cache.bm.append_slots(case.seqs, [1] * s)
+    assert len(cows) == 0
+    tables, lens, max_len = case.cache.tables(case.seqs)
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    k_new = torch.randn((s, 8, 128), device="cuda", generator=gen).to(torch.bfloat16)
+    v_new = torch.randn((s, 8, 128), device="cuda", generator=gen).to(torch.bfloat16)
+    q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+    k_a, v_a = case.cache.k_cache.clone(), case.cache.v_cache.clone()
+    ws_a = torch.empty(pa.pa_decode_workspace_bytes(s, 32, 8, 128, max_len, 64) + 16,
+                       dtype=torch.uint8, device="cuda")
+    out_a = torch.empty_like(q)
+    pa.pa_decode_append(out_a, q, k_new, v_new, k_a, v_a, tables, lens, max_len, wl.scale, 64,
+                        ws_a)
+    ws_b = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(s, 32, 8, 128, 256, max_len, 64),
+                       dtype=torch.uint8, device="cuda")
+    out_b = torch.empty_like(q)
+    pa.pa_decode_shared_prefix(out_b, q, k_new, v_new, case.cache.k_cache, case.cache.v_cache,
+                               tables, lens, 256, max_len, wl.scale, 64, ws_b)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(case.cache.k_cache, k_a) and torch.equal(case.cache.v_cache, v_a)
+    gh.assert_close(out_b.float().cpu().numpy(), out_a.float().cpu().numpy(), "bf16", "append")
+
+
+def test_context_shorter_than_the_prefix_is_flagged():
+    wl = _custom(32, 8, 16, 256, [10, 20], 2)
+    case = gh.build_case(wl)
+    tables, lens, max_len = case.cache.tables(case.seqs)
+    short = lens.clone()
+    short[1] = 100                     # shorter than the 256-token prefix
+    q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(2, 32, 8, 128, 256, max_len, 0),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    pa.pa_decode_shared_prefix(out, q, None, None, case.cache.k_cache, case.cache.v_cache, tables,
+                               short, 256, max_len, wl.scale, 0, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT
+    # the sequence with a valid context is still right
+    ref = gh.expected_all(case)
+    gh.assert_close(out[0].float().cpu().numpy(), ref[0], "bf16", "valid row")
