@@ -59,6 +59,9 @@ def parse_args():
                     help="tokens per split-K partition (-1: tuned default, 0: library choice)")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared_prefix only: time pa_decode_shared_prefix (the prefix once "
+                         "for the batch) instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-back-to-back", action="store_true")
     ap.add_argument("--compact-pool", action="store_true",
@@ -307,6 +310,7 @@ class StepCalls:
             self.fns = (self.fns[0], self.fns[1], self.lib.pa_decode_shared_prefix)
             self.fused = True
             self.launches_per_step = 3
+            self.partition_size = partition_size   # 0: the library's choice for the suffixes
 
     def _call(self, fn, args):
         st = fn(*args)
@@ -790,7 +794,8 @@ def pa_device_errors_or_raise():
         raise RuntimeError("device error word set")
 
 
-def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp8=False):
+def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp8=False,
+                  prefix_len=0):
     """StepCalls over `layers` copies of the cache (one per model layer)."""
     import paged_kv_cache_345_b200 as pa  # noqa: F401
 
@@ -800,7 +805,8 @@ def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp
         view.k_cache, view.v_cache = cache.k_cache.clone(), cache.v_cache.clone()
         if fp8:
             view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
-        out.append(StepCalls(view, dev, max_len, scale, ps, stream, fused=fused))
+        out.append(StepCalls(view, dev, max_len, scale, ps, stream, fused=fused,
+                             prefix_len=prefix_len))
     return out
 
 
@@ -832,7 +838,8 @@ def back_to_back(layer_calls, stream, reps, early):
     return per_layer
 
 
-def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early, fp8=False):
+def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early, fp8=False,
+                   prefix_len=0):
     """End to end through the C ABI with the host copies pipelined: two pinned
     host packs and two device packs; for step i the inputs go host -> device on
     an upload stream (pack i % 2, once step i - 2 has finished reading it), the
@@ -853,7 +860,8 @@ def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early,
         view.k_cache, view.v_cache = cache.k_cache.clone(), cache.v_cache.clone()
         if fp8:
             view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
-        calls.append(StepCalls(view, packs[i % 2][1], max_len, scale, ps, stream))
+        calls.append(StepCalls(view, packs[i % 2][1], max_len, scale, ps, stream,
+                               prefix_len=prefix_len))
     outs_host = [torch.empty(calls[0].out.shape, dtype=calls[0].out.dtype).pin_memory()
                  for _ in range(2)]
     up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
@@ -923,7 +931,14 @@ def run_b200(args, wl, rank, world, local_rank):
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl, device, args.placement)
     ps = TUNED_PARTITION[wl.name.split("_bs")[0].replace("_compact", "")] \
         if args.partition_size < 0 else args.partition_size
-    calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused)
+    prefix_len = 0
+    if args.cascade:
+        if not wl.shared_prefix:
+            raise SystemExit("--cascade needs a workload with a shared prefix")
+        prefix_len = (wl.shared_prefix // wl.block_size) * wl.block_size
+        ps = 0 if args.partition_size < 0 else args.partition_size
+    calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused,
+                      prefix_len=prefix_len)
     launches_per_step, part_size = calls.launches_per_step, calls.partition_size
     num_partitions = calls.num_partitions
     bytes_step = kv_bytes_unique(wl)
@@ -971,7 +986,7 @@ def run_b200(args, wl, rank, world, local_rank):
             ov_ms, oh2d, od2h = e2e_overlapped(cache, host, max_len, wl.scale,
                                                calls.partition_size, stream, args.layers,
                                                max(5, min(50, args.steps // args.layers)), early,
-                                               calls.fp8)
+                                               calls.fp8, prefix_len)
             pa_device_errors_or_raise()
             e2e["overlapped"] = {
                 "value": bytes_step / (ov_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -984,7 +999,8 @@ def run_b200(args, wl, rank, world, local_rank):
     b2b = None
     if not args.no_back_to_back and world == 1:
         layer_calls = replica_calls(cache, dev, max_len, wl.scale, calls.partition_size, stream,
-                                    args.layers, fused=calls.fused, fp8=calls.fp8)
+                                    args.layers, fused=calls.fused, fp8=calls.fp8,
+                                    prefix_len=prefix_len)
         reps = max(5, min(50, args.steps // args.layers))
         per_layer_ms = back_to_back(layer_calls, stream, reps, early)
         pa_device_errors_or_raise()
@@ -1013,7 +1029,8 @@ def run_b200(args, wl, rank, world, local_rank):
     # ---- roofline of the headline step
     dec_s = statistics.mean(step_ms) * 1e-3
     achieved = bytes_step / dec_s / 1e9
-    traffic = load_traffic(f"pa_decode_{wl.name}" + ("_fp8" if wl.cache_dtype != "bf16" else ""))
+    traffic = load_traffic(f"pa_decode_{wl.name}" + ("_fp8" if wl.cache_dtype != "bf16" else "")
+                           + ("_cascade" if prefix_len else ""))
 
     # ---- host side and CPU baseline (rank 0, one GPU only)
     host_side = host_allocator_metrics() if rank == 0 else None
@@ -1034,14 +1051,16 @@ def run_b200(args, wl, rank, world, local_rank):
                    "partition_size": part_size, "num_partitions": num_partitions,
                    "copy_on_write_pairs": cow_pairs,
                    "placement": args.placement, "kv_cache": wl.cache_dtype,
-                   "early_cache_reads": bool(early),
+                   "early_cache_reads": bool(early), "shared_prefix_len": prefix_len,
                    "l2": flush.describe(), "parallelism": f"replicas x{world}"},
         "attended_tokens_per_s": whole_job_rate(tokens_step, args.steps, world, total_ms),
         "us_per_step": 1e3 * total_ms / args.steps,
         "step_us_p10_p50_p90": [1e3 * float(np.percentile(step_ms, p)) for p in (10, 50, 90)],
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": ("pa_decode_append (fused append + decode kernel, split-K "
+                     "kernel": ("pa_decode_shared_prefix (prefix attention kernel, fused "
+                                "append + suffix decode kernel, merge kernel)" if prefix_len else
+                                "pa_decode_append (fused append + decode kernel, split-K "
                                 "merge kernel)" if not args.unfused else
                                 "pa_kv_append + pa_decode (decode + split-K merge kernels)"),
                      "peak_source": f"{peak_src} hbm_gbs"},

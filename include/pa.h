@@ -333,6 +333,11 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
  *   - each sequence's own tokens [prefix_len, context_lens[s]) with the decode
  *     kernel (appending each newest token there when k_new / v_new are given);
  *   - the partial results of both combined per row with a log-sum-exp rescale.
+ * Three kernels on `stream`: the prefix pass (a few SMs) and the suffix decode
+ * run at the same time, the merge after both. The call waits for all earlier
+ * work on the stream before it reads q, k_new or v_new or writes anything, as
+ * pa_decode does; PA_DECODE_EARLY_CACHE_READS does not apply to it.
+ * partition_size (0: the library's choice) sets the suffix partitions.
  *
  *   k_new, v_new   NULL (attend only) or each sequence's newest K/V row
  *                  [num_seqs][num_kv_heads][head_dim], written at position

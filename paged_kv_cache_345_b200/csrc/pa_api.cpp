@@ -404,11 +404,21 @@ PrefixPlan plan_shared_prefix(int num_seqs, int num_heads, int num_kv_heads, int
                               int max_context_len, int partition_size) {
   PrefixPlan pl{};
   const int rest = max_context_len - prefix_len;
-  pl.suffix_part = partition_size == 0
-                       ? pa_decode_partition_size(num_seqs, num_kv_heads, rest > 0 ? rest : 0)
-                       : partition_size;
+  if (partition_size == 0) {
+    // the suffix decode runs on the SMs the prefix pass leaves and its end is
+    // the critical path: two thirds of the plain decode's partition, for a
+    // shorter tail (64 sequences, suffixes of 50..1000 tokens: 208 tokens
+    // 41.0 us a step, the plain choice 304 tokens 45.5 us)
+    const int c = pa::kChunkTokens;
+    const int plain = pa_decode_partition_size(num_seqs, num_kv_heads, rest > 0 ? rest : 0);
+    pl.suffix_part = ((plain * 2 / 3 + c - 1) / c) * c;
+    if (pl.suffix_part < 64) pl.suffix_part = 64;
+  } else {
+    pl.suffix_part = partition_size;
+  }
   pl.suffix_parts = rest <= 0 ? 1 : (rest + pl.suffix_part - 1) / pl.suffix_part;
-  pl.prefix_part = pa::prefix_partition_keys(num_seqs, num_heads, num_kv_heads, prefix_len);
+  pl.prefix_part =
+      pa::prefix_partition_keys(num_seqs, num_heads, num_kv_heads, prefix_len, max_context_len);
   pl.prefix_parts = (prefix_len + pl.prefix_part - 1) / pl.prefix_part;
   return pl;
 }

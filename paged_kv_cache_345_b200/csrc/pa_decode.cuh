@@ -58,7 +58,7 @@ struct DecodeParams {
   // E4M3 caches: cache value = code * scale, one scale per KV head [Hkv]. Null otherwise.
   const float* k_scale;
   const float* v_scale;
-  int num_heads, num_kv_heads, block_size, log2_block_size, num_blocks;
+  int num_seqs, num_heads, num_kv_heads, block_size, log2_block_size, num_blocks;
   int max_blocks_per_seq, max_context_len, partition_size, num_partitions;
   float q_scale;  // scale * log2(e)
   // PA_DECODE_EARLY_CACHE_READS: the caller vouches that no kernel still
@@ -86,8 +86,10 @@ __device__ __forceinline__ void append_newest_rows(const DecodeParams& p, int s,
   const int64_t dst =
       ((static_cast<int64_t>(blk) * p.block_size + off) * p.num_kv_heads + h0) * row_bytes;
   for (int64_t i = lane; i < vec; i += 32) {
-    const uint4 a = ldg_stream(p.k_new + src + i * 16);
-    const uint4 b = ldg_stream(p.v_new + src + i * 16);
+    // read at L2 (not through L1): under a shared-prefix decode these rows
+    // are read without a dependent-launch wait in this kernel
+    const uint4 a = __ldcg(reinterpret_cast<const uint4*>(p.k_new + src + i * 16));
+    const uint4 b = __ldcg(reinterpret_cast<const uint4*>(p.v_new + src + i * 16));
     *reinterpret_cast<uint4*>(p.k_cache_w + dst + i * 16) = a;
     *reinterpret_cast<uint4*>(p.v_cache_w + dst + i * 16) = b;
   }
@@ -108,8 +110,8 @@ __device__ __forceinline__ void append_newest_rows_fp8(const DecodeParams& p, in
     const int h = h0 + i * 16 / head_dim;
     const uint4* ks = reinterpret_cast<const uint4*>(p.k_new + src) + 2 * i;
     const uint4* vs = reinterpret_cast<const uint4*>(p.v_new + src) + 2 * i;
-    const uint4 kc = bf16x16_to_e4m3(ldg_stream(ks), ldg_stream(ks + 1), __ldg(p.k_scale + h));
-    const uint4 vc = bf16x16_to_e4m3(ldg_stream(vs), ldg_stream(vs + 1), __ldg(p.v_scale + h));
+    const uint4 kc = bf16x16_to_e4m3(__ldcg(ks), __ldcg(ks + 1), __ldg(p.k_scale + h));
+    const uint4 vc = bf16x16_to_e4m3(__ldcg(vs), __ldcg(vs + 1), __ldg(p.v_scale + h));
     *reinterpret_cast<uint4*>(p.k_cache_w + dst + i * 16) = kc;
     *reinterpret_cast<uint4*>(p.v_cache_w + dst + i * 16) = vc;
   }
@@ -439,37 +441,49 @@ __global__ void __launch_bounds__(DecodeConfig<T, D, G>::kThreads)
 }
 
 
-// Split-K merge: one CTA of 4 warps per (sequence, query head) row with more
-// than one partition:
+// Split-K merge, for rows (sequence, query head) with more than one partial
+// result:
 //   M = max_p m_p,  Lambda = sum_p l_p 2^(m_p - M),  out = sum_p 2^(m_p - M) acc_p / Lambda.
-// Warp w takes partitions w, w + 4, ... in batches of 8: a batch's maxima,
-// sums and accumulator rows (each lane owns D / 32 columns) are loaded
-// together, so a row with up to 32 partitions costs one round trip; batches
-// are folded in with an online rescale. The four warps' results are combined
-// in warp order through shared memory: the result depends only on the
-// partials (deterministic). Launched with programmatic dependent launch.
-template <typename T, int D>
+// W warps per row (1, 2 or 4, chosen on the host from the partition count),
+// 4 / W rows per CTA of 4 warps: few partials need few threads, and the grid
+// stays within one wave of resident CTAs. Warp w of a row takes partitions
+// w, w + W, ... in batches of 8: a batch's maxima, sums and accumulator rows
+// (each lane owns D / 32 columns) are loaded together, so a row with up to
+// 8 W partitions costs one round trip; batches are folded in with an online
+// rescale. With W > 1 the row's warps are combined in warp order through
+// shared memory. The result depends only on the partials (deterministic).
+// Launched with programmatic dependent launch.
+template <typename T, int D, int W>
 __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
+  static_assert(W == 1 || W == 2 || W == 4, "warps per row");
   constexpr int E = D / 32;  // columns per lane
   constexpr int B = 8;       // partitions per warp per batch
+  constexpr int R = 4 / W;   // rows per CTA
   using Vec = typename std::conditional<E == 4, float4, float2>::type;
   __shared__ float s_m[4], s_l[4], s_acc[4][D];
-  const int64_t r = blockIdx.x;  // row = s * num_heads + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wr = warp % W;  // this warp's place among its row's warps
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * R + warp / W;  // s * num_heads + j
   const int s = static_cast<int>(r / p.num_heads);
   // The context length is read before the dependent-launch wait: the kernel
   // before this one is the decode kernel of the same call, which waited for all
   // earlier work before letting this kernel start (or, under
   // PA_DECODE_EARLY_CACHE_READS, the caller vouches that nothing still running
-  // writes it), and neither kernel writes it.
-  const int L = __ldg(p.context_lens + s);
-  if (L < 0 || L > p.max_context_len ||
-      static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size ||
-      L < p.first_token)
-    return;  // flagged (and, without a prefix, zero-filled) by the decode kernel
-  // partial results: the prefix's slots, then this row's own partitions
-  const int np = p.prefix_slots + (L - p.first_token + p.partition_size - 1) / p.partition_size;
-  if (np <= 1 && p.prefix_slots == 0) return;  // written directly by the decode kernel
+  // writes it), and neither kernel writes it. Rows without partials (flagged,
+  // and without a prefix zero-filled, by the decode kernel; or written there
+  // directly) are skipped.
+  int np = 0;
+  if (s < p.num_seqs) {
+    const int L = __ldg(p.context_lens + s);
+    if (!(L < 0 || L > p.max_context_len ||
+          static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size ||
+          L < p.first_token)) {
+      // partial results: the prefix's slots, then this row's own partitions
+      np = p.prefix_slots + (L - p.first_token + p.partition_size - 1) / p.partition_size;
+      if (np <= 1 && p.prefix_slots == 0) np = 0;
+    }
+  }
+  if (W == 1 && np == 0) return;  // (W > 1: every warp reaches the barrier below)
   // The next kernel may start its launch now: whatever it reads before its
   // own wait is, by the same contract, not written here.
   pdl_launch_dependents();
@@ -479,12 +493,12 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
   float Mw = -INFINITY, Lw = 0.0f, acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-  for (int q0 = warp; q0 < np; q0 += 4 * B) {
+  for (int q0 = wr; q0 < np; q0 += W * B) {
     float mq[B], lq[B];
     Vec vq[B];
 #pragma unroll
     for (int j = 0; j < B; ++j) {
-      const int q = q0 + 4 * j;
+      const int q = q0 + W * j;
       if (q < np) {
         mq[j] = __ldcg(p.ws_m + row + q);
         lq[j] = __ldcg(p.ws_l + row + q);
@@ -512,24 +526,37 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
     }
     Mw = bm;
   }
+  if constexpr (W == 1) {
 #pragma unroll
-  for (int e = 0; e < E; ++e) s_acc[warp][lane * E + e] = acc[e];
-  if (lane == 0) {
-    s_m[warp] = Mw;
-    s_l[warp] = Lw;
-  }
-  __syncthreads();
-  if (threadIdx.x < D) {
-    const int d = threadIdx.x;
-    const float M = fmaxf(fmaxf(s_m[0], s_m[1]), fmaxf(s_m[2], s_m[3]));
-    float lsum = 0.0f, v = 0.0f;
+    for (int e = 0; e < E; ++e)
+      ElemTraits<T>::store(static_cast<T*>(p.out) + r * D + lane * E + e, acc[e] / Lw);
+  } else {
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = s_m[w] == -INFINITY ? 0.0f : exp2f(s_m[w] - M);
-      lsum = fmaf(f, s_l[w], lsum);
-      v = fmaf(f, s_acc[w][d], v);
+    for (int e = 0; e < E; ++e) s_acc[warp][lane * E + e] = acc[e];
+    if (lane == 0) {
+      s_m[warp] = Mw;
+      s_l[warp] = Lw;
     }
-    ElemTraits<T>::store(static_cast<T*>(p.out) + r * D + d, v / lsum);
+    __syncthreads();
+    // the row's 32 W threads: columns t, t + 32 W, ... of the row
+    const int t = threadIdx.x % (32 * W), w0 = warp - wr;
+    if (np > 0) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < W; ++w) M = fmaxf(M, s_m[w0 + w]);
+      float f[W], lsum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        f[w] = s_m[w0 + w] == -INFINITY ? 0.0f : exp2f(s_m[w0 + w] - M);
+        lsum = fmaf(f[w], s_l[w0 + w], lsum);
+      }
+      for (int d = t; d < D; d += 32 * W) {
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) v = fmaf(f[w], s_acc[w0 + w][d], v);
+        ElemTraits<T>::store(static_cast<T*>(p.out) + r * D + d, v / lsum);
+      }
+    }
   }
 }
 

@@ -135,8 +135,18 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   // ring stages fill while that kernel drains; the waits then come right
   // before q (consumers), before the fused append reads k_new / v_new
   // (producer), and before any write.
+  //
+  // A shared-prefix decode (prefix_slots > 0) runs beside the prefix kernel
+  // launched just before it, which waited for all earlier work before letting
+  // this grid start and reads neither the rows this kernel writes nor their
+  // workspace slots: no thread here waits, q and k_new / v_new are read
+  // through L2, and one thread of the grid (gate) waits for the prefix kernel
+  // before its CTA ends, so that the merge, which waits for this grid, also
+  // finds the prefix's partial results.
   const bool early = p.early_reads != 0;
-  if (!early) pdl_wait();
+  const bool cascade = p.prefix_slots > 0;
+  const bool gate = cascade && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  if (!early && !cascade) pdl_wait();
   pdl_launch_dependents();
 
   // Independent loads first so their latencies overlap: the context length,
@@ -162,8 +172,9 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     if constexpr (!FP8) {
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        qa[ks][0] = real_row ? __ldg(qp + ks * 8 + qc) : 0u;
-        qa[ks][1] = real_row ? __ldg(qp + ks * 8 + 4 + qc) : 0u;
+        qa[ks][0] = real_row ? (cascade ? __ldcg(qp + ks * 8 + qc) : __ldg(qp + ks * 8 + qc)) : 0u;
+        qa[ks][1] = real_row ? (cascade ? __ldcg(qp + ks * 8 + 4 + qc) : __ldg(qp + ks * 8 + 4 + qc))
+                             : 0u;
       }
     } else {
       // k-step 4kq + j covers head_dim 16 (2 qc + kq) + 4j .. +3 (b0: +0, +1; b1: +2, +3),
@@ -171,8 +182,8 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
 #pragma unroll
       for (int kq = 0; kq < D / 64; ++kq) {
         const uint4* q4 = reinterpret_cast<const uint4*>(qp) + 2 * (2 * qc + kq);
-        const uint4 lo = real_row ? __ldg(q4) : make_uint4(0, 0, 0, 0);
-        const uint4 hi = real_row ? __ldg(q4 + 1) : make_uint4(0, 0, 0, 0);
+        const uint4 lo = real_row ? (cascade ? __ldcg(q4) : __ldg(q4)) : make_uint4(0, 0, 0, 0);
+        const uint4 hi = real_row ? (cascade ? __ldcg(q4 + 1) : __ldg(q4 + 1)) : make_uint4(0, 0, 0, 0);
         const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -186,7 +197,8 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   // waited; under early reads only after the CTA barrier below, so that the
   // producer, which does not wait before its first loads, is never held back
   // by consumers that do
-  if (warp < HB && !early) load_q();
+  const bool q_late = early && !cascade;
+  if (warp < HB && !q_late) load_q();
 
   if (L < 0 || L > p.max_context_len ||
       static_cast<int64_t>(L) > static_cast<int64_t>(p.max_blocks_per_seq) * bs ||
@@ -197,15 +209,13 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   L -= p.first_token;  // the tokens this kernel attends (all of them without a prefix)
   const int n_part_s = (L + P - 1) / P;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-  const bool to_merge = p.prefix_slots > 0;  // every row is left to the merge
+  const bool to_merge = cascade;  // every row is left to the merge
 
   if (L == 0) {  // empty context: zeros for every query head of the group
     if (to_merge) {  // the prefix's partial results are the whole row
       // (a newest token to append would lie inside the shared prefix)
       if (p.k_new != nullptr && threadIdx.x == 0 && hg == 0) atomicOr(p.err, PA_DEVERR_CONTEXT);
-      // the merge waits for this grid only: this grid must not end before the
-      // prefix kernel ahead of it, even when no CTA of it has tokens to attend
-      if (early) pdl_wait();
+      if (gate && threadIdx.x == 0) pdl_wait();
       return;
     }
     if (early) pdl_wait();
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   const int t1 = min(t0 + P, L);
   const int nchunks = (t1 - t0 + C - 1) / C;
   __syncthreads();
-  if (warp < HB && early) {
+  if (warp < HB && q_late) {
     pdl_wait();
     load_q();
   }
@@ -257,7 +267,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
         // this CTA holds the sequence's newest token: write it before reading it
         const int tn = L - 1;
         const int bn = __shfl_sync(kFullMask, ent, (tn >> lg) - base);
-        if (early) pdl_wait();  // k_new / v_new come from the previous kernel
+        if (q_late) pdl_wait();  // k_new / v_new come from the previous kernel
         if (static_cast<unsigned>(bn) < static_cast<unsigned>(p.num_blocks)) {
           if constexpr (FP8)
             append_newest_rows_fp8(p, s, bn, tn & (bs - 1), hg * HB, HB, D, lane);
@@ -282,6 +292,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
         tma_load_4d(d + TB, &v_map, 0, off, hg * HB, blk, full_bar);
       }
     }
+    if (gate && lane == 0) pdl_wait();
     return;
   }
 

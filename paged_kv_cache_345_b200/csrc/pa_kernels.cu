@@ -349,8 +349,14 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<unsigned long long
 template <typename T, int D>
 cudaError_t launch_merge(const DecodeShape& sh, const DecodeParams& p, cudaStream_t stream) {
   if (sh.num_partitions <= 1 && sh.prefix_slots == 0) return cudaSuccess;
+  // warps per row: enough to load every partial of a row in one batch of 8
+  // per warp, at most 4
   const unsigned rows = static_cast<unsigned>(sh.num_seqs) * sh.num_heads;
-  return launch_pdl(pa_merge_kernel<T, D>, dim3(rows), dim3(128), 0, stream, p);
+  if (sh.num_partitions <= 8)
+    return launch_pdl(pa_merge_kernel<T, D, 1>, dim3((rows + 3) / 4), dim3(128), 0, stream, p);
+  if (sh.num_partitions <= 16)
+    return launch_pdl(pa_merge_kernel<T, D, 2>, dim3((rows + 1) / 2), dim3(128), 0, stream, p);
+  return launch_pdl(pa_merge_kernel<T, D, 4>, dim3(rows), dim3(128), 0, stream, p);
 }
 
 // float32 caches: CUDA-core kernel (tensor maps, exact fp32 products).
@@ -502,6 +508,7 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   }
   cudaError_t e = device_error_word(&p.err);
   if (e != cudaSuccess) return e;
+  p.num_seqs = sh.num_seqs;
   p.num_heads = sh.num_heads;
   p.num_kv_heads = sh.num_kv_heads;
   p.block_size = sh.block_size;
