@@ -448,8 +448,9 @@ __global__ void __launch_bounds__(DecodeConfig<T, D, G>::kThreads)
 // 4 / W rows per CTA of 4 warps: few partials need few threads, and the grid
 // stays within one wave of resident CTAs. Warp w of a row takes partitions
 // w, w + W, ... in batches of 8: a batch's maxima, sums and accumulator rows
-// (each lane owns D / 32 columns) are loaded together, so a row with up to
-// 8 W partitions costs one round trip; batches are folded in with an online
+// (each lane owns D / 32 columns) are loaded together (volatile loads, kept
+// ahead of their uses), so a row with up to 8 W partitions costs one round
+// trip; batches are folded in with an online
 // rescale. With W > 1 the row's warps are combined in warp order through
 // shared memory. The result depends only on the partials (deterministic).
 // Launched with programmatic dependent launch.
@@ -496,14 +497,21 @@ __global__ void __launch_bounds__(128) pa_merge_kernel(const DecodeParams p) {
   for (int q0 = wr; q0 < np; q0 += W * B) {
     float mq[B], lq[B];
     Vec vq[B];
+    // no branch around the loads: a slot past the row's last partial loads
+    // that partial again and is masked below
 #pragma unroll
     for (int j = 0; j < B; ++j) {
-      const int q = q0 + W * j;
-      if (q < np) {
-        mq[j] = __ldcg(p.ws_m + row + q);
-        lq[j] = __ldcg(p.ws_l + row + q);
-        vq[j] = __ldcg(reinterpret_cast<const Vec*>(a + static_cast<int64_t>(q) * D));
-      } else {
+      const int q = min(q0 + W * j, np - 1);
+      mq[j] = ld_cg_f32(p.ws_m + row + q);
+      lq[j] = ld_cg_f32(p.ws_l + row + q);
+      if constexpr (E == 4)
+        vq[j] = ld_cg_f32x4(a + static_cast<int64_t>(q) * D);
+      else
+        vq[j] = ld_cg_f32x2(a + static_cast<int64_t>(q) * D);
+    }
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      if (q0 + W * j >= np) {
         mq[j] = -INFINITY;
         lq[j] = 0.0f;
         vq[j] = Vec{};
