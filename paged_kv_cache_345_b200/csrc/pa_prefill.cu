@@ -89,14 +89,13 @@ struct PrefillConfig {
   static constexpr int kQHalf = kQBytes / 2;
   static constexpr int kKVBytes = kKeys * kD * 2;    // a K or V tile: two halves of 8 KB
   static constexpr int kKVHalf = kKVBytes / 2;
-  static constexpr int kPBytes = kRows * kKeys * 2;  // a P tile: one 16 KB swizzle atom wide
   static constexpr int kNS = 4;                      // K/V stages
-  static constexpr int kQ = 0, kP = kQT * kQBytes, kStage0 = kP + kQT * kPBytes;
+  static constexpr int kQ = 0, kStage0 = kQT * kQBytes;  // (P lives in tensor memory)
   static constexpr int kBars = kStage0 + kNS * 2 * kKVBytes;
   static constexpr int kSmemBytes = kBars + 256;     // the base is 1024-byte aligned
   // producer, S-MMA issuer, 2 x 4 softmax warps, P V-MMA issuer
   static constexpr int kThreads = 352;
-  static constexpr uint32_t kTmemCols = 512;         // S[x][2] (64 each), O[x] (128 each)
+  static constexpr uint32_t kTmemCols = 512;  // S[x][2] (64 each; P over its first 32), O[x] (128 each)
   static_assert(kRows % G == 0, "group must divide the row tile");
 };
 
@@ -109,8 +108,8 @@ enum : int {
   kKVEmpty = 5,   // [kNS]: a commit of each MMA issuer
   kSFull = 9,     // [query tile][j % 2]
   kPFull = 13,    // [query tile][j % 2]
-  kODone = 17,    // [query tile]
-  kNumBars = 19
+  kODone = 17,    // [query tile][j % 2]: P V of tile j done (its P read, O updated)
+  kNumBars = 21
 };
 constexpr int kTmemSlotOffset = 192;  // after the barriers
 
@@ -219,7 +218,6 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kBars + kTmemSlotOffset);
   auto bar = [&](int i) { return smem_u32(bars + i); };
   auto q_s = [&](int x) { return smem_u32(sm + Cfg::kQ + x * Cfg::kQBytes); };
-  auto p_s = [&](int x) { return smem_u32(sm + Cfg::kP + x * Cfg::kPBytes); };
   auto k_s = [&](int st) { return smem_u32(sm + Cfg::kStage0 + st * 2 * Cfg::kKVBytes); };
   auto v_s = [&](int st) { return k_s(st) + Cfg::kKVBytes; };
 
@@ -299,8 +297,8 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     for (int i = 0; i < 2 * Cfg::kQT; ++i) {
       mbar_init(bar(kSFull + i), 1);    // MMA commit after S of the tile
       mbar_init(bar(kPFull + i), 128);  // every thread of the softmax warpgroup
+      mbar_init(bar(kODone + i), 1);    // commit after P V of the tile
     }
-    for (int x = 0; x < Cfg::kQT; ++x) mbar_init(bar(kODone + x), 1);  // commit after P V
     fence_barrier_init();
   }
   if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
@@ -356,7 +354,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     // A tcgen05.mma issue blocks while the tensor pipe's queue is full, so the
     // S and P V MMAs come from two warps: a ready P V never waits behind a
     // batch of S. Tile j + 2's S reuses the tensor-memory buffers of tile j once
-    // both P of tile j are published (their S was read).
+    // both P V of tile j are done: P is stored over the S it was computed from.
     constexpr uint32_t kIdS = tc::idesc_bf16_f32(128, KEYN, 0);  // B = K rows (K-major)
     auto issue_s = [&](int j) {  // S_x = Q_x K_j^T for both query tiles
       const uint32_t kb = k_s(j % NS);
@@ -376,7 +374,7 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     for (int j = 0; j < nt && ok; ++j) {
       if (j >= 2) {
         for (int x = 0; x < Cfg::kQT && ok; ++x)
-          ok = wait_all(bar(kPFull + 2 * x + (j & 1)), ((j - 2) >> 1) & 1);
+          ok = wait_all(bar(kODone + 2 * x + (j & 1)), ((j - 2) >> 1) & 1);
         if (!ok) break;
       }
       if (!wait_all(bar(kKVFull + j % NS), (j / NS) & 1)) break;
@@ -397,12 +395,13 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
         }
         tc::fence_after_sync();
         if (lane == 0) {
+          // A = P from tensor memory (16 keys = 8 columns per k-step)
 #pragma unroll
           for (int ks = 0; ks < KEYN / 16; ++ks)
-            tc::mma_bf16(t_o(x), tc::smem_desc_sw128(p_s(x) + ks * 32, 16, 1024),
-                         tc::smem_desc_sw128(vb + ks * 2048, KVHALF, 1024), kIdPV,
-                         j > 0 || ks > 0);
-          tc::commit(bar(kODone + x));
+            tc::mma_bf16_tmem_a(t_o(x), t_s(x, j & 1) + ks * 8,
+                                tc::smem_desc_sw128(vb + ks * 2048, KVHALF, 1024), kIdPV,
+                                j > 0 || ks > 0);
+          tc::commit(bar(kODone + 2 * x + (j & 1)));
         }
       }
       if (ok && lane == 0) tc::commit(bar(kKVEmpty + j % NS));  // V of tile j read
@@ -475,35 +474,34 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
       }
       l_run = l_run * alpha + (rs0 + rs1);
       m_use = m_new;
-      // the previous P V must be done before P is rewritten or O rescaled
-      if (j > 0) {
-        if (!wait_all(bar(kODone + x), (j - 1) & 1)) {
+      // The previous P V (tile j - 1) must be done before O is rescaled: wait
+      // for it here only when some row of this warp moved its reference;
+      // otherwise P is published first and the wait comes after, so this tile's
+      // P V can follow the previous one at once. Either way every tile waits
+      // once, before the next tile's P, which keeps this warp within one
+      // phase of the barrier pair.
+      const bool rescale = j > 0 && __any_sync(kFullMask, alpha != 1.0f);
+      if (rescale) {
+        if (!wait_all(bar(kODone + 2 * x + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        if (__any_sync(kFullMask, alpha != 1.0f)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t ov[32];
-            tc::ld32(t_o(x) + lane_off + c * 32, ov);
-            tc::wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          tc::ld32(t_o(x) + lane_off + c * 32, ov);
+          tc::wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tc::st32(t_o(x) + lane_off + c * 32, ov);
-          }
-          tc::wait_st();
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tc::st32(t_o(x) + lane_off + c * 32, ov);
         }
       }
-      // P into the swizzled K-major tile: 16-byte chunk cc of row r sits at
-      // r * 128 + ((cc ^ (r % 8)) * 16)
-#pragma unroll
-      for (int c8 = 0; c8 < KEYN / 8; ++c8) {
-        const uint32_t addr = p_s(x) + r * 128 + (((c8 & 7) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[4 * c8]),
-                     "r"(pw[4 * c8 + 1]), "r"(pw[4 * c8 + 2]), "r"(pw[4 * c8 + 3])
-                     : "memory");
-      }
+      // P (bf16 pairs, the lower key in the low half) over the first KEYN / 2
+      // columns of this tile's S, which this thread has read: the A operand of
+      // the P V MMA, from tensor memory
+      tc::st32(t_s(x, j & 1) + lane_off, pw);
+      tc::wait_st();
       if (x == 0 && j == nt - 1) {
         // keys past the context in the last tile: stale or unwritten V rows become
         // zeros (their P is 0, but 0 * NaN would not be); both P V of the tile
@@ -518,14 +516,20 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
                          "r"(0u)
                          : "memory");
           }
+          // generic-proxy writes before the MMA's async-proxy reads
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
       }
-      // generic-proxy writes (P, zeroed V) before the MMA's async-proxy reads
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc::fence_before_sync();
       mbar_arrive(bar(kPFull + 2 * x + (j & 1)));
+      if (j > 0 && !rescale) {
+        if (!wait_all(bar(kODone + 2 * x + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+      }
     }
-    if (PREFIX && ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
+    if (PREFIX && ok && wait_all(bar(kODone + 2 * x + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1)) {
       // the row's partial result over this key partition, for the decode merge
       tc::fence_after_sync();
       const int64_t row =
@@ -547,7 +551,8 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
                 make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
         }
       }
-    } else if (!PREFIX && ok && wait_all(bar(kODone + x), (nt - 1) & 1)) {
+    } else if (!PREFIX && ok &&
+               wait_all(bar(kODone + 2 * x + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1)) {
       tc::fence_after_sync();
       const float inv = 1.0f / l_run;
       __nv_bfloat16* dst = p.out + ((static_cast<int64_t>(q0) + tx0 + tok) * p.num_heads +

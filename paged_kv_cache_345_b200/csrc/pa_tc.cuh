@@ -60,6 +60,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// D (tensor memory) = A * B (+ D when `accumulate`), A from tensor memory:
+// row r of A in lane r, its K values two to a 32-bit column (the lower K index
+// in the low half), K / 2 columns from `a_tmem`; B from shared memory.
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // The mbarrier completes (one arrival) when every MMA issued so far by this
 // thread has finished.
 __device__ __forceinline__ void commit(uint32_t mbar) {
