@@ -188,22 +188,32 @@ unsigned int pa_set_decode_options(unsigned int options) {
   return old;
 }
 
-int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
-  // The bf16 kernel runs one CTA per (group of up to 4 KV heads, partition,
-  // sequence), two per SM. Aim for about three CTAs per SM if every sequence
-  // were as long as the longest, with partitions of 64..768 tokens: long
-  // enough to amortise a CTA's start-up, short enough to bound the tail
-  // (measured on the 256-sequence lognormal batch: 512 -> 82 %, 768 -> 84 %,
-  // 1024 -> 80 % of HBM bandwidth).
+namespace {
+// Partition length for about `ctas_per_sm` CTAs per SM if every sequence were
+// as long as max_context_len (one CTA per group of up to 4 KV heads,
+// partition and sequence), 64..768 tokens, a multiple of the chunk.
+int partition_for(int num_seqs, int num_kv_heads, int max_context_len, double ctas_per_sm) {
   const int groups = num_kv_heads % 4 == 0 ? num_kv_heads / 4
                      : num_kv_heads % 2 == 0 ? num_kv_heads / 2 : num_kv_heads;
   const double work = static_cast<double>(max_context_len) * (num_seqs > 0 ? num_seqs : 1) *
                       (groups > 0 ? groups : 1);
-  double p = std::ceil(work / (148.0 * 3.0));
+  double p = std::ceil(work / (148.0 * ctas_per_sm));
   if (p < 64) p = 64;
   if (p > 768) p = 768;
   const int c = pa::kChunkTokens;
   return (static_cast<int>(p) + c - 1) / c * c;
+}
+}  // namespace
+
+int pa_decode_partition_size(int num_seqs, int num_kv_heads, int max_context_len) {
+  // Two bf16 CTAs per SM are resident; aim for about five per SM over the
+  // launch, so that most sequences are shorter than the longest still leaves
+  // every SM a CTA (Llama-3-8B batch, 8 sequences up to 4,101 tokens: 96
+  // tokens 11.8 us per layer back to back, 160 tokens 12.4 us). Partitions
+  // of 64..768 tokens: long enough to amortise a CTA's start-up, short enough
+  // to bound the tail (256-sequence lognormal batch: 512 -> 82 %, 768 -> 84 %,
+  // 1024 -> 80 % of HBM bandwidth).
+  return partition_for(num_seqs, num_kv_heads, max_context_len, 5.0);
 }
 
 static int resolve_partitions(int max_context_len, int* partition_size) {
@@ -406,13 +416,9 @@ PrefixPlan plan_shared_prefix(int num_seqs, int num_heads, int num_kv_heads, int
   const int rest = max_context_len - prefix_len;
   if (partition_size == 0) {
     // the suffix decode runs on the SMs the prefix pass leaves and its end is
-    // the critical path: two thirds of the plain decode's partition, for a
-    // shorter tail (64 sequences, suffixes of 50..1000 tokens: 208 tokens
-    // 41.0 us a step, the plain choice 304 tokens 45.5 us)
-    const int c = pa::kChunkTokens;
-    const int plain = pa_decode_partition_size(num_seqs, num_kv_heads, rest > 0 ? rest : 0);
-    pl.suffix_part = ((plain * 2 / 3 + c - 1) / c) * c;
-    if (pl.suffix_part < 64) pl.suffix_part = 64;
+    // the critical path (64 sequences, suffixes of 50..1000 tokens: 208
+    // tokens 41.0 us a step, 176 42.6, 304 45.5)
+    pl.suffix_part = partition_for(num_seqs, num_kv_heads, rest > 0 ? rest : 0, 4.5);
   } else {
     pl.suffix_part = partition_size;
   }
