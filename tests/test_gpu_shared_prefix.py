@@ -58,6 +58,7 @@ def _custom(hq, hkv, bs, prefix, suffixes, seed):
 
 @pytest.mark.parametrize("hq,hkv,bs,prefix,nseq", [
     (8, 8, 16, 144, 5),      # group 1; a prefix that is not a multiple of 64 keys
+    (16, 8, 32, 320, 12),    # group 2, block 32
     (32, 8, 8, 512, 70),     # group 4, block 8, two pairs of query tiles (64 rows each)
     (16, 2, 64, 1024, 9),    # group 8, block 64
 ])
@@ -121,3 +122,43 @@ def test_context_shorter_than_the_prefix_is_flagged():
     # the sequence with a valid context is still right
     ref = gh.expected_all(case)
     gh.assert_close(out[0].float().cpu().numpy(), ref[0], "bf16", "valid row")
+
+
+def test_every_context_is_the_prefix():
+    """No sequence has tokens of its own (contexts of exactly the prefix, no
+    newest token to append): every CTA of the suffix decode leaves at once, and
+    the merge still waits for the prefix pass; each row is the attention over
+    the prefix alone."""
+    from oracle import attention as oatt
+
+    wl = _custom(32, 8, 16, 512, [0, 5, 9], 3)
+    case = gh.build_case(wl)
+    tables, lens, _ = case.cache.tables(case.seqs)
+    lens = torch.full_like(lens, 512)           # the same blocks, attended up to the prefix
+    q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(3, 32, 8, 128, 512, 512, 0),
+                     dtype=torch.uint8, device="cuda")
+    ws.fill_(0xFF)
+    out = torch.full_like(q, float("nan"))
+    pa.pa_decode_shared_prefix(out, q, None, None, case.cache.k_cache, case.cache.v_cache, tables,
+                               lens, 512, 512, wl.scale, 0, ws)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    got = out.float().cpu().numpy()
+    for s in range(3):
+        for j in range(32):
+            h = oatt.kv_head_of(j, 4)
+            ref = oatt.softmax_attention(case.q[s, j], case.rows_k[s][:512, h],
+                                         case.rows_v[s][:512, h], wl.scale)
+            gh.assert_close(got[s, j], ref, "bf16", f"seq {s} head {j}")
+
+
+def test_under_the_early_read_option():
+    """The cascade ignores PA_DECODE_EARLY_CACHE_READS: same result with it set."""
+    wl = _custom(32, 8, 16, 256, [3, 40, 17, 200], 4)
+    case = gh.build_case(wl)
+    plain = _shared_decode(case, 256, ps=64)
+    with pa.decode_options(pa.PA_DECODE_EARLY_CACHE_READS):
+        early = _shared_decode(case, 256, ps=64)
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(plain, early)
