@@ -162,3 +162,48 @@ def test_under_the_early_read_option():
         early = _shared_decode(case, 256, ps=64)
     assert pa.pa_device_errors() == 0
     assert torch.equal(plain, early)
+
+
+def test_graph_of_cascades_equals_eager():
+    """Three cascade calls (one per cache copy, as a model's layers) captured in
+    one CUDA graph: every replay equals the eager calls bit for bit."""
+    wl = configs.shared_prefix()
+    case = gh.build_case(wl)
+    prefix = (wl.shared_prefix // wl.block_size) * wl.block_size
+    tables, lens, max_len = case.cache.tables(case.seqs)
+    q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+    s, hq, d = q.shape
+    need = pa.pa_decode_shared_prefix_workspace_bytes(s, hq, wl.num_kv_heads, d, prefix, max_len, 0)
+    layers = []
+    for i in range(3):
+        k = case.cache.k_cache.clone()
+        k.mul_(1.0 + 0.5 * i)                    # every layer different
+        layers.append((k, case.cache.v_cache.clone(), torch.empty_like(q),
+                       torch.empty(need, dtype=torch.uint8, device="cuda")))
+    ref = []
+    for k, v, _, ws in layers:
+        o = torch.empty_like(q)
+        pa.pa_decode_shared_prefix(o, q, None, None, k, v, tables, lens, prefix, max_len,
+                                   wl.scale, 0, ws)
+        ref.append(o)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for k, v, o, ws in layers:
+            pa.pa_decode_shared_prefix(o, q, None, None, k, v, tables, lens, prefix, max_len,
+                                       wl.scale, 0, ws)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for k, v, o, ws in layers:
+                pa.pa_decode_shared_prefix(o, q, None, None, k, v, tables, lens, prefix,
+                                           max_len, wl.scale, 0, ws)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for _, _, o, _ in layers:
+            o.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        for (_, _, o, _), r in zip(layers, ref):
+            assert torch.equal(o, r)
+    assert pa.pa_device_errors() == 0
+    del graph
