@@ -139,8 +139,9 @@ def whole_job_rate(units_per_step: float, steps: int, world: int, time_ms: float
 
 # ------------------------------------------------------------------ GPU setup
 
-def build_on_gpu(wl, device, placement="random"):
-    """Prefill every sequence through the library, then prepare one decode step."""
+def build_on_gpu(wl, device, placement="random", extra_tokens=0):
+    """Prefill every sequence through the library, then prepare one decode step.
+    extra_tokens: room in the block tables for that many more decode steps."""
     import torch
 
     from paged_kv_cache_345_b200.cache import PagedKVCache
@@ -148,7 +149,7 @@ def build_on_gpu(wl, device, placement="random"):
 
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     bs = wl.block_size
-    max_blocks = max(-(-(n + 1) // bs) for n in wl.context_lens)
+    max_blocks = max(-(-(n + 1 + extra_tokens) // bs) for n in wl.context_lens)
     order = synth.block_permutation(wl.num_blocks, wl.placement_seed) if placement == "random" \
         else np.arange(wl.num_blocks, dtype=np.int32)
     fp8 = wl.cache_dtype == "fp8_e4m3"
@@ -743,7 +744,9 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
     import torch
 
     wl2 = make_workload(name, 16)
-    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl2, device)
+    steps_after = 10 if name == "large_batch" else 0
+    cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl2, device,
+                                                              extra_tokens=steps_after)
     ps = TUNED_PARTITION[wl2.name.split("_bs")[0]]
     calls = StepCalls(cache, dev, max_len, wl2.scale, ps, stream)
     clocks = ClockSampler(device.index or 0)
@@ -763,6 +766,9 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
         res["kv_bytes_logical"] = logical
         res["GB_per_s_logical"] = logical / mean_s / 1e9
         res["copy_on_write_pairs"] = cow_pairs
+    if steps_after:
+        res["ten_steps"] = serving_steps(cache, seqs, host, dev, max_len, wl2, stream,
+                                         steps_after)
     if wl2.shared_prefix:
         # the same step through the cascade entry point: the shared blocks read
         # once for the whole batch
@@ -785,6 +791,72 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
     del calls, cache, dev, host
     torch.cuda.empty_cache()
     return res
+
+
+def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
+    """`steps` decode steps of a serving loop after the timed step above: per
+    step, the host block manager's step through the C ABI (the next slot of
+    every sequence, a new block where the tail is full, the copy-on-write
+    check, the new tables), its output (slots, tables, lengths) host -> device
+    in one copy, and the fused append + decode. q and the new K/V rows are the
+    previous layer's output in a model, so they are staged on the device
+    beforehand (one set per step, each step's call reading its own). Contexts grow by one token a step. Host
+    time by perf_counter, device time (the copy + the kernels) by CUDA events."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+    from workloads import synth
+
+    s = len(seqs)
+    mbps = dev["tables"].shape[1]
+    tdt = dev["q"].dtype
+    staged = [(torch.from_numpy(synth.queries(wl.value_seed, 100 + i, s, wl.num_heads,
+                                              wl.head_dim)).to(dev["q"].device, tdt),
+               *[torch.from_numpy(a).to(dev["q"].device, tdt) for a in
+                 synth.new_token_kv(wl.value_seed, 100 + i, s, wl.num_kv_heads, wl.head_dim)])
+              for i in range(steps)]
+    # one marshalled call per step, reading that step's staged q and rows
+    calls = [StepCalls(cache, dict(dev, q=q, k_new=k, v_new=v), max_len + steps, wl.scale, 0,
+                       stream) for q, k, v in staged]
+    # the block manager's part of the packed inputs: slots, tables, lengths (contiguous)
+    lo = dev["slots"].data_ptr() - dev["_pack"].data_ptr()
+    hi = dev["lens"].data_ptr() + dev["lens"].numel() * 4 - dev["_pack"].data_ptr()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    host_us, bytes_step, new_blocks = [], [], 0
+    torch.cuda.synchronize()
+    for i in range(steps):
+        free_before = cache.bm.allocator.num_free()
+        t0 = time.perf_counter()
+        slots, cows = cache.bm.append_slots(seqs, [1] * s)
+        tables, lens = cache.bm.block_tables(seqs, mbps)
+        host_us.append(1e6 * (time.perf_counter() - t0))
+        new_blocks += free_before - cache.bm.allocator.num_free()
+        if len(cows):
+            pa.pa_copy_blocks(cache.k_cache, cache.v_cache, torch.from_numpy(cows).to(dev["q"].device))
+        host["slots"].copy_(torch.from_numpy(slots))
+        host["tables"].copy_(torch.from_numpy(tables))
+        host["lens"].copy_(torch.from_numpy(lens))
+        bytes_step.append(int(lens.astype(np.int64).sum()) * wl.num_kv_heads * 2 * wl.head_dim *
+                          wl.cache_elem_bytes)
+        ev[i][0].record(stream)
+        dev["_pack"][lo:hi].copy_(host["_pack"][lo:hi], non_blocking=True)
+        calls[i].step()
+        ev[i][1].record(stream)
+        stream.synchronize()
+    dev_us = [1e3 * a.elapsed_time(b) for a, b in ev]
+    pa_device_errors_or_raise()
+    return {"steps": steps, "host_block_manager_us": [round(x, 1) for x in host_us],
+            "device_us": [round(x, 2) for x in dev_us], "h2d_bytes_per_step": hi - lo,
+            "mean_host_us": statistics.mean(host_us), "mean_device_us": statistics.mean(dev_us),
+            "median_host_us": statistics.median(host_us),
+            "median_device_us": statistics.median(dev_us),
+            "mean_kv_GB_per_s": statistics.mean(b / (u * 1e-6) / 1e9
+                                                for b, u in zip(bytes_step, dev_us)),
+            "new_blocks": new_blocks,
+            "how": "per step: pa_bm_append_slots + pa_bm_block_tables (host, C ABI through the "
+                   "binding); slots, tables and lengths host -> device in one copy; "
+                   "pa_decode_append on q and new rows staged on the device (a model's "
+                   "previous layer makes them); no L2 flush (the cache is 0.63 GB)"}
 
 
 def pa_device_errors_or_raise():
