@@ -14,7 +14,10 @@ workspace. Each method marshals arguments and calls libpa.so:
   decode_step(q, k_new, v_new, seq_ids)  one decode step: reserve each sequence's
       next slot (native; shared tail blocks copied first), then pa_decode_append
       writes the new K/V rows and attends in one launch (fused=False: separate
-      pa_kv_append and pa_decode calls, same result).
+      pa_kv_append and pa_decode calls, same result). shared_prefix=n: the
+      sequences' first n tokens (a multiple of the block size) sit in the same
+      blocks (forked from one parent): pa_decode_shared_prefix attends them once
+      for the batch, beside the decode of each sequence's own tokens; bf16.
 
 dtype "fp8_e4m3": the caches hold uint8 E4M3 codes with one float32 scale per
 KV head (k_scale, v_scale); rows come in as bfloat16 and are quantised on the
@@ -34,7 +37,8 @@ import numpy as np
 import torch
 
 from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_decode_append_fp8,
-               pa_decode_fp8, pa_decode_partition_size, pa_decode_workspace_bytes, pa_kv_append,
+               pa_decode_fp8, pa_decode_partition_size, pa_decode_shared_prefix,
+               pa_decode_shared_prefix_workspace_bytes, pa_decode_workspace_bytes, pa_kv_append,
                pa_kv_append_fp8, pa_prefill)
 
 _TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}
@@ -136,6 +140,25 @@ class PagedKVCache:
         return self._to_device(tables), self._to_device(lens), int(lens.max(initial=0))
 
     @_on_stream
+    def _decode_step_shared(self, q, k_new, v_new, seq_ids, scale, partition_size, out,
+                            prefix_len):
+        _, cows = self.bm.append_slots(seq_ids, [1] * len(seq_ids))
+        if len(cows):
+            pa_copy_blocks(self.k_cache, self.v_cache, self._to_device(cows), stream=self.stream)
+        num_seqs, num_heads, _ = q.shape
+        block_tables, context_lens, max_len = self.tables(seq_ids)
+        out = torch.empty_like(q) if out is None else out
+        scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+        need = pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, self.num_kv_heads,
+                                                       self.head_dim, prefix_len, max_len,
+                                                       partition_size)
+        if need > self._workspace.numel():
+            self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+        pa_decode_shared_prefix(out, q, k_new, v_new, self.k_cache, self.v_cache, block_tables,
+                                context_lens, prefix_len, max_len, scale, partition_size,
+                                self._workspace, stream=self.stream)
+        return out
+
     def workspace(self, num_seqs, num_heads, max_context_len, partition_size=0):
         need = pa_decode_workspace_bytes(num_seqs, num_heads, self.num_kv_heads, self.head_dim,
                                          max_context_len, partition_size)
@@ -163,7 +186,12 @@ class PagedKVCache:
 
     @_on_stream
     def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
-                    out=None, fused: bool = True):
+                    out=None, fused: bool = True, shared_prefix: int = 0):
+        if shared_prefix:
+            if self.fp8 or not fused:
+                raise ValueError("shared_prefix: a bf16 cache and the fused step")
+            return self._decode_step_shared(q, k_new, v_new, seq_ids, scale, partition_size, out,
+                                            shared_prefix)
         if not fused:
             self.write(seq_ids, [1] * len(seq_ids), k_new, v_new)
             return self.decode(q, seq_ids, scale, partition_size, out)

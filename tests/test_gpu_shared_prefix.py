@@ -207,3 +207,40 @@ def test_graph_of_cascades_equals_eager():
             assert torch.equal(o, r)
     assert pa.pa_device_errors() == 0
     del graph
+
+
+def _forked_cache(seed):
+    from paged_kv_cache_345_b200.cache import PagedKVCache
+    from workloads import synth
+
+    cache = PagedKVCache(96, 16, 8, 128, "bf16", "cuda", max_blocks_per_seq=32,
+                         free_order=synth.block_permutation(96, seed))
+    root = cache.add_sequence()
+    k, v = synth.kv_rows(seed, 0, 64, 8, 128)
+    to = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)  # noqa: E731
+    cache.write([root], [64], to(k), to(v))
+    seqs = [root] + [cache.fork(root) for _ in range(3)]
+    for i, (sq, n) in enumerate(zip(seqs, [7, 30, 0, 91])):
+        if n:
+            k, v = synth.kv_rows(seed, 1 + i, n, 8, 128)
+            cache.write([sq], [n], to(k), to(v))
+    return cache, seqs
+
+
+def test_cache_decode_step_with_shared_prefix():
+    """PagedKVCache.decode_step(shared_prefix=64) against the plain fused step
+    on an identical cache: same cache contents after the step, outputs within
+    the bf16 tolerance of each other."""
+    from workloads import synth
+
+    a, sa = _forked_cache(77)
+    b, sb = _forked_cache(77)
+    q = torch.from_numpy(synth.queries(77, 9, 4, 32, 128)).cuda().to(torch.bfloat16)
+    kn, vn = [torch.from_numpy(x).cuda().to(torch.bfloat16)
+              for x in synth.new_token_kv(77, 9, 4, 8, 128)]
+    out_a = a.decode_step(q, kn, vn, sa, shared_prefix=64)
+    out_b = b.decode_step(q, kn, vn, sb)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    assert torch.equal(a.k_cache, b.k_cache) and torch.equal(a.v_cache, b.v_cache)
+    gh.assert_close(out_a.float().cpu().numpy(), out_b.float().cpu().numpy(), "bf16", "step")
