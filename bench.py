@@ -653,11 +653,22 @@ def host_allocator_metrics(steps: int = 10):
         slots, cows = bm.append_slots(seqs, ones)
         tables, lens = bm.block_tables(seqs, mb)
         times.append(time.perf_counter() - t0)
-    # the same step called through the C ABI with preallocated buffers (what a
-    # native caller pays): 10 more steps
+    # through the binding with the caller's buffers (no allocation per step)
     ids = np.asarray(seqs, dtype=np.int32)
     cnt = np.ones(len(seqs), dtype=np.int32)
-    mb2 = mb + steps // wl.block_size + 1
+    mb2 = mb + 2 * steps // wl.block_size + 2
+    b_slots = np.empty(len(seqs), dtype=np.int64)
+    b_cows = np.empty((len(seqs), 2), dtype=np.int64)
+    b_tabs = np.empty(len(seqs) * mb2, dtype=np.int32)
+    b_lens = np.empty(len(seqs), dtype=np.int32)
+    b_times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        bm.append_slots(ids, cnt, b_slots, b_cows)
+        bm.block_tables(ids, mb2, b_tabs, b_lens)
+        b_times.append(time.perf_counter() - t0)
+    # the same step called through the C ABI with preallocated buffers (what a
+    # native caller pays): 10 more steps
     slot_buf = np.empty(len(seqs), dtype=np.int64)
     cow_buf = np.empty((len(seqs), 2), dtype=np.int64)
     tab_buf = np.empty((len(seqs), mb2), dtype=np.int32)
@@ -697,12 +708,14 @@ def host_allocator_metrics(steps: int = 10):
         "allocator_step": {
             "us_per_step_mean": 1e6 * statistics.mean(times),
             "us_per_step_p50": 1e6 * statistics.median(times),
+            "us_per_step_buffers_p50": 1e6 * statistics.median(b_times),
             "us_per_step_c_abi_p50": 1e6 * statistics.median(c_times),
-            "sequences": len(seqs), "steps": 2 * steps, "new_blocks": int(new_blocks),
+            "sequences": len(seqs), "steps": 3 * steps, "new_blocks": int(new_blocks),
             "what": "pa_bm_append_slots (slot, new block when the tail is full, copy-on-write "
                     "check) + pa_bm_block_tables: the first figures through the Python binding "
-                    "(10 steps), the c_abi one through ctypes with preallocated buffers (10 "
-                    "more steps)",
+                    "with Python lists (10 steps), the buffers one through the binding with "
+                    "the caller's arrays (10 more), the c_abi one through ctypes with "
+                    "preallocated buffers (10 more)",
             "utilisation_after": tokens / (held * wl.block_size)},
         "cache_utilisation": {
             "workload": "worked example (8 requests, block 16)",
@@ -823,19 +836,21 @@ def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
     hi = dev["lens"].data_ptr() + dev["lens"].numel() * 4 - dev["_pack"].data_ptr()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     host_us, bytes_step, new_blocks = [], [], 0
+    # the block manager writes straight into the pinned pack (no allocation per step)
+    ids, ones = np.asarray(seqs, dtype=np.int32), np.ones(s, dtype=np.int32)
+    slot_buf, tab_buf, len_buf = (host["slots"].numpy(), host["tables"].numpy(),
+                                  host["lens"].numpy())
+    cow_buf = np.empty((s, 2), dtype=np.int64)
     torch.cuda.synchronize()
     for i in range(steps):
         free_before = cache.bm.allocator.num_free()
         t0 = time.perf_counter()
-        slots, cows = cache.bm.append_slots(seqs, [1] * s)
-        tables, lens = cache.bm.block_tables(seqs, mbps)
+        slots, cows = cache.bm.append_slots(ids, ones, slot_buf, cow_buf)
+        tables, lens = cache.bm.block_tables(ids, mbps, tab_buf, len_buf)
         host_us.append(1e6 * (time.perf_counter() - t0))
         new_blocks += free_before - cache.bm.allocator.num_free()
         if len(cows):
             pa.pa_copy_blocks(cache.k_cache, cache.v_cache, torch.from_numpy(cows).to(dev["q"].device))
-        host["slots"].copy_(torch.from_numpy(slots))
-        host["tables"].copy_(torch.from_numpy(tables))
-        host["lens"].copy_(torch.from_numpy(lens))
         bytes_step.append(int(lens.astype(np.int64).sum()) * wl.num_kv_heads * 2 * wl.head_dim *
                           wl.cache_elem_bytes)
         ev[i][0].record(stream)
@@ -853,8 +868,9 @@ def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
             "mean_kv_GB_per_s": statistics.mean(b / (u * 1e-6) / 1e9
                                                 for b, u in zip(bytes_step, dev_us)),
             "new_blocks": new_blocks,
-            "how": "per step: pa_bm_append_slots + pa_bm_block_tables (host, C ABI through the "
-                   "binding); slots, tables and lengths host -> device in one copy; "
+            "how": "per step: pa_bm_append_slots + pa_bm_block_tables (host, through the "
+                   "binding, written straight into the pinned input pack); slots, tables and "
+                   "lengths host -> device in one copy; "
                    "pa_decode_append on q and new rows staged on the device (a model's "
                    "previous layer makes them); no L2 flush (the cache is 0.63 GB)"}
 

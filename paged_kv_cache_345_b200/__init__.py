@@ -562,6 +562,16 @@ def _i32_array(x):
     return a, a.ctypes.data_as(_i32p)
 
 
+def _out_array(a, dtype, need, name):
+    """A caller's output buffer, checked: a C-contiguous numpy array of `dtype`
+    with at least `need` elements; returned flattened (a view, no copy)."""
+    if not isinstance(a, np.ndarray) or a.dtype != dtype or not a.flags.c_contiguous:
+        raise ValueError(f"{name} must be a C-contiguous numpy {np.dtype(dtype).name} array")
+    if a.size < need:
+        raise ValueError(f"{name} holds {a.size} elements, {need} needed")
+    return a.reshape(-1)
+
+
 class Allocator:
     """Free list + reference counts of a block pool (pa_alloc_*).
 
@@ -647,25 +657,41 @@ class BlockManager:
     def seq_num_blocks(self, seq: int) -> int:
         return int(_lib.pa_bm_seq_num_blocks(self._h, seq))
 
-    def append_slots(self, seq_ids, counts):
-        """Reserve slots; returns (slot_mapping int64 [sum(counts)], cow_pairs int64 [k, 2])."""
+    def append_slots(self, seq_ids, counts, slots_out=None, cows_out=None):
+        """Reserve slots; returns (slot_mapping int64 [sum(counts)], cow_pairs int64 [k, 2]).
+
+        slots_out (int64, >= sum(counts) elements) and cows_out (int64 [>= n, 2],
+        n = len(seq_ids)), both C-contiguous, are written in place and views of
+        them returned: a serving loop then allocates nothing per step."""
         ids, pids = _i32_array(seq_ids)
         cnt, pcnt = _i32_array(counts)
         if ids.shape != cnt.shape:
             raise ValueError("seq_ids and counts differ in length")
-        slots = np.empty(int(cnt.sum()), dtype=np.int64)
-        cows = np.empty((max(ids.size, 1), 2), dtype=np.int64)
+        total = int(cnt.sum())
+        slots = np.empty(total, dtype=np.int64) if slots_out is None else \
+            _out_array(slots_out, np.int64, total, "slots_out")
+        cows = np.empty((max(ids.size, 1), 2), dtype=np.int64) if cows_out is None else \
+            _out_array(cows_out, np.int64, 2 * max(ids.size, 1), "cows_out").reshape(-1, 2)
         ncow = ctypes.c_int(0)
         _check(_lib.pa_bm_append_slots(self._h, pids, pcnt, ids.size,
                                        slots.ctypes.data_as(_i64p), cows.ctypes.data_as(_i64p),
                                        cows.shape[0], ctypes.byref(ncow)))
+        if slots_out is not None:
+            return slots[:total], cows[:ncow.value]
         return slots, cows[:ncow.value].copy()
 
-    def block_tables(self, seq_ids, max_blocks_per_seq: int):
-        """(tables int32 [n, max_blocks_per_seq], context_lens int32 [n]) for the sequences."""
+    def block_tables(self, seq_ids, max_blocks_per_seq: int, tables_out=None, lens_out=None):
+        """(tables int32 [n, max_blocks_per_seq], context_lens int32 [n]) for the sequences.
+
+        tables_out / lens_out (int32, C-contiguous, n * max_blocks_per_seq and n
+        elements at least) are written in place and views of them returned."""
         ids, pids = _i32_array(seq_ids)
-        tables = np.empty((ids.size, max_blocks_per_seq), dtype=np.int32)
-        lens = np.empty(ids.size, dtype=np.int32)
-        _check(_lib.pa_bm_block_tables(self._h, pids, ids.size, tables.ctypes.data_as(_i32p),
+        n = ids.size
+        tables = np.empty((n, max_blocks_per_seq), dtype=np.int32) if tables_out is None else \
+            _out_array(tables_out, np.int32, n * max_blocks_per_seq,
+                       "tables_out")[:n * max_blocks_per_seq].reshape(n, max_blocks_per_seq)
+        lens = np.empty(n, dtype=np.int32) if lens_out is None else \
+            _out_array(lens_out, np.int32, n, "lens_out")[:n]
+        _check(_lib.pa_bm_block_tables(self._h, pids, n, tables.ctypes.data_as(_i32p),
                                        max_blocks_per_seq, lens.ctypes.data_as(_i32p)))
         return tables, lens

@@ -133,3 +133,39 @@ def test_unfused_step_writes_then_decodes(rec):
     slots, _ = ref.add_tokens(r0, 1)
     assert [n for n, _ in rec] == ["pa_kv_append", "pa_decode"]
     assert rec[0][1][2].tolist() == slots and rec[1][1][5].tolist() == [5]
+
+
+def test_block_manager_output_buffers():
+    """append_slots / block_tables into caller buffers give what the allocating
+    calls give, on two identical managers, including a copy-on-write step."""
+    import numpy as np
+
+    import paged_kv_cache_345_b200 as pa
+
+    def make():
+        bm = pa.BlockManager(200, 16)
+        seqs = [bm.add_seq() for _ in range(5)]
+        bm.append_slots(seqs, [3, 16, 17, 40, 1])
+        seqs.append(bm.fork(seqs[2]))            # shares a partly filled tail
+        return bm, seqs
+
+    a, sa = make()
+    b, sb = make()
+    slot_buf = np.full(32, -7, np.int64)
+    cow_buf = np.full((8, 2), -7, np.int64)
+    tab_buf = np.full(64, -7, np.int32)
+    len_buf = np.full(8, -7, np.int32)
+    for step in range(3):
+        s1, c1 = a.append_slots(sa, [1] * len(sa))
+        t1, l1 = a.block_tables(sa, 5)
+        s2, c2 = b.append_slots(sb, np.ones(len(sb), np.int32), slot_buf, cow_buf)
+        t2, l2 = b.block_tables(sb, 5, tab_buf, len_buf)
+        assert np.array_equal(s1, s2) and np.array_equal(c1, c2)
+        assert np.array_equal(t1, t2) and np.array_equal(l1, l2)
+        assert np.shares_memory(s2, slot_buf) and np.shares_memory(t2, tab_buf)
+        if step == 0:
+            assert len(c2) == 1                  # the fork's shared tail copied once
+    with pytest.raises(ValueError):
+        b.append_slots(sb, [1] * len(sb), np.empty(2, np.int64))
+    with pytest.raises(ValueError):
+        b.block_tables(sb, 5, np.empty(64, np.int64))
