@@ -112,7 +112,13 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
                                              ~uintptr_t(127));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);  // full[NS], empty[NS]
 
-  const int hg = blockIdx.x, part = blockIdx.y, s = blockIdx.z;
+  // grid (head group, partition, sequence); E4M3: (head group, sequence,
+  // partition) with the highest partition first, so that the long sequences'
+  // full later partitions start before the many short first ones (the E4M3
+  // kernel's CTAs are slower per byte, and its tail was the longer)
+  const int hg = blockIdx.x;
+  const int part = FP8 ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.y);
+  const int s = FP8 ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = p.partition_size, bs = p.block_size, lg = p.log2_block_size;
   const int rows_per_box = (!TABLE || bs >= C) ? C : bs;
@@ -226,7 +232,10 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
     }
     return;
   }
-  if (t0 >= L) return;
+  if (t0 >= L) {
+    if (gate && threadIdx.x == 0) pdl_wait();
+    return;
+  }
   const int t1 = min(t0 + P, L);
   const int nchunks = (t1 - t0 + C - 1) / C;
   __syncthreads();

@@ -428,8 +428,11 @@ cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
   const int rows = (sh.contiguous || sh.block_size >= Cfg::kC) ? Cfg::kC : sh.block_size;
   if ((e = encode_group_map(&kmap, k_cache, sh, rows, HB)) != cudaSuccess) return e;
   if ((e = encode_group_map(&vmap, v_cache, sh, rows, HB)) != cudaSuccess) return e;
-  // (a shared-prefix call's own partitions follow the prefix's slots)
-  dim3 grid(sh.num_kv_heads / HB, sh.num_partitions - sh.prefix_slots, sh.num_seqs);
+  // (a shared-prefix call's own partitions follow the prefix's slots; E4M3:
+  // partitions slowest, see the kernel)
+  const unsigned parts = static_cast<unsigned>(sh.num_partitions - sh.prefix_slots);
+  const dim3 grid = FP8 ? dim3(sh.num_kv_heads / HB, sh.num_seqs, parts)
+                        : dim3(sh.num_kv_heads / HB, parts, sh.num_seqs);
   e = launch_pdl(kernel, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, kmap, vmap, p);
   if (e != cudaSuccess) return e;
   return launch_merge<__nv_bfloat16, D>(sh, p, stream);
