@@ -410,6 +410,38 @@ namespace {
 struct PrefixPlan {
   int suffix_part, suffix_parts, prefix_part, prefix_parts;
 };
+
+// Keys per partition of the prefix pass. Its CTAs (one per SM: KV heads x
+// pairs of 128-row query tiles x key partitions) run beside the suffix
+// decode, which takes the other SMs. Beside a decode that keeps HBM busy a CTA
+// costs about kStartUs + (its key tiles) * kTileUs (4, 8, 16 tiles of 256
+// query rows: 17, 20, 35 us); the decode about its bytes, sequences' own
+// tokens taken as half the longest, at kDecodeBytesPerUs (measured beside the
+// pass: the 64-sequence workload's estimate of 131 MB took ~30 us). Take the
+// fewest partitions whose CTAs end within that estimate, at most a quarter of
+// the SMs (that workload: 2 / 3 / 4 / 5 / 6 / 8 partitions gave 43.9 / 40.1 /
+// 40.9 / 42.0 / 42.0 / 43.9 us a step; the rule takes 3).
+int prefix_partition_keys(int num_seqs, int num_heads, int num_kv_heads, int prefix_len,
+                          int max_context_len) {
+  constexpr double kStartUs = 10.0, kTileUs = 1.6, kDecodeBytesPerUs = 4.4e6;
+  constexpr int kTile = pa::kPrefillKeyTile;
+  const int tok = 2 * (128 / (num_heads / num_kv_heads));  // query tokens per CTA
+  const int64_t pairs = (static_cast<int64_t>(num_seqs) + tok - 1) / tok;
+  const int64_t base = static_cast<int64_t>(num_kv_heads) * pairs;
+  const int64_t tiles = (prefix_len + kTile - 1) / kTile;
+  const int64_t rest = max_context_len > prefix_len ? max_context_len - prefix_len : 0;
+  const double decode_us = static_cast<double>(num_seqs) * num_kv_heads * rest * 0.5 * 512.0 /
+                           kDecodeBytesPerUs;
+  int64_t max_parts = 37 / base;
+  if (max_parts < 1) max_parts = 1;
+  if (max_parts > tiles) max_parts = tiles;
+  int64_t parts = 1;
+  while (parts < max_parts &&
+         kStartUs + static_cast<double>((tiles + parts - 1) / parts) * kTileUs > decode_us)
+    ++parts;
+  return static_cast<int>(((tiles + parts - 1) / parts) * kTile);
+}
+
 PrefixPlan plan_shared_prefix(int num_seqs, int num_heads, int num_kv_heads, int prefix_len,
                               int max_context_len, int partition_size) {
   PrefixPlan pl{};
@@ -424,7 +456,7 @@ PrefixPlan plan_shared_prefix(int num_seqs, int num_heads, int num_kv_heads, int
   }
   pl.suffix_parts = rest <= 0 ? 1 : (rest + pl.suffix_part - 1) / pl.suffix_part;
   pl.prefix_part =
-      pa::prefix_partition_keys(num_seqs, num_heads, num_kv_heads, prefix_len, max_context_len);
+      prefix_partition_keys(num_seqs, num_heads, num_kv_heads, prefix_len, max_context_len);
   pl.prefix_parts = (prefix_len + pl.prefix_part - 1) / pl.prefix_part;
   return pl;
 }

@@ -92,12 +92,9 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
 // queries q [num_seqs][num_heads][128] (bf16) attend keys [0, prefix_len) read
 // through the first row of block_tables, on the tcgen05 tensor cores, in
 // partitions of prefix_part keys (a multiple of 64); partition k of row r is
-// written to the decode workspace as slot k (ws_slots slots per row). The
-// pass runs beside the decode of the sequences' own tokens (at most
-// max_context_len - prefix_len each): prefix_partition_keys picks partitions
-// long enough to keep it on few SMs, short enough to end before that decode.
-int prefix_partition_keys(int num_seqs, int num_heads, int num_kv_heads, int prefix_len,
-                          int max_context_len);
+// written to the decode workspace as slot k (ws_slots slots per row).
+// Partitions are whole key tiles of the pass.
+constexpr int kPrefillKeyTile = 64;
 cudaError_t launch_prefix_attention(int num_seqs, int num_heads, int num_kv_heads, int block_size,
                                     int num_blocks, int max_blocks_per_seq, int prefix_len,
                                     int prefix_part, float scale, const void* q,

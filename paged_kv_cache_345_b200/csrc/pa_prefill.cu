@@ -97,6 +97,7 @@ struct PrefillConfig {
   static constexpr int kThreads = 352;
   static constexpr uint32_t kTmemCols = 512;  // S[x][2] (64 each; P over its first 32), O[x] (128 each)
   static_assert(kRows % G == 0, "group must divide the row tile");
+  static_assert(kKeys == kPrefillKeyTile, "prefix partitions are whole key tiles");
 };
 
 // mbarrier slots
@@ -713,33 +714,6 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
   const int tok = 2 * (128 / (sh.num_heads / sh.num_kv_heads));  // query tokens per CTA
   const int64_t items = static_cast<int64_t>(sh.num_seqs) * ((sh.max_query_len + tok - 1) / tok);
   return dispatch_prefill<false>(p, q, k_cache, v_cache, items * sh.num_kv_heads, stream);
-}
-
-int prefix_partition_keys(int num_seqs, int num_heads, int num_kv_heads, int prefix_len,
-                          int max_context_len) {
-  // One CTA per SM (KV heads x query-tile pairs x key partitions) runs beside
-  // the suffix decode, which takes the other SMs. Beside a decode that keeps
-  // HBM busy a CTA costs about kStartUs + (its 64-key tiles) * kTileUs
-  // (measured: 4, 8, 16 tiles of 256 query rows in 17, 20, 35 us); the decode
-  // about its K/V bytes (sequences' own tokens taken as half the longest) at
-  // kDecodeBytesPerUs. Take the fewest partitions whose CTAs end within that
-  // estimate, and no more CTAs than a quarter of the SMs.
-  constexpr double kStartUs = 10.0, kTileUs = 1.6, kDecodeBytesPerUs = 5.0e6;
-  const int tok = 2 * (128 / (num_heads / num_kv_heads));
-  const int64_t pairs = (static_cast<int64_t>(num_seqs) + tok - 1) / tok;
-  const int64_t base = static_cast<int64_t>(num_kv_heads) * pairs;
-  const int64_t tiles = (prefix_len + 63) / 64;
-  const int64_t rest = max_context_len > prefix_len ? max_context_len - prefix_len : 0;
-  const double decode_us = static_cast<double>(num_seqs) * num_kv_heads * rest * 0.5 * 512.0 /
-                           kDecodeBytesPerUs;
-  int64_t max_parts = 37 / base;
-  if (max_parts < 1) max_parts = 1;
-  if (max_parts > tiles) max_parts = tiles;
-  int64_t parts = 1;
-  while (parts < max_parts &&
-         kStartUs + static_cast<double>((tiles + parts - 1) / parts) * kTileUs > decode_us)
-    ++parts;
-  return static_cast<int>(((tiles + parts - 1) / parts) * 64);
 }
 
 cudaError_t launch_prefix_attention(int num_seqs, int num_heads, int num_kv_heads, int block_size,
