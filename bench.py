@@ -57,6 +57,9 @@ def parse_args():
                     help="cache element type (fp8_e4m3: 8-bit codes, per-KV-head scales)")
     ap.add_argument("--partition-size", type=int, default=-1,
                     help="tokens per split-K partition (-1: tuned default, 0: library choice)")
+    ap.add_argument("--unplanned", action="store_true",
+                    help="decode on the (partition, sequence) grid up to the longest context "
+                         "instead of a pa_decode_plan work list")
     ap.add_argument("--unfused", action="store_true",
                     help="time pa_kv_append + pa_decode instead of the fused pa_decode_append")
     ap.add_argument("--cascade", action="store_true",
@@ -236,16 +239,40 @@ def pack_step_inputs(arrays, device):
     return host, dev
 
 
+def plan_inputs(host, dev, partition_size, capacity_len=0):
+    """The packed step inputs with the decode work list added: pa_decode_plan of
+    the host lengths for this partition size, in room for every item a context
+    of up to capacity_len tokens (default: the longest now) could need. Returns
+    (host, dev, num_items); the device pack then carries the list with the
+    other inputs, in the same one copy."""
+    import torch
+
+    import paged_kv_cache_345_b200 as pa
+
+    lens = host["lens"].numpy()
+    cap_len = max(int(capacity_len), int(lens.max(initial=0)))
+    cap = max(1, lens.size * max(1, -(-cap_len // partition_size)))
+    work = np.zeros((cap, 2), dtype=np.int32)
+    n = len(pa.pa_decode_plan(lens, partition_size, out=work))
+    arrays = {k: v for k, v in host.items() if k != "_pack"}
+    arrays["work"] = torch.from_numpy(work)
+    host2, dev2 = pack_step_inputs(arrays, dev["_pack"].device)
+    return host2, dev2, n
+
+
 class StepCalls:
     """The C-ABI calls of one decode step with their arguments marshalled once.
 
     fused: the step is one pa_decode_append call (append each newest token, then
     attend); otherwise pa_kv_append followed by pa_decode (same result).
+    num_items > 0 (with dev["work"], a plan_inputs pack; bf16 and E4M3 caches):
+    the decode runs on the work list's grid through pa_decode_planned (same
+    result, no CTAs for partitions past a sequence's end).
     prefix_len > 0: the step is one pa_decode_shared_prefix call with the append
     (every sequence's first prefix_len tokens in the same blocks)."""
 
     def __init__(self, cache, dev, max_len, scale, partition_size, stream, fused=True,
-                 prefix_len=0):
+                 prefix_len=0, num_items=0):
         import torch
 
         import paged_kv_cache_345_b200 as pa
@@ -293,6 +320,22 @@ class StepCalls:
                               p(dev["lens"]), s, hq, hkv, d, bs, nb, mbps, max_len, scale,
                               self.partition_size, *ws, dt, st)
             self.fns = (self.lib.pa_kv_append, self.lib.pa_decode, self.lib.pa_decode_append)
+        self.planned = bool(num_items) and "work" in dev and not prefix_len and \
+            cache.k_cache.dtype in (torch.bfloat16, torch.uint8)
+        if self.planned:
+            sc = (p(cache.k_scale), p(cache.v_scale)) if self.fp8 else (None, None)
+            dcode = pa.PA_FP8_E4M3 if self.fp8 else pa.PA_BF16
+            head = (p(self.out), p(dev["q"]))
+            tail = (p(cache.k_cache), p(cache.v_cache), *sc, p(dev["tables"]), p(dev["lens"]),
+                    p(dev["work"]))
+            rest = (s, hq, hkv, d, bs, nb, mbps, max_len, scale, self.partition_size, *ws,
+                    dcode, st)
+            self._items_at = len(head) + 2 + len(tail)   # where num_items sits in the args
+            self.decode_args = (*head, None, None, *tail, int(num_items), *rest)
+            self.step_args = (*head, p(dev["k_new"]), p(dev["v_new"]), *tail, int(num_items),
+                              *rest)
+            self.fns = (self.fns[0], self.lib.pa_decode_planned, self.lib.pa_decode_planned)
+        self.num_items = int(num_items) if self.planned else 0
         self.fused = fused
         self.launches_per_step = (1 if fused else 2) + (1 if self.num_partitions > 1 else 0)
         self.prefix_len = prefix_len
@@ -312,6 +355,13 @@ class StepCalls:
             self.fused = True
             self.launches_per_step = 3
             self.partition_size = partition_size   # 0: the library's choice for the suffixes
+
+    def set_items(self, num_items):
+        """A new plan of another length in the same work-list buffer."""
+        i = self._items_at
+        self.decode_args = (*self.decode_args[:i], int(num_items), *self.decode_args[i + 1:])
+        self.step_args = (*self.step_args[:i], int(num_items), *self.step_args[i + 1:])
+        self.num_items = int(num_items)
 
     def _call(self, fn, args):
         st = fn(*args)
@@ -760,8 +810,14 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
     steps_after = 10 if name == "large_batch" else 0
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl2, device,
                                                               extra_tokens=steps_after)
-    ps = TUNED_PARTITION[wl2.name.split("_bs")[0]]
-    calls = StepCalls(cache, dev, max_len, wl2.scale, ps, stream)
+    import paged_kv_cache_345_b200 as pa
+
+    ps = TUNED_PARTITION[wl2.name.split("_bs")[0]] or \
+        pa.pa_decode_partition_size(wl2.num_seqs, wl2.num_kv_heads, max_len)
+    items = 0
+    if not args.unplanned:
+        host, dev, items = plan_inputs(host, dev, ps, max_len + steps_after)
+    calls = StepCalls(cache, dev, max_len, wl2.scale, ps, stream, num_items=items)
     clocks = ClockSampler(device.index or 0)
     clocks.start()
     ms = cold_steps(calls.step, flush, steps, warmup, stream)
@@ -774,14 +830,15 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
            "frac": unique / mean_s / 1e9 / peak,
            "attended_tokens_per_s": sum(n + 1 for n in wl2.context_lens) / mean_s,
            "num_seqs": wl2.num_seqs, "block_size": wl2.block_size,
-           "partition_size": calls.partition_size, "steps": steps, "clocks": clk}
+           "partition_size": calls.partition_size, "planned_grid": calls.planned,
+           "steps": steps, "clocks": clk}
     if unique != logical:
         res["kv_bytes_logical"] = logical
         res["GB_per_s_logical"] = logical / mean_s / 1e9
         res["copy_on_write_pairs"] = cow_pairs
     if steps_after:
         res["ten_steps"] = serving_steps(cache, seqs, host, dev, max_len, wl2, stream,
-                                         steps_after)
+                                         steps_after, ps)
     if wl2.shared_prefix:
         # the same step through the cascade entry point: the shared blocks read
         # once for the whole batch
@@ -806,15 +863,17 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
     return res
 
 
-def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
+def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps, partition_size):
     """`steps` decode steps of a serving loop after the timed step above: per
     step, the host block manager's step through the C ABI (the next slot of
     every sequence, a new block where the tail is full, the copy-on-write
     check, the new tables), its output (slots, tables, lengths) host -> device
     in one copy, and the fused append + decode. q and the new K/V rows are the
     previous layer's output in a model, so they are staged on the device
-    beforehand (one set per step, each step's call reading its own). Contexts grow by one token a step. Host
-    time by perf_counter, device time (the copy + the kernels) by CUDA events."""
+    beforehand (one set per step, each step's call reading its own). Contexts grow by one token a step. With a
+    work list in the pack (plan_inputs), each step also plans its decode grid
+    from the new lengths (pa_decode_plan, host) into the pack. Host time by
+    perf_counter, device time (the copy + the kernels) by CUDA events."""
     import torch
 
     import paged_kv_cache_345_b200 as pa
@@ -829,11 +888,16 @@ def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
                  synth.new_token_kv(wl.value_seed, 100 + i, s, wl.num_kv_heads, wl.head_dim)])
               for i in range(steps)]
     # one marshalled call per step, reading that step's staged q and rows
-    calls = [StepCalls(cache, dict(dev, q=q, k_new=k, v_new=v), max_len + steps, wl.scale, 0,
-                       stream) for q, k, v in staged]
-    # the block manager's part of the packed inputs: slots, tables, lengths (contiguous)
+    planned = "work" in dev
+    calls = [StepCalls(cache, dict(dev, q=q, k_new=k, v_new=v), max_len + steps, wl.scale,
+                       partition_size, stream, num_items=1 if planned else 0)
+             for q, k, v in staged]
+    # the host-made part of the packed inputs: slots, tables, lengths (and the
+    # work list), contiguous
+    last = dev["work"] if planned else dev["lens"]
     lo = dev["slots"].data_ptr() - dev["_pack"].data_ptr()
-    hi = dev["lens"].data_ptr() + dev["lens"].numel() * 4 - dev["_pack"].data_ptr()
+    hi = last.data_ptr() + last.numel() * 4 - dev["_pack"].data_ptr()
+    work_buf = host["work"].numpy() if planned else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     host_us, bytes_step, new_blocks = [], [], 0
     # the block manager writes straight into the pinned pack (no allocation per step)
@@ -847,7 +911,11 @@ def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
         t0 = time.perf_counter()
         slots, cows = cache.bm.append_slots(ids, ones, slot_buf, cow_buf)
         tables, lens = cache.bm.block_tables(ids, mbps, tab_buf, len_buf)
+        if planned:
+            n_items = len(pa.pa_decode_plan(lens, partition_size, out=work_buf))
         host_us.append(1e6 * (time.perf_counter() - t0))
+        if planned:
+            calls[i].set_items(n_items)
         new_blocks += free_before - cache.bm.allocator.num_free()
         if len(cows):
             pa.pa_copy_blocks(cache.k_cache, cache.v_cache, torch.from_numpy(cows).to(dev["q"].device))
@@ -868,10 +936,13 @@ def serving_steps(cache, seqs, host, dev, max_len, wl, stream, steps):
             "mean_kv_GB_per_s": statistics.mean(b / (u * 1e-6) / 1e9
                                                 for b, u in zip(bytes_step, dev_us)),
             "new_blocks": new_blocks,
-            "how": "per step: pa_bm_append_slots + pa_bm_block_tables (host, through the "
-                   "binding, written straight into the pinned input pack); slots, tables and "
-                   "lengths host -> device in one copy; "
-                   "pa_decode_append on q and new rows staged on the device (a model's "
+            "how": "per step: pa_bm_append_slots + pa_bm_block_tables" +
+                   (" + pa_decode_plan" if planned else "") +
+                   " (host, through the binding, written straight into the pinned input "
+                   "pack); slots, tables, lengths" + (" and work list" if planned else "") +
+                   " host -> device in one copy; " +
+                   ("pa_decode_planned" if planned else "pa_decode_append") +
+                   " (append + decode) on q and new rows staged on the device (a model's "
                    "previous layer makes them); no L2 flush (the cache is 0.63 GB)"}
 
 
@@ -883,7 +954,7 @@ def pa_device_errors_or_raise():
 
 
 def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp8=False,
-                  prefix_len=0):
+                  prefix_len=0, num_items=0):
     """StepCalls over `layers` copies of the cache (one per model layer)."""
     import paged_kv_cache_345_b200 as pa  # noqa: F401
 
@@ -894,7 +965,7 @@ def replica_calls(cache, dev, max_len, scale, ps, stream, layers, fused=True, fp
         if fp8:
             view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
         out.append(StepCalls(view, dev, max_len, scale, ps, stream, fused=fused,
-                             prefix_len=prefix_len))
+                             prefix_len=prefix_len, num_items=num_items))
     return out
 
 
@@ -927,7 +998,7 @@ def back_to_back(layer_calls, stream, reps, early):
 
 
 def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early, fp8=False,
-                   prefix_len=0):
+                   prefix_len=0, num_items=0):
     """End to end through the C ABI with the host copies pipelined: two pinned
     host packs and two device packs; for step i the inputs go host -> device on
     an upload stream (pack i % 2, once step i - 2 has finished reading it), the
@@ -949,7 +1020,7 @@ def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early,
         if fp8:
             view.k_scale, view.v_scale = cache.k_scale, cache.v_scale
         calls.append(StepCalls(view, packs[i % 2][1], max_len, scale, ps, stream,
-                               prefix_len=prefix_len))
+                               prefix_len=prefix_len, num_items=num_items))
     outs_host = [torch.empty(calls[0].out.shape, dtype=calls[0].out.dtype).pin_memory()
                  for _ in range(2)]
     up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
@@ -1025,9 +1096,15 @@ def run_b200(args, wl, rank, world, local_rank):
             raise SystemExit("--cascade needs a workload with a shared prefix")
         prefix_len = (wl.shared_prefix // wl.block_size) * wl.block_size
         ps = 0 if args.partition_size < 0 else args.partition_size
+    items = 0
+    if not prefix_len and not args.unplanned and wl.cache_dtype in ("bf16", "fp8_e4m3"):
+        # the decode grid from the host lengths: no CTAs past a sequence's end
+        ps = ps or pa.pa_decode_partition_size(wl.num_seqs, wl.num_kv_heads, max_len)
+        host, dev, items = plan_inputs(host, dev, ps)
     calls = StepCalls(cache, dev, max_len, wl.scale, ps, stream, fused=not args.unfused,
-                      prefix_len=prefix_len)
+                      prefix_len=prefix_len, num_items=items)
     launches_per_step, part_size = calls.launches_per_step, calls.partition_size
+    planned = calls.planned
     num_partitions = calls.num_partitions
     bytes_step = kv_bytes_unique(wl)
     bytes_logical = kv_bytes(wl)
@@ -1054,7 +1131,7 @@ def run_b200(args, wl, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         out_host = torch.empty(calls.out.shape, dtype=calls.out.dtype).pin_memory()
-        h2d = host["_pack"].numel()     # q, new K/V rows, slot mapping, tables, lengths
+        h2d = host["_pack"].numel()     # q, new K/V rows, slot mapping, tables, lengths, work list
         d2h = out_host.numel() * out_host.element_size()
 
         def e2e_step():
@@ -1074,7 +1151,7 @@ def run_b200(args, wl, rank, world, local_rank):
             ov_ms, oh2d, od2h = e2e_overlapped(cache, host, max_len, wl.scale,
                                                calls.partition_size, stream, args.layers,
                                                max(5, min(50, args.steps // args.layers)), early,
-                                               calls.fp8, prefix_len)
+                                               calls.fp8, prefix_len, items)
             pa_device_errors_or_raise()
             e2e["overlapped"] = {
                 "value": bytes_step / (ov_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -1088,7 +1165,7 @@ def run_b200(args, wl, rank, world, local_rank):
     if not args.no_back_to_back and world == 1:
         layer_calls = replica_calls(cache, dev, max_len, wl.scale, calls.partition_size, stream,
                                     args.layers, fused=calls.fused, fp8=calls.fp8,
-                                    prefix_len=prefix_len)
+                                    prefix_len=prefix_len, num_items=items)
         reps = max(5, min(50, args.steps // args.layers))
         per_layer_ms = back_to_back(layer_calls, stream, reps, early)
         pa_device_errors_or_raise()
@@ -1137,6 +1214,7 @@ def run_b200(args, wl, rank, world, local_rank):
                    "attended_tokens": tokens_step, "kv_bytes_per_step": bytes_step,
                    "kv_bytes_logical_per_step": bytes_logical,
                    "partition_size": part_size, "num_partitions": num_partitions,
+                   "planned_grid": planned, "work_items": items,
                    "copy_on_write_pairs": cow_pairs,
                    "placement": args.placement, "kv_cache": wl.cache_dtype,
                    "early_cache_reads": bool(early), "shared_prefix_len": prefix_len,
@@ -1148,9 +1226,12 @@ def run_b200(args, wl, rank, world, local_rank):
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": ("pa_decode_shared_prefix (prefix attention kernel, fused "
                                 "append + suffix decode kernel, merge kernel)" if prefix_len else
-                                "pa_decode_append (fused append + decode kernel, split-K "
-                                "merge kernel)" if not args.unfused else
-                                "pa_kv_append + pa_decode (decode + split-K merge kernels)"),
+                                ("pa_decode_planned" if planned else "pa_decode_append") +
+                                " (fused append + decode kernel, split-K merge kernel)"
+                                if not args.unfused else
+                                "pa_kv_append + " +
+                                ("pa_decode_planned" if planned else "pa_decode") +
+                                " (decode + split-K merge kernels)"),
                      "peak_source": f"{peak_src} hbm_gbs"},
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -77,6 +77,9 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
                                      a bad query_start range or chunk length (below)      */
 #define PA_DEVERR_COPY_PAIR 0x8u  /* pa_copy_blocks: src or dst outside [0, num_blocks)  */
 #define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up               */
+#define PA_DEVERR_PLAN 0x20u      /* pa_decode_planned: a work item outside the batch, or
+                                     a sequence whose partition count differs from the
+                                     one its items were planned with                      */
 
 /* ------------------------------------------------------------------ cache writes */
 
@@ -315,6 +318,80 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                          int max_blocks_per_seq, int max_context_len, float scale,
                          int partition_size, void* workspace, size_t workspace_bytes,
                          pa_stream_t stream);
+
+/*
+ * pa_decode_plan — host-side work list for pa_decode_planned.
+ * The plain decode grid has one CTA per (partition, sequence) up to
+ * max_context_len, so a batch of mixed lengths launches many CTAs that find
+ * their partition past their sequence's end and exit; on the GPU each costs
+ * about as much scheduling time as a short CTA with work. A serving loop
+ * knows every length on the host (its block manager made the tables), so it
+ * can list only the (sequence, partition) pairs that hold tokens, in the
+ * order that shortens the tail of the grid: whole partitions first, then each
+ * sequence's last, shorter one, longest first. "Paged Attention"
+ * (klaylearn.com glossary), definition: the kernel reads a sequence's blocks
+ * through its table; the split of a context into partitions and the order in
+ * which they run change no result.
+ *
+ *   context_lens   HOST int32 [num_seqs]: the lengths the planned call will
+ *                  find in its device context_lens (after the step's append).
+ *   partition_size tokens per partition: a multiple of 16 in [16, 2^20], the
+ *                  value the planned call is given (pa_decode_partition_size()
+ *                  gives the automatic one).
+ *   work           HOST int32 [capacity][2], written: item i is
+ *                  {sequence, partition | (partitions of that sequence << 16)}.
+ *                  A sequence of length L has max(1, ceil(L / partition_size))
+ *                  items (an empty sequence one, which writes its zero rows).
+ *   capacity       items work can hold; num_seqs * ceil(max length /
+ *                  partition_size) (at least num_seqs) always suffices.
+ *   num_items      written: the items listed.
+ * Returns PA_ERR_INVALID for a null pointer, a negative length or a bad
+ * partition_size, PA_ERR_UNSUPPORTED for a sequence of more than 65535
+ * partitions, PA_ERR_INVALID when capacity is too small (num_items then holds
+ * the capacity needed). No GPU work; thread-safe.
+ */
+int pa_decode_plan(const int32_t* context_lens, int num_seqs, int partition_size, int32_t* work,
+                   int capacity, int* num_items);
+
+/*
+ * pa_decode_planned — pa_decode / pa_decode_append / pa_decode_fp8 /
+ * pa_decode_append_fp8 on the grid of a pa_decode_plan work list: one CTA per
+ * item and group of KV heads, none for partitions past a sequence's end. The
+ * arithmetic is that of the unplanned call with the same partition_size, so
+ * the results are bit-identical to it. When one wave of resident CTAs holds
+ * every item (items x KV-head groups <= CTAs per SM x SMs), the order of the
+ * list cannot shorten the tail and the call launches the plain grid instead
+ * (which spares each CTA the read of its item); the list is then not read.
+ *
+ *   k_new, v_new   both NULL (attend only, as pa_decode) or both set (append
+ *                  each newest token first, as pa_decode_append).
+ *   k_scale, v_scale  E4M3 caches (dtype PA_FP8_E4M3): as pa_decode_fp8; NULL
+ *                  for bfloat16 caches.
+ *   work           device int32 [num_items][2] (8-byte aligned), as written by
+ *                  pa_decode_plan for these context lengths and this
+ *                  partition_size; read by the kernel at its start (under
+ *                  PA_DECODE_EARLY_CACHE_READS before the dependent-launch
+ *                  wait, like the tables).
+ *   num_items      in [num_seqs, 65535].
+ *   partition_size the plan's, > 0.
+ *   dtype          PA_BF16 or PA_FP8_E4M3.
+ * Everything else as the unplanned calls, including the workspace
+ * (pa_decode_workspace_bytes with this partition_size). Where the list is
+ * read: an item naming a sequence outside the batch or a partition past
+ * max_context_len sets PA_DEVERR_PLAN and its CTA does nothing; a sequence
+ * whose device length needs another number of partitions than its items say
+ * sets PA_DEVERR_PLAN (its output is then undefined). A list that omits or
+ * repeats items of a sequence while giving the right count is not detected:
+ * the output of that sequence is undefined.
+ */
+int pa_decode_planned(void* out, const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, const float* k_scale, const float* v_scale,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      const int32_t* work, int num_items, int num_seqs, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, void* workspace, size_t workspace_bytes,
+                      pa_dtype dtype, pa_stream_t stream);
 
 /*
  * pa_decode_shared_prefix — decode attention (optionally with the step's

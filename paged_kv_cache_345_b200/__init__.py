@@ -15,6 +15,9 @@ Entry points (same names as the C ABI):
   pa_prefill       causal (chunked) prefill attention over the paged context
   pa_kv_append_fp8, pa_decode_fp8, pa_decode_append_fp8
                    the same over 8-bit E4M3 caches with per-KV-head scales
+  pa_decode_plan, pa_decode_planned
+                   host work list of the (sequence, partition) pairs that hold
+                   tokens, and the decode (bf16 or E4M3) on that grid
   BlockManager     host free list + reference counts + block tables
 """
 
@@ -29,7 +32,7 @@ import numpy as np
 __all__ = [
     "PagedAttentionError", "PA_OK", "PA_ERR_INVALID", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_NO_BLOCKS", "PA_ERR_DEVICE_CHECK", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID",
-    "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
+    "PA_DEVERR_CONTEXT", "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT", "PA_DEVERR_PLAN",
     "lib_path", "pa_kv_append", "pa_copy_blocks", "pa_swap_blocks", "pa_decode",
     "pa_decode_append", "pa_kv_append_fp8", "pa_decode_fp8", "pa_decode_append_fp8", "PA_FP8_E4M3",
     "pa_prefill",
@@ -37,6 +40,7 @@ __all__ = [
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
     "pa_set_decode_options", "PA_DECODE_EARLY_CACHE_READS", "decode_options",
     "pa_decode_contiguous", "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
+    "pa_decode_plan", "pa_decode_planned",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
@@ -44,6 +48,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR
 PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_CONTEXT, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
+PA_DEVERR_PLAN = 0x20
 
 lib_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
 if not os.path.exists(lib_path):
@@ -85,6 +90,9 @@ _sig("pa_decode_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, 
      _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
 _sig("pa_decode_append_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
      _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp)
+_sig("pa_decode_plan", _i32, _i32p, _i32, _i32, _i32p, _i32, ctypes.POINTER(ctypes.c_int))
+_sig("pa_decode_planned", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _i32, _vp)
 _sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _f32, _i32, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
@@ -120,7 +128,8 @@ EXPORTED = (
     "pa_decode_partition_size", "pa_set_decode_options", "pa_decode_workspace_bytes",
     "pa_decode", "pa_decode_append", "pa_decode_contiguous", "pa_decode_shared_prefix",
     "pa_decode_shared_prefix_workspace_bytes",
-    "pa_decode_fp8", "pa_decode_append_fp8", "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
+    "pa_decode_fp8", "pa_decode_append_fp8", "pa_decode_plan", "pa_decode_planned",
+    "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
     "pa_num_blocks", "pa_alloc_set_free_order", "pa_bm_create", "pa_bm_destroy",
@@ -515,6 +524,73 @@ def pa_decode_append_fp8(out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scal
             _dev_ptr(k_new, "k_new", torch.bfloat16), _dev_ptr(v_new, "v_new", torch.bfloat16),
             a["k_cache"], a["v_cache"], a["k_scale"], a["v_scale"], a["tables"], a["lens"],
             *a["sizes"], int(max_context_len), float(scale), int(partition_size), *a["ws"], st))
+
+
+def pa_decode_plan(context_lens, partition_size: int, out=None):
+    """Work list of a planned decode from HOST context lengths (int32 [S]; the
+    lengths the step's device context_lens will hold): int32 [num_items, 2],
+    item = (sequence, partition | partitions of the sequence << 16), whole
+    partitions first, then the ragged last ones, longest first. out: an int32
+    [capacity, 2] array to write into (a view of its first rows is returned).
+    See pa_decode_plan in include/pa.h."""
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    if lens.ndim != 1:
+        raise ValueError("context_lens must be 1-D")
+    ps = int(partition_size)
+    if out is None:
+        per = 1 if lens.size == 0 or ps <= 0 else max(1, -(-int(lens.max()) // ps))
+        out = np.empty((max(1, lens.size * per), 2), dtype=np.int32)
+    elif out.dtype != np.int32 or out.ndim != 2 or out.shape[1] != 2 or \
+            not out.flags.c_contiguous:
+        raise ValueError("out must be a C-contiguous int32 [capacity, 2] array")
+    n = ctypes.c_int(0)
+    _check(_lib.pa_decode_plan(lens.ctypes.data_as(_i32p), lens.size, ps,
+                               out.ctypes.data_as(_i32p), out.shape[0], ctypes.byref(n)))
+    return out[:n.value]
+
+
+def pa_decode_planned(out, q, k_cache, v_cache, block_tables, context_lens, work,
+                      max_context_len: int, scale: float, partition_size: int, workspace=None,
+                      k_new=None, v_new=None, k_scale=None, v_scale=None, stream=None) -> None:
+    """pa_decode (k_new / v_new None) or pa_decode_append on the grid of a work
+    list (device int32 [num_items, 2] from pa_decode_plan with this
+    partition_size), for bf16 caches or E4M3 caches (with k_scale / v_scale).
+    See pa_decode_planned in include/pa.h."""
+    torch = _torch()
+    nb, bs, hkv, d = k_cache.shape
+    s, hq, dq = q.shape
+    if dq != d or out.shape != q.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("q/out/cache shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [S, max_blocks], context_lens [S]")
+    if work.dim() != 2 or work.shape[1] != 2:
+        raise ValueError("work must be [num_items, 2]")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None and (k_new.shape != (s, hkv, d) or v_new.shape != k_new.shape):
+        raise ValueError("k_new/v_new must be [S, num_kv_heads, head_dim]")
+    fp8 = _is_fp8(k_cache)
+    if fp8 != (k_scale is not None) or (k_scale is None) != (v_scale is None):
+        raise ValueError("k_scale and v_scale go with (and only with) E4M3 caches")
+    dt = torch.bfloat16
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev_ptr(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    opt = lambda t, n, ty=None: None if t is None else _dev_ptr(t, n, ty)  # noqa: E731
+    guard, st = _on_device((out, q, k_new, v_new, k_cache, v_cache, k_scale, v_scale,
+                            block_tables, context_lens, work, workspace), stream)
+    with guard:
+        _check(_lib.pa_decode_planned(
+            _dev_ptr(out, "out", dt), _dev_ptr(q, "q", dt), opt(k_new, "k_new", dt),
+            opt(v_new, "v_new", dt), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache", None if fp8 else dt),
+            opt(k_scale, "k_scale", torch.float32), opt(v_scale, "v_scale", torch.float32),
+            _dev_ptr(block_tables, "block_tables", torch.int32),
+            _dev_ptr(context_lens, "context_lens", torch.int32),
+            _dev_ptr(work, "work", torch.int32), work.shape[0], s, hq, hkv, d, bs, nb,
+            block_tables.shape[1], int(max_context_len), float(scale), int(partition_size),
+            ws_ptr, ws_bytes, _dtype_code(k_cache), st))
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,

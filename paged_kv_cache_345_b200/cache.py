@@ -10,11 +10,14 @@ workspace. Each method marshals arguments and calls libpa.so:
   prefill(q, k_rows, v_rows, seq_ids, counts)  append each sequence's chunk
       of counts[i] tokens (write), then causal attention of the chunk's query
       rows over the whole context (pa_prefill); bf16 caches.
-  decode(q, seq_ids)  block tables to the device, then pa_decode.
+  decode(q, seq_ids)  block tables to the device, then pa_decode (bf16 and
+      E4M3 caches: pa_decode_planned on the grid pa_decode_plan lists from the
+      host lengths, which the block manager knows; planned=False: the plain
+      grid, same result).
   decode_step(q, k_new, v_new, seq_ids)  one decode step: reserve each sequence's
       next slot (native; shared tail blocks copied first), then pa_decode_append
       writes the new K/V rows and attends in one launch (fused=False: separate
-      pa_kv_append and pa_decode calls, same result). shared_prefix=n: the
+      pa_kv_append and pa_decode calls, same result); planned grid as decode. shared_prefix=n: the
       sequences' first n tokens (a multiple of the block size) sit in the same
       blocks (forked from one parent): pa_decode_shared_prefix attends them once
       for the batch, beside the decode of each sequence's own tokens; bf16.
@@ -37,7 +40,8 @@ import numpy as np
 import torch
 
 from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_decode_append_fp8,
-               pa_decode_fp8, pa_decode_partition_size, pa_decode_shared_prefix,
+               pa_decode_fp8, pa_decode_partition_size, pa_decode_plan, pa_decode_planned,
+               pa_decode_shared_prefix,
                pa_decode_shared_prefix_workspace_bytes, pa_decode_workspace_bytes, pa_kv_append,
                pa_kv_append_fp8, pa_prefill)
 
@@ -134,10 +138,28 @@ class PagedKVCache:
     # --------------------------------------------------------------- decode
     @_on_stream
     def tables(self, seq_ids, max_blocks_per_seq: int | None = None):
-        """(block_tables, context_lens) of the sequences, as device int32 tensors."""
+        """(block_tables, context_lens, max_context_len) of the sequences: device
+        int32 tensors and the host maximum."""
         mbps = max_blocks_per_seq or max(1, max(self.bm.seq_num_blocks(s) for s in seq_ids))
         tables, lens = self.bm.block_tables(seq_ids, mbps)
         return self._to_device(tables), self._to_device(lens), int(lens.max(initial=0))
+
+    def _planned_decode(self, out, q, k_new, v_new, seq_ids, scale, partition_size):
+        """Tables, lengths and the work list of the host lengths to the device,
+        then pa_decode_planned (with the append when k_new is given)."""
+        num_seqs, num_heads, _ = q.shape
+        mbps = max(1, max(self.bm.seq_num_blocks(s) for s in seq_ids))
+        tables, lens = self.bm.block_tables(seq_ids, mbps)
+        max_len = int(lens.max(initial=0))
+        if partition_size == 0:
+            partition_size = pa_decode_partition_size(num_seqs, self.num_kv_heads, max_len)
+        work = pa_decode_plan(lens, partition_size)
+        ws = self.workspace(num_seqs, num_heads, max_len, partition_size)
+        sc = dict(k_scale=self.k_scale, v_scale=self.v_scale) if self.fp8 else {}
+        pa_decode_planned(out, q, self.k_cache, self.v_cache, self._to_device(tables),
+                          self._to_device(lens), self._to_device(work), max_len, scale,
+                          partition_size, ws, k_new=k_new, v_new=v_new, stream=self.stream, **sc)
+        return out
 
     @_on_stream
     def _decode_step_shared(self, q, k_new, v_new, seq_ids, scale, partition_size, out,
@@ -167,7 +189,12 @@ class PagedKVCache:
         return self._workspace if need > 0 else None
 
     @_on_stream
-    def decode(self, q, seq_ids, scale: float | None = None, partition_size: int = 0, out=None):
+    def decode(self, q, seq_ids, scale: float | None = None, partition_size: int = 0, out=None,
+               planned: bool = True):
+        if planned and self.k_cache.dtype != torch.float32 and len(seq_ids):
+            out = torch.empty_like(q) if out is None else out
+            scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+            return self._planned_decode(out, q, None, None, seq_ids, scale, partition_size)
         num_seqs, num_heads, _ = q.shape
         block_tables, context_lens, max_len = self.tables(seq_ids)
         if partition_size == 0:
@@ -186,7 +213,7 @@ class PagedKVCache:
 
     @_on_stream
     def decode_step(self, q, k_new, v_new, seq_ids, scale=None, partition_size: int = 0,
-                    out=None, fused: bool = True, shared_prefix: int = 0):
+                    out=None, fused: bool = True, shared_prefix: int = 0, planned: bool = True):
         if shared_prefix:
             if self.fp8 or not fused:
                 raise ValueError("shared_prefix: a bf16 cache and the fused step")
@@ -194,10 +221,14 @@ class PagedKVCache:
                                             shared_prefix)
         if not fused:
             self.write(seq_ids, [1] * len(seq_ids), k_new, v_new)
-            return self.decode(q, seq_ids, scale, partition_size, out)
+            return self.decode(q, seq_ids, scale, partition_size, out, planned)
         _, cows = self.bm.append_slots(seq_ids, [1] * len(seq_ids))
         if len(cows):
             pa_copy_blocks(self.k_cache, self.v_cache, self._to_device(cows), stream=self.stream)
+        if planned and self.k_cache.dtype != torch.float32 and len(seq_ids):
+            out = torch.empty_like(q) if out is None else out
+            scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+            return self._planned_decode(out, q, k_new, v_new, seq_ids, scale, partition_size)
         num_seqs, num_heads, _ = q.shape
         block_tables, context_lens, max_len = self.tables(seq_ids)
         if partition_size == 0:

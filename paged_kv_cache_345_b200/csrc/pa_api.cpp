@@ -2,8 +2,10 @@
 // Nothing here touches device memory except through the launchers.
 #include <cmath>
 #include <cstdarg>
+#include <algorithm>
 #include <cstdio>
 #include <string>
+#include <vector>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -402,6 +404,116 @@ int pa_decode_append_fp8(void* out, const void* q, const void* k_new, const void
                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
                        max_context_len, scale, partition_size, workspace, workspace_bytes,
                        PA_FP8_E4M3, k_new, v_new, k_scale, v_scale, stream);
+}
+
+int pa_decode_plan(const int32_t* context_lens, int num_seqs, int partition_size, int32_t* work,
+                   int capacity, int* num_items) {
+  if (!num_items || (num_seqs > 0 && (!context_lens || !work)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_plan: null pointer");
+  *num_items = 0;
+  if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_decode_plan: num_seqs < 0");
+  if (partition_size <= 0 || partition_size % pa::kChunkTokens != 0 ||
+      partition_size > pa::kMaxPartitionSize)
+    return pa_fail(PA_ERR_INVALID,
+                   "pa_decode_plan: partition_size %d not a multiple of %d in [%d, %d]",
+                   partition_size, pa::kChunkTokens, pa::kChunkTokens, pa::kMaxPartitionSize);
+  // count first: whole partitions, then one shorter last partition per
+  // sequence (or the single item of an empty one)
+  int64_t total = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int L = context_lens[s];
+    if (L < 0) return pa_fail(PA_ERR_INVALID, "pa_decode_plan: context_lens[%d] = %d", s, L);
+    const int64_t n = L == 0 ? 1 : (static_cast<int64_t>(L) + partition_size - 1) / partition_size;
+    if (n > 65535)
+      return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_plan: sequence %d needs %lld partitions",
+                     s, static_cast<long long>(n));
+    total += n;
+  }
+  if (total > capacity) {
+    *num_items = static_cast<int>(std::min<int64_t>(total, INT32_MAX));
+    return pa_fail(PA_ERR_INVALID, "pa_decode_plan: %lld items > capacity %d",
+                   static_cast<long long>(total), capacity);
+  }
+  // Whole partitions first, sequence by sequence; then the ragged last ones
+  // (every sequence whose length is not a multiple of the partition, and the
+  // empty ones), longest first, ties by sequence. The block scheduler hands
+  // CTAs out in grid order, so the short ones fill the tail.
+  thread_local std::vector<int64_t> ragged;
+  ragged.clear();
+  int64_t i = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const int L = context_lens[s];
+    const int n = L == 0 ? 1 : static_cast<int>((static_cast<int64_t>(L) + partition_size - 1) /
+                                                partition_size);
+    const int whole = L / partition_size;
+    for (int k = 0; k < whole; ++k, ++i) {
+      work[2 * i] = s;
+      work[2 * i + 1] = static_cast<int32_t>(static_cast<uint32_t>(n) << 16 | static_cast<uint32_t>(k));
+    }
+    if (whole < n) {
+      const int rest = L - whole * partition_size;  // tokens of the last partition (0: empty)
+      ragged.push_back((static_cast<int64_t>(partition_size - rest) << 32) | s);
+    }
+  }
+  std::sort(ragged.begin(), ragged.end());
+  for (const int64_t key : ragged) {
+    const int s = static_cast<int>(key & 0xffffffff);
+    const int L = context_lens[s];
+    const int n = L == 0 ? 1 : static_cast<int>((static_cast<int64_t>(L) + partition_size - 1) /
+                                                partition_size);
+    work[2 * i] = s;
+    work[2 * i + 1] = static_cast<int32_t>(static_cast<uint32_t>(n) << 16 | static_cast<uint32_t>(n - 1));
+    ++i;
+  }
+  *num_items = static_cast<int>(i);
+  return PA_OK;
+}
+
+int pa_decode_planned(void* out, const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, const float* k_scale, const float* v_scale,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      const int32_t* work, int num_items, int num_seqs, int num_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      int max_blocks_per_seq, int max_context_len, float scale,
+                      int partition_size, void* workspace, size_t workspace_bytes,
+                      pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs == 0) return PA_OK;
+  if (dtype != PA_BF16 && dtype != PA_FP8_E4M3)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_planned: dtype %d (bf16 or E4M3 caches)",
+                   dtype);
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: k_new and v_new must both be set or null");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: misaligned k_new or v_new");
+  if (dtype == PA_BF16 && (k_scale || v_scale))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: scales given for a bf16 cache");
+  if (!work || !aligned(work, 8))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: null or misaligned work list");
+  if (partition_size <= 0)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: partition_size must be the plan's (> 0)");
+  pa::DecodeShape sh;
+  const int st = pa::check_decode_args(out, q, k_cache, v_cache, block_tables, context_lens,
+                                       num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                       num_blocks, max_blocks_per_seq, max_context_len, scale,
+                                       partition_size, workspace, dtype, k_scale, v_scale, &sh);
+  if (st != PA_OK) return st;
+  const int64_t most = static_cast<int64_t>(num_seqs) * std::max(sh.num_partitions, 1);
+  if (num_items < num_seqs || num_items > 65535 || num_items > most)
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: num_items %d outside [%d, %lld]",
+                   num_items, num_seqs, static_cast<long long>(std::min<int64_t>(most, 65535)));
+  const size_t need =
+      pa::workspace_layout(num_seqs, num_heads, num_kv_heads, head_dim, sh.num_partitions).total;
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return pa_fail(PA_ERR_INVALID, "pa_decode_planned: workspace %zu B < %zu B needed",
+                   workspace ? workspace_bytes : size_t(0), need);
+  sh.work = work;
+  sh.num_items = num_items;
+  cudaError_t e = pa::launch_decode(sh, out, q, k_cache, v_cache, block_tables, context_lens,
+                                    workspace, k_new, v_new, k_scale, v_scale,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_decode_planned: no kernel for this shape");
+  return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode_planned launch", e);
 }
 
 // Sizes of a shared-prefix call: suffix partition size, suffix partitions,

@@ -72,6 +72,11 @@ struct DecodeParams {
   // prefix_slots + p, slots 0 .. prefix_slots - 1 holding the prefix's
   // partial results. Both 0 for the other calls.
   int first_token, prefix_slots;
+  // Planned decode (pa_decode_planned): num_items work items {sequence,
+  // partition | partitions of the sequence << 16} made on the host from the
+  // context lengths, one CTA per item and head group. Null otherwise.
+  const int32_t* work;
+  int num_items;
 };
 
 

@@ -112,13 +112,7 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
                                              ~uintptr_t(127));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kRingBytes);  // full[NS], empty[NS]
 
-  // grid (head group, partition, sequence); E4M3: (head group, sequence,
-  // partition) with the highest partition first, so that the long sequences'
-  // full later partitions start before the many short first ones (the E4M3
-  // kernel's CTAs are slower per byte, and its tail was the longer)
   const int hg = blockIdx.x;
-  const int part = FP8 ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.y);
-  const int s = FP8 ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int P = p.partition_size, bs = p.block_size, lg = p.log2_block_size;
   const int rows_per_box = (!TABLE || bs >= C) ? C : bs;
@@ -154,6 +148,27 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   const bool gate = cascade && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
   if (!early && !cascade) pdl_wait();
   pdl_launch_dependents();
+
+  // grid (head group, partition, sequence); E4M3: (head group, sequence,
+  // partition) with the highest partition first, so that the long sequences'
+  // full later partitions start before the many short first ones (the E4M3
+  // kernel's CTAs are slower per byte, and its tail was the longer).
+  // Planned calls: grid (head group, work item), item y = (sequence, partition
+  // | partitions of that sequence << 16), longest items first, no empty CTAs.
+  int part = FP8 ? static_cast<int>(gridDim.z - 1 - blockIdx.z) : static_cast<int>(blockIdx.y);
+  int s = FP8 ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.z);
+  int planned_parts = 0;
+  if (p.work != nullptr) {
+    const int2 it = __ldg(reinterpret_cast<const int2*>(p.work) + blockIdx.y);
+    s = it.x;
+    part = it.y & 0xffff;
+    planned_parts = static_cast<int>(static_cast<unsigned>(it.y) >> 16);
+    if (static_cast<unsigned>(s) >= static_cast<unsigned>(p.num_seqs) ||
+        part >= p.num_partitions - p.prefix_slots) {
+      if (threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_PLAN);
+      return;
+    }
+  }
 
   // Independent loads first so their latencies overlap: the context length,
   // the first 32 block-table entries of this partition (producer warp) and
@@ -214,6 +229,11 @@ __global__ void __launch_bounds__(GroupConfig<D, G, HB, NS, FP8>::kThreads)
   }
   L -= p.first_token;  // the tokens this kernel attends (all of them without a prefix)
   const int n_part_s = (L + P - 1) / P;
+  if (p.work != nullptr && planned_parts != max(n_part_s, 1)) {
+    // the plan was made for another length of this sequence: flagged, and
+    // the CTA still attends what the real length asks of this partition
+    if (threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_PLAN);
+  }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   const bool to_merge = cascade;  // every row is left to the merge
 

@@ -34,6 +34,10 @@ struct DecodeShape {
   // num_partitions counts the prefix_slots workspace slots before this
   // call's own partitions, and every row goes through the merge
   int first_token, prefix_slots;
+  // pa_decode_planned: the device work list (num_items items) that replaces
+  // the (partition, sequence) grid; null otherwise
+  const int32_t* work;
+  int num_items;
 };
 
 // Byte offsets of the split-K workspace regions.

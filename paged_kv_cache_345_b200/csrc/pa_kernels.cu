@@ -428,14 +428,39 @@ cudaError_t launch_decode_group_t(const DecodeShape& sh, const DecodeParams& p,
   const int rows = (sh.contiguous || sh.block_size >= Cfg::kC) ? Cfg::kC : sh.block_size;
   if ((e = encode_group_map(&kmap, k_cache, sh, rows, HB)) != cudaSuccess) return e;
   if ((e = encode_group_map(&vmap, v_cache, sh, rows, HB)) != cudaSuccess) return e;
+  // A work list pays where its items take more than one wave of resident
+  // CTAs: the longest start first and the short ones fill the tail. When
+  // every item fits in one wave the order does not matter, and the plain
+  // grid (whose CTAs past a sequence's end exit at once) saves each CTA the
+  // read of its item before its table read: same results either way.
+  DecodeParams q = p;
+  const unsigned groups = static_cast<unsigned>(sh.num_kv_heads / HB);
+  if (sh.work != nullptr) {
+    static std::atomic<int> per_sm{0};
+    int fit = per_sm.load(std::memory_order_relaxed);
+    if (fit == 0) {
+      if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kernel, Cfg::kThreads,
+                                                             Cfg::kSmemBytes)) != cudaSuccess)
+        return e;
+      fit = fit < 1 ? 1 : fit;
+      per_sm.store(fit, std::memory_order_relaxed);
+    }
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    if (static_cast<int64_t>(sh.num_items) * groups <= static_cast<int64_t>(fit) * sms)
+      q.work = nullptr;
+  }
   // (a shared-prefix call's own partitions follow the prefix's slots; E4M3:
   // partitions slowest, see the kernel)
   const unsigned parts = static_cast<unsigned>(sh.num_partitions - sh.prefix_slots);
-  const dim3 grid = FP8 ? dim3(sh.num_kv_heads / HB, sh.num_seqs, parts)
-                        : dim3(sh.num_kv_heads / HB, parts, sh.num_seqs);
-  e = launch_pdl(kernel, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, kmap, vmap, p);
+  const dim3 grid = q.work != nullptr ? dim3(groups, sh.num_items, 1)
+                    : FP8            ? dim3(groups, sh.num_seqs, parts)
+                                     : dim3(groups, parts, sh.num_seqs);
+  e = launch_pdl(kernel, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, kmap, vmap, q);
   if (e != cudaSuccess) return e;
-  return launch_merge<__nv_bfloat16, D>(sh, p, stream);
+  return launch_merge<__nv_bfloat16, D>(sh, q, stream);
 }
 
 template <int D, int G, bool FP8>
@@ -527,6 +552,8 @@ cudaError_t launch_decode(const DecodeShape& sh, void* out, const void* q, const
   p.early_reads = sh.early_reads ? 1 : 0;
   p.first_token = sh.first_token;
   p.prefix_slots = sh.prefix_slots;
+  p.work = sh.work;
+  p.num_items = sh.num_items;
   switch (sh.head_dim) {
     case 64: return dispatch_group<64>(sh, p, k_cache, v_cache, stream);
     case 128: return dispatch_group<128>(sh, p, k_cache, v_cache, stream);

@@ -118,10 +118,12 @@ def stage_rows(wl, device="cuda", keep=None):
 
 
 def build_case(wl, device="cuda", free_order=None, partition_size=None, share_prefix=True,
-               staged=None, keep=None, fused=True, poisoned=False):
+               staged=None, keep=None, fused=True, poisoned=False, planned=True):
     """Prefill every sequence, then one decode step (append one token each + attend).
     E4M3 caches (wl.kv_dtype): rows are quantised on the device; the kept rows
-    are replaced by the oracle's cache values of the same rows."""
+    are replaced by the oracle's cache values of the same rows. planned: the
+    step's decode on the work-list grid (bf16 and E4M3 caches; the cache's
+    default), else on the plain (partition, sequence) grid."""
     from paged_kv_cache_345_b200.cache import PagedKVCache
 
     bs = wl.block_size
@@ -170,7 +172,7 @@ def build_case(wl, device="cuda", free_order=None, partition_size=None, share_pr
     k_new, v_new = sk.index_select(0, last), sv.index_select(0, last)
     ps = wl.partition_size if partition_size is None else partition_size
     qd = torch.from_numpy(q).to(device=device, dtype=tdt)
-    out = cache.decode_step(qd, k_new, v_new, seqs, wl.scale, ps, fused=fused)
+    out = cache.decode_step(qd, k_new, v_new, seqs, wl.scale, ps, fused=fused, planned=planned)
     torch.cuda.synchronize()
     if fp8:
         rows_k = {s: e4m3_values(e4m3_codes(r, ks), ks) for s, r in rows_k.items()}

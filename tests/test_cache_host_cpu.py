@@ -16,7 +16,7 @@ from paged_kv_cache_345_b200.cache import PagedKVCache
 
 NB, BS, HKV, HQ, D = 32, 4, 2, 4, 8
 CALLS = ("pa_kv_append", "pa_kv_append_fp8", "pa_copy_blocks", "pa_decode", "pa_decode_fp8",
-         "pa_decode_append", "pa_decode_append_fp8", "pa_prefill")
+         "pa_decode_append", "pa_decode_append_fp8", "pa_decode_planned", "pa_prefill")
 
 
 @pytest.fixture
@@ -24,8 +24,9 @@ def rec(monkeypatch):
     log = []
 
     def recorder(name):
+        # positional arguments, then the keyword ones as one dict at the end
         def fn(*args, **kwargs):
-            log.append((name, args))
+            log.append((name, args + (kwargs,)))
         return fn
 
     for name in CALLS:
@@ -67,23 +68,36 @@ def test_write_fork_decode_step_and_prefill_match_the_oracle(rec):
     # the shared, partly filled tail first
     s1, r1 = cache.fork(s0), ref.fork(r0)
     rec.clear()
-    out = cache.decode_step(torch.zeros((2, HQ, D), dtype=torch.bfloat16), rows(2), rows(2),
-                            [s0, s1])
+    kn, vn = rows(2), rows(2)
+    out = cache.decode_step(torch.zeros((2, HQ, D), dtype=torch.bfloat16), kn, vn, [s0, s1])
     _, cow0 = ref.append_slot(r0)
     _, cow1 = ref.append_slot(r1)
     assert cow0 is not None and cow1 is None
-    assert [n for n, _ in rec] == ["pa_copy_blocks", "pa_decode_append"]
+    assert [n for n, _ in rec] == ["pa_copy_blocks", "pa_decode_planned"]
     assert rec[0][1][2].tolist() == [list(cow0)]
+    # (out, q, k_cache, v_cache, tables, lens, work, max_len, scale, partition, ws, kwargs)
     a = rec[1][1]
     t, lens = _tables(ref, [r0, r1])
-    assert np.array_equal(a[6].numpy(), t) and a[7].tolist() == lens.tolist() == [7, 7]
-    assert a[8] == 7 and a[9] == pytest.approx(1 / np.sqrt(D)) and out.shape == (2, HQ, D)
+    assert np.array_equal(a[4].numpy(), t) and a[5].tolist() == lens.tolist() == [7, 7]
+    ps = a[9]
+    assert ps == cm.pa_decode_partition_size(2, HKV, 7)
+    assert np.array_equal(a[6].numpy(), cm.pa_decode_plan(lens, ps))
+    assert a[7] == 7 and a[8] == pytest.approx(1 / np.sqrt(D)) and out.shape == (2, HQ, D)
+    assert a[-1]["k_new"] is kn and a[-1]["v_new"] is vn
 
     # decode: the same tables, no writes
     rec.clear()
     cache.decode(torch.zeros((2, HQ, D), dtype=torch.bfloat16), [s1, s0])
     (name, a), = rec
     t, lens = _tables(ref, [r1, r0])
+    assert name == "pa_decode_planned" and np.array_equal(a[4].numpy(), t)
+    assert a[5].tolist() == lens.tolist() and a[7] == 7
+    assert a[-1]["k_new"] is None and a[-1]["v_new"] is None
+
+    # the plain grid on request: pa_decode_append / pa_decode with the same tables
+    rec.clear()
+    cache.decode(torch.zeros((2, HQ, D), dtype=torch.bfloat16), [s1, s0], planned=False)
+    (name, a), = rec
     assert name == "pa_decode" and np.array_equal(a[4].numpy(), t)
     assert a[5].tolist() == lens.tolist() and a[6] == 7
 
@@ -116,8 +130,14 @@ def test_fp8_cache_routes_to_the_e4m3_calls(rec):
     slots, _ = ref.add_tokens(r0, 5)
     cache.decode_step(torch.zeros((1, HQ, D), dtype=torch.bfloat16), rows(1), rows(1), [s0])
     cache.decode(torch.zeros((1, HQ, D), dtype=torch.bfloat16), [s0])
-    assert [n for n, _ in rec] == ["pa_kv_append_fp8", "pa_decode_append_fp8", "pa_decode_fp8"]
+    cache.decode_step(torch.zeros((1, HQ, D), dtype=torch.bfloat16), rows(1), rows(1), [s0],
+                      planned=False)
+    cache.decode(torch.zeros((1, HQ, D), dtype=torch.bfloat16), [s0], planned=False)
+    assert [n for n, _ in rec] == ["pa_kv_append_fp8", "pa_decode_planned", "pa_decode_planned",
+                                   "pa_decode_append_fp8", "pa_decode_fp8"]
     assert rec[0][1][2].tolist() == slots
+    for _, a in rec[1:3]:   # the planned calls carry the per-head scales
+        assert a[-1]["k_scale"] is cache.k_scale and a[-1]["v_scale"] is cache.v_scale
     with pytest.raises(NotImplementedError):
         cache.prefill(torch.zeros((1, HQ, D), dtype=torch.bfloat16), rows(1), rows(1), [s0], [1])
 
@@ -131,8 +151,14 @@ def test_unfused_step_writes_then_decodes(rec):
     cache.decode_step(torch.zeros((1, HQ, D), dtype=torch.bfloat16), rows(1), rows(1), [s0],
                       fused=False)
     slots, _ = ref.add_tokens(r0, 1)
-    assert [n for n, _ in rec] == ["pa_kv_append", "pa_decode"]
+    assert [n for n, _ in rec] == ["pa_kv_append", "pa_decode_planned"]
     assert rec[0][1][2].tolist() == slots and rec[1][1][5].tolist() == [5]
+    rec.clear()
+    cache.decode_step(torch.zeros((1, HQ, D), dtype=torch.bfloat16), rows(1), rows(1), [s0],
+                      fused=False, planned=False)
+    slots, _ = ref.add_tokens(r0, 1)
+    assert [n for n, _ in rec] == ["pa_kv_append", "pa_decode"]
+    assert rec[0][1][2].tolist() == slots and rec[1][1][5].tolist() == [6]
 
 
 def test_block_manager_output_buffers():
