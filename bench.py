@@ -803,10 +803,14 @@ def cpu_baseline_line(wl, bytes_step, budget_s):
 
 def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
     """One more workload in the same process: the fused decode step, cold (L2
-    flushed), its rate against the HBM peak, with its own clock record."""
+    flushed), its rate against the HBM peak, with its own clock record. A name
+    ending in _fp8 is the same workload over an E4M3 cache."""
     import torch
 
-    wl2 = make_workload(name, 16)
+    fp8 = name.endswith("_fp8")
+    wl2 = make_workload(name[:-4] if fp8 else name, 16)
+    if fp8:
+        wl2 = dataclasses.replace(wl2, kv_dtype="fp8_e4m3")
     steps_after = 10 if name == "large_batch" else 0
     cache, seqs, host, dev, max_len, cow_pairs = build_on_gpu(wl2, device,
                                                               extra_tokens=steps_after)
@@ -829,7 +833,7 @@ def measure_workload(name, args, device, stream, flush, peak, steps, warmup=3):
            "kv_bytes_per_step": unique, "GB_per_s": unique / mean_s / 1e9,
            "frac": unique / mean_s / 1e9 / peak,
            "attended_tokens_per_s": sum(n + 1 for n in wl2.context_lens) / mean_s,
-           "num_seqs": wl2.num_seqs, "block_size": wl2.block_size,
+           "num_seqs": wl2.num_seqs, "block_size": wl2.block_size, "kv_cache": wl2.cache_dtype,
            "partition_size": calls.partition_size, "planned_grid": calls.planned,
            "steps": steps, "clocks": clk}
     if unique != logical:
@@ -1068,7 +1072,7 @@ def e2e_overlapped(cache, host, max_len, scale, ps, stream, layers, reps, early,
 
 
 # workloads measured beside the headline one, in the same process
-SIDE_WORKLOADS = ("large_batch", "long_context", "shared_prefix")
+SIDE_WORKLOADS = ("large_batch", "large_batch_fp8", "long_context", "shared_prefix")
 
 
 def run_b200(args, wl, rank, world, local_rank):
