@@ -186,3 +186,57 @@ def test_planned_steps_in_a_serving_loop_and_a_graph():
     assert torch.equal(out, eager)
     del graph
     assert pa.pa_device_errors() == 0
+
+
+LLAMA_LENS = (128, 700, 1500, 300, 2900, 50, 4100, 900)
+
+
+@pytest.mark.parametrize("kv", ["", gh.FP8])
+@pytest.mark.parametrize("hq,hkv,ps", [(32, 8, 96), (32, 8, 512), (8, 8, 128), (32, 4, 160)])
+def test_one_wave_planned_calls_match_the_unplanned_ones(kv, hq, hkv, ps):
+    """Batches whose items fit one wave (the Llama-3-8B layer's lengths): the
+    planned call runs the plain grid; it equals the unplanned call bit for bit,
+    call after call, and in a CUDA graph replayed three times."""
+    wl = _custom(hq, hkv, 128, 16, LLAMA_LENS, kv, seed=21)
+    a, b = _pair(wl, ps)
+    _same(a, b, f"{kv or 'bf16'} {hq}/{hkv} P={ps}")
+    tables, lens_d, max_len = a.cache.tables(a.seqs)
+    lens = lens_d.cpu().numpy()
+    work = torch.from_numpy(np.ascontiguousarray(pa.pa_decode_plan(lens, ps))).cuda()
+    n = len(LLAMA_LENS)
+    ws = a.cache.workspace(n, hq, max_len, ps)
+    sc = dict(k_scale=a.cache.k_scale, v_scale=a.cache.v_scale) if kv else {}
+    rng = np.random.default_rng(ps + hq)
+    for i in range(3):
+        q = torch.from_numpy(rng.standard_normal((n, hq, 128)).astype(np.float32))
+        q = q.to("cuda", torch.bfloat16)
+        got, want = torch.empty_like(q), torch.empty_like(q)
+        pa.pa_decode_planned(got, q, a.cache.k_cache, a.cache.v_cache, tables, lens_d, work,
+                             max_len, wl.scale, ps, ws, **sc)
+        if kv:
+            pa.pa_decode_fp8(want, q, b.cache.k_cache, b.cache.v_cache, b.cache.k_scale,
+                             b.cache.v_scale, tables, lens_d, max_len, wl.scale, ps,
+                             b.cache.workspace(n, hq, max_len, ps))
+        else:
+            pa.pa_decode(want, q, b.cache.k_cache, b.cache.v_cache, tables, lens_d, max_len,
+                         wl.scale, ps, b.cache.workspace(n, hq, max_len, ps))
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), f"call {i}"
+    q = torch.from_numpy(rng.standard_normal((n, hq, 128)).astype(np.float32))
+    q = q.to("cuda", torch.bfloat16)
+    eager, out = torch.empty_like(q), torch.zeros_like(q)
+    pa.pa_decode_planned(eager, q, a.cache.k_cache, a.cache.v_cache, tables, lens_d, work,
+                         max_len, wl.scale, ps, ws, **sc)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        pa.pa_decode_planned(out, q, a.cache.k_cache, a.cache.v_cache, tables, lens_d, work,
+                             max_len, wl.scale, ps, ws, stream=stream, **sc)
+    for _ in range(3):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    del graph
+    assert pa.pa_device_errors() == 0
