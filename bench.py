@@ -749,6 +749,25 @@ def host_allocator_metrics(steps: int = 10):
         if pa._lib.pa_bm_append_slots(*args_a) or pa._lib.pa_bm_block_tables(*args_t):
             raise RuntimeError(pa._lib.pa_last_error().decode())
         c_times.append(time.perf_counter() - t0)
+    # the decode's work list for the lengths the last step left (pa_decode_plan,
+    # host only): through the binding into a caller buffer, then through the C ABI
+    plan_lens = len_buf.copy()
+    ps = pa.pa_decode_partition_size(len(seqs), wl.num_kv_heads, int(plan_lens.max()))
+    cap = len(seqs) * max(1, -(-int(plan_lens.max()) // ps))
+    work_buf = np.empty((cap, 2), dtype=np.int32)
+    nitems = ctypes.c_int(0)
+    args_p = (plan_lens.ctypes.data_as(i32p), len(seqs), ps, work_buf.ctypes.data_as(i32p), cap,
+              ctypes.byref(nitems))
+    p_times, pc_times = [], []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        pa.pa_decode_plan(plan_lens, ps, out=work_buf)
+        p_times.append(time.perf_counter() - t0)
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        if pa._lib.pa_decode_plan(*args_p):
+            raise RuntimeError(pa._lib.pa_last_error().decode())
+        pc_times.append(time.perf_counter() - t0)
     new_blocks = free0 - bm.allocator.num_free()
     held = sum(bm.seq_num_blocks(s) for s in seqs)
     tokens = sum(bm.seq_len(s) for s in seqs)
@@ -780,6 +799,12 @@ def host_allocator_metrics(steps: int = 10):
                     "the caller's arrays (10 more), the c_abi one through ctypes with "
                     "preallocated buffers (10 more)",
             "utilisation_after": tokens / (held * wl.block_size)},
+        "decode_plan": {
+            "us_p50_binding": 1e6 * statistics.median(p_times),
+            "us_p50_c_abi": 1e6 * statistics.median(pc_times),
+            "items": int(nitems.value), "partition_size": ps, "sequences": len(seqs),
+            "what": "pa_decode_plan of the 256 lengths (the planned decode's work list), "
+                    "into a caller buffer: through the binding, then through ctypes"},
         "cache_utilisation": {
             "workload": "worked example (8 requests, block 16)",
             "paged_before_step": t_pre / s_pre, "paged_after_step": t_post / s_post,

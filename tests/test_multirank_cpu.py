@@ -155,3 +155,5 @@ def test_host_metrics_reproduce_the_worked_example():
     a = m["allocator_step"]
     assert a["sequences"] == 256 and a["us_per_step_p50"] > 0 and a["us_per_step_c_abi_p50"] > 0
     assert 0.9 < a["utilisation_after"] <= 1.0
+    dp = m["decode_plan"]
+    assert dp["sequences"] == 256 and dp["items"] >= 256 and dp["us_p50_c_abi"] > 0
