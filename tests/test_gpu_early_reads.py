@@ -143,3 +143,55 @@ def test_option_is_per_thread_and_restored():
         assert pa.pa_set_decode_options(pa.PA_DECODE_EARLY_CACHE_READS) == \
             pa.PA_DECODE_EARLY_CACHE_READS
     assert pa.pa_set_decode_options(0) == 0
+
+
+@pytest.mark.parametrize("kv", ["", "fp8_e4m3"])
+def test_chained_planned_decodes_equal_normal_mode(kv):
+    """The same chain through pa_decode_planned with a work list of more items
+    than one wave (partitions of 16 tokens: 665 items), so the list is read
+    before the dependent-launch wait under the option: bit-identical to the
+    chain without it, and to the unplanned chain."""
+    import dataclasses
+
+    import numpy as np
+
+    wl = configs.llama3_8b_layer()
+    if kv:
+        wl = dataclasses.replace(wl, kv_dtype=kv)
+    ps = 16
+    case = gh.build_case(wl, partition_size=ps)
+    tables, lens, max_len = case.cache.tables(case.seqs)
+    work = torch.from_numpy(np.ascontiguousarray(pa.pa_decode_plan(lens.cpu().numpy(), ps)))
+    work = work.cuda()
+    assert work.shape[0] * 2 > 444
+    s, hq, d = case.q.shape
+    need = pa.pa_decode_workspace_bytes(s, hq, case.cache.num_kv_heads, d, max_len, ps)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    sc = dict(k_scale=case.cache.k_scale, v_scale=case.cache.v_scale) if kv else {}
+
+    def chain(early, planned):
+        q = torch.from_numpy(case.q).cuda().to(torch.bfloat16)
+        outs = []
+        with pa.decode_options(pa.PA_DECODE_EARLY_CACHE_READS if early else 0):
+            for _ in range(4):
+                out = torch.empty_like(q)
+                if planned:
+                    pa.pa_decode_planned(out, q, case.cache.k_cache, case.cache.v_cache, tables,
+                                         lens, work, max_len, case.scale, ps, ws, **sc)
+                elif kv:
+                    pa.pa_decode_fp8(out, q, case.cache.k_cache, case.cache.v_cache,
+                                     case.cache.k_scale, case.cache.v_scale, tables, lens,
+                                     max_len, case.scale, ps, ws)
+                else:
+                    pa.pa_decode(out, q, case.cache.k_cache, case.cache.v_cache, tables, lens,
+                                 max_len, case.scale, ps, ws)
+                outs.append(out)
+                q = out
+        torch.cuda.synchronize()
+        return outs
+
+    ref = chain(False, False)
+    for early in (False, True):
+        for a, b in zip(ref, chain(early, True)):
+            assert torch.equal(a, b)
+    assert pa.pa_device_errors() == 0
