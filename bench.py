@@ -1541,13 +1541,25 @@ def run_prefill(args, rank, world, local_rank):
     lib = pa._lib
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
     st = ctypes.c_void_p(stream.cuda_stream)
-    call_args = (ptr(out), ptr(q), ptr(cache.k_cache), ptr(cache.v_cache), ptr(tables), ptr(ctx),
-                 ptr(qs_dev), len(lens), total_q, hq, hkv, d, bs, nb, tables.shape[1],
-                 int(max(chunks)), 1 / float(np.sqrt(d)), pa.PA_BF16, st)
+    head = (ptr(out), ptr(q), ptr(cache.k_cache), ptr(cache.v_cache), ptr(tables), ptr(ctx),
+            ptr(qs_dev))
+    rest = (len(lens), total_q, hq, hkv, d, bs, nb, tables.shape[1], int(max(chunks)),
+            1 / float(np.sqrt(d)), pa.PA_BF16, st)
+    planned = not args.unplanned
+    if planned:
+        # the work items listed on the host in the kernel's own order
+        # (pa_prefill_plan): each CTA reads its item instead of searching
+        work_h = pa.pa_prefill_plan(qs, np.asarray(lens, dtype=np.int32), hq, hkv)
+        work_d = torch.from_numpy(np.ascontiguousarray(work_h)).to(device)
+        call_args = (*head, ptr(work_d), len(work_h), *rest)
+        fn, name = lib.pa_prefill_planned, "pa_prefill_planned"
+    else:
+        call_args = (*head, *rest)
+        fn, name = lib.pa_prefill, "pa_prefill"
 
     def step():
-        if lib.pa_prefill(*call_args):
-            raise RuntimeError(f"pa_prefill: {lib.pa_last_error().decode()}")
+        if fn(*call_args):
+            raise RuntimeError(f"{name}: {lib.pa_last_error().decode()}")
 
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush_w = torch.empty(2 * l2 + (64 << 20), dtype=torch.uint8, device=device)
@@ -1610,12 +1622,13 @@ def run_prefill(args, rank, world, local_rank):
             "config": {"workload": args.workload, "num_seqs": len(lens), "cached_before": before,
                        "chunk_tokens": chunks, "num_heads": hq, "num_kv_heads": hkv,
                        "head_dim": d, "block_size": bs, "causal_flops_per_step": flops,
+                       "planned_grid": planned,
                        "l2": "flushed between steps (outside the timed events)"},
             "step_us_p10_p50_p90": [1e3 * float(np.percentile(ms, p)) for p in (10, 50, 90)],
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak,
                          "traffic": load_traffic(f"pa_prefill_{args.workload}", PREFILL_SOURCES),
-                         "kernel": "pa_prefill_kernel",
+                         "kernel": "pa_prefill_kernel (" + name + ")",
                          "peak_source": src},
             "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}), flush=True)
 

@@ -79,7 +79,8 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 #define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up               */
 #define PA_DEVERR_PLAN 0x20u      /* pa_decode_planned: a work item outside the batch, or
                                      a sequence whose partition count differs from the
-                                     one its items were planned with                      */
+                                     one its items were planned with; pa_prefill_planned:
+                                     an item naming a sequence outside the batch          */
 
 /* ------------------------------------------------------------------ cache writes */
 
@@ -510,6 +511,42 @@ int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cach
                int num_kv_heads, int head_dim, int block_size, int num_blocks,
                int max_blocks_per_seq, int max_query_len, float scale, pa_dtype dtype,
                pa_stream_t stream);
+
+/*
+ * pa_prefill_plan — host-side work list for pa_prefill_planned: every work
+ * item (two query tiles of one sequence's chunk, counted from the chunk's
+ * end) in the order pa_prefill's CTAs find for themselves — most key tiles
+ * visited first, ties by sequence, then by item — so that the kernel reads
+ * its item instead of searching for it, and the grid has no CTA past the
+ * last item. The host knows the chunk and context lengths of a step (the
+ * serving loop made them).
+ *
+ *   query_start    HOST int32 [num_seqs + 1], context_lens HOST int32
+ *                  [num_seqs]: the values the planned call's device arrays
+ *                  hold.
+ *   work           HOST int32 [capacity][2], written: {sequence, item}.
+ *   capacity       num_seqs * ceil(max_query_len / (256 / group)) suffices.
+ *   num_items      written: the items listed (capacity needed on
+ *                  PA_ERR_INVALID for a small capacity).
+ * PA_ERR_INVALID for a null pointer, negative rows or more rows than context;
+ * PA_ERR_UNSUPPORTED for a group size outside {1, 2, 4, 8}. No GPU work.
+ *
+ * pa_prefill_planned — pa_prefill on such a list (device int32
+ * [num_items][2], 8-byte aligned; num_items in [0, num_seqs *
+ * ceil(max_query_len / (256 / group))]). Same results, bit for bit. An item
+ * naming a sequence outside the batch sets PA_DEVERR_PLAN and its CTA does
+ * nothing; one past its sequence's items does nothing. Everything else as
+ * pa_prefill.
+ */
+int pa_prefill_plan(const int32_t* query_start, const int32_t* context_lens, int num_seqs,
+                    int num_heads, int num_kv_heads, int32_t* work, int capacity,
+                    int* num_items);
+int pa_prefill_planned(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens,
+                       const int32_t* query_start, const int32_t* work, int num_items,
+                       int num_seqs, int total_q, int num_heads, int num_kv_heads, int head_dim,
+                       int block_size, int num_blocks, int max_blocks_per_seq,
+                       int max_query_len, float scale, pa_dtype dtype, pa_stream_t stream);
 
 /*
  * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.

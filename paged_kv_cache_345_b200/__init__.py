@@ -40,7 +40,7 @@ __all__ = [
     "pa_decode_partition_size", "pa_device_errors", "Allocator", "BlockManager",
     "pa_set_decode_options", "PA_DECODE_EARLY_CACHE_READS", "decode_options",
     "pa_decode_contiguous", "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_bytes",
-    "pa_decode_plan", "pa_decode_planned",
+    "pa_decode_plan", "pa_decode_planned", "pa_prefill_plan", "pa_prefill_planned",
 ]
 
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_DEVICE_CHECK = \
@@ -93,6 +93,10 @@ _sig("pa_decode_append_fp8", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, 
 _sig("pa_decode_plan", _i32, _i32p, _i32, _i32, _i32p, _i32, ctypes.POINTER(ctypes.c_int))
 _sig("pa_decode_planned", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
      _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _i32, _vp)
+_sig("pa_prefill_plan", _i32, _i32p, _i32p, _i32, _i32, _i32, _i32p, _i32,
+     ctypes.POINTER(ctypes.c_int))
+_sig("pa_prefill_planned", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+     _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp)
 _sig("pa_prefill", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
      _i32, _i32, _f32, _i32, _vp)
 _sig("pa_decode_noalloc", _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
@@ -129,6 +133,7 @@ EXPORTED = (
     "pa_decode", "pa_decode_append", "pa_decode_contiguous", "pa_decode_shared_prefix",
     "pa_decode_shared_prefix_workspace_bytes",
     "pa_decode_fp8", "pa_decode_append_fp8", "pa_decode_plan", "pa_decode_planned",
+    "pa_prefill_plan", "pa_prefill_planned",
     "pa_prefill", "pa_decode_noalloc", "pa_decode_noalloc_scratch_bytes", "pa_device_errors",
     "pa_last_error", "pa_status_string", "pa_alloc_create",
     "pa_alloc_destroy", "pa_alloc_block", "pa_incref", "pa_decref", "pa_refcount", "pa_num_free",
@@ -594,7 +599,7 @@ def pa_decode_planned(out, q, k_cache, v_cache, block_tables, context_lens, work
 
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
-               max_query_len: int, scale: float, stream=None) -> None:
+               max_query_len: int, scale: float, stream=None, work=None) -> None:
     """Causal attention of each sequence's newest query rows over its paged context.
 
     q, out: bf16 [total_q, Hq, 128]; sequence s's rows are query_start[s] ..
@@ -609,16 +614,46 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start
         raise ValueError("q/out/cache shape mismatch")
     if block_tables.dim() != 2 or block_tables.shape[0] != s or query_start.shape != (s + 1,):
         raise ValueError("block_tables must be [S, max_blocks], query_start [S + 1]")
+    if work is not None and (work.dim() != 2 or work.shape[1] != 2):
+        raise ValueError("work must be [num_items, 2]")
     bf = torch.bfloat16
-    guard, st = _on_device((out, q, k_cache, v_cache, block_tables, context_lens, query_start),
-                           stream)
-    with guard:
-        _check(_lib.pa_prefill(
-            _dev_ptr(out, "out", bf), _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf),
+    guard, st = _on_device((out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                            work), stream)
+    head = (_dev_ptr(out, "out", bf), _dev_ptr(q, "q", bf), _dev_ptr(k_cache, "k_cache", bf),
             _dev_ptr(v_cache, "v_cache", bf), _dev_ptr(block_tables, "block_tables", torch.int32),
             _dev_ptr(context_lens, "context_lens", torch.int32),
-            _dev_ptr(query_start, "query_start", torch.int32), s, total_q, hq, hkv, d, bs, nb,
-            block_tables.shape[1], int(max_query_len), float(scale), PA_BF16, st))
+            _dev_ptr(query_start, "query_start", torch.int32))
+    rest = (s, total_q, hq, hkv, d, bs, nb, block_tables.shape[1], int(max_query_len),
+            float(scale), PA_BF16, st)
+    with guard:
+        if work is None:
+            _check(_lib.pa_prefill(*head, *rest))
+        else:   # pa_prefill_planned: the kernel reads its item from the list
+            _check(_lib.pa_prefill_planned(*head, _dev_ptr(work, "work", torch.int32),
+                                           work.shape[0], *rest))
+
+
+def pa_prefill_plan(query_start, context_lens, num_heads: int, num_kv_heads: int, out=None):
+    """Work list of a planned prefill from HOST query_start (int32 [S + 1]) and
+    context_lens (int32 [S]): int32 [num_items, 2] of {sequence, item}, in the
+    order pa_prefill's CTAs would find. See pa_prefill_plan in include/pa.h."""
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    if qs.ndim != 1 or lens.ndim != 1 or qs.size != lens.size + 1:
+        raise ValueError("query_start must be [S + 1] and context_lens [S]")
+    if out is None:
+        group = max(1, num_heads // max(1, num_kv_heads))
+        tok = max(1, 256 // group)
+        rows = np.diff(qs).astype(np.int64)
+        out = np.empty((max(1, int(np.sum(np.maximum(0, -(-rows // tok))))), 2), dtype=np.int32)
+    elif out.dtype != np.int32 or out.ndim != 2 or out.shape[1] != 2 or \
+            not out.flags.c_contiguous:
+        raise ValueError("out must be a C-contiguous int32 [capacity, 2] array")
+    n = ctypes.c_int(0)
+    _check(_lib.pa_prefill_plan(qs.ctypes.data_as(_i32p), lens.ctypes.data_as(_i32p), lens.size,
+                                int(num_heads), int(num_kv_heads), out.ctypes.data_as(_i32p),
+                                out.shape[0], ctypes.byref(n)))
+    return out[:n.value]
 
 
 def pa_device_errors(stream=None) -> int:

@@ -9,6 +9,7 @@
 
 #include "pa.h"
 #include "pa_internal.h"
+#include "pa_prefill_order.h"
 
 namespace {
 
@@ -727,12 +728,13 @@ int pa_decode_contiguous(void* out, const void* q, const void* k, const void* v,
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_decode_contiguous launch", e);
 }
 
-int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
-               const int32_t* block_tables, const int32_t* context_lens,
-               const int32_t* query_start, int num_seqs, int total_q, int num_heads,
-               int num_kv_heads, int head_dim, int block_size, int num_blocks,
-               int max_blocks_per_seq, int max_query_len, float scale, pa_dtype dtype,
-               pa_stream_t stream) {
+// pa_prefill, and with a work list (work != null) pa_prefill_planned.
+static int prefill_common(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* query_start, const int32_t* work, int num_items,
+                          int num_seqs, int total_q, int num_heads, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                          int max_query_len, float scale, pa_dtype dtype, pa_stream_t stream) {
   if (num_seqs < 0 || total_q < 0 || max_query_len < 0)
     return pa_fail(PA_ERR_INVALID, "pa_prefill: negative size");
   if (num_seqs == 0 || total_q == 0 || max_query_len == 0) return PA_OK;
@@ -778,11 +780,95 @@ int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cach
   sh.max_blocks_per_seq = max_blocks_per_seq;
   sh.max_query_len = max_query_len;
   sh.scale = scale;
+  if (work != nullptr) {
+    const int64_t most = static_cast<int64_t>(num_seqs) * ((max_query_len + tok - 1) / tok);
+    if (num_items < 0 || num_items > most)
+      return pa_fail(PA_ERR_INVALID, "pa_prefill_planned: num_items %d outside [0, %lld]",
+                     num_items, static_cast<long long>(most));
+    if (num_items == 0) return PA_OK;
+    sh.work = work;
+    sh.num_items = num_items;
+  }
   cudaError_t e = pa::launch_prefill(sh, out, q, k_cache, v_cache, block_tables, context_lens,
                                      query_start, reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported)
     return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill: no kernel for this shape");
   return e == cudaSuccess ? PA_OK : cuda_fail("pa_prefill launch", e);
+}
+
+int pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* block_tables, const int32_t* context_lens,
+               const int32_t* query_start, int num_seqs, int total_q, int num_heads,
+               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               int max_blocks_per_seq, int max_query_len, float scale, pa_dtype dtype,
+               pa_stream_t stream) {
+  return prefill_common(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                        nullptr, 0, num_seqs, total_q, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, max_blocks_per_seq, max_query_len, scale, dtype,
+                        stream);
+}
+
+int pa_prefill_plan(const int32_t* query_start, const int32_t* context_lens, int num_seqs,
+                    int num_heads, int num_kv_heads, int32_t* work, int capacity,
+                    int* num_items) {
+  namespace po = pa::prefill_order;
+  if (!num_items || (num_seqs > 0 && (!query_start || !context_lens || !work)))
+    return pa_fail(PA_ERR_INVALID, "pa_prefill_plan: null pointer");
+  *num_items = 0;
+  if (num_seqs < 0) return pa_fail(PA_ERR_INVALID, "pa_prefill_plan: num_seqs < 0");
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
+    return pa_fail(PA_ERR_INVALID,
+                   "pa_prefill_plan: num_heads %d not a multiple of num_kv_heads %d", num_heads,
+                   num_kv_heads);
+  const int group = num_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8)
+    return pa_fail(PA_ERR_UNSUPPORTED, "pa_prefill_plan: group size %d (built: 1, 2, 4, 8)",
+                   group);
+  const int ctok = 256 / group, keyn = pa::kPrefillKeyTile;
+  // (cost, sequence, item) of every item, then longest first, ties by
+  // sequence, then item: the order the kernel's own search gives
+  struct Item {
+    int cost, s, z;
+  };
+  thread_local std::vector<Item> items;
+  items.clear();
+  for (int s = 0; s < num_seqs; ++s) {
+    const int n = query_start[s + 1] - query_start[s], L = context_lens[s];
+    if (query_start[s] < 0 || n < 0 || L < n)
+      return pa_fail(PA_ERR_INVALID,
+                     "pa_prefill_plan: sequence %d: %d query rows from %d over %d tokens", s, n,
+                     query_start[s], L);
+    const int m = po::num_items(n, ctok);
+    for (int z = 0; z < m; ++z) items.push_back(Item{po::cost(L, n, z, ctok, keyn), s, z});
+  }
+  if (static_cast<int64_t>(items.size()) > capacity) {
+    *num_items = static_cast<int>(std::min<size_t>(items.size(), INT32_MAX));
+    return pa_fail(PA_ERR_INVALID, "pa_prefill_plan: %zu items > capacity %d", items.size(),
+                   capacity);
+  }
+  std::sort(items.begin(), items.end(), [](const Item& a, const Item& b) {
+    return a.cost != b.cost ? a.cost > b.cost : a.s != b.s ? a.s < b.s : a.z < b.z;
+  });
+  for (size_t i = 0; i < items.size(); ++i) {
+    work[2 * i] = items[i].s;
+    work[2 * i + 1] = items[i].z;
+  }
+  *num_items = static_cast<int>(items.size());
+  return PA_OK;
+}
+
+int pa_prefill_planned(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens,
+                       const int32_t* query_start, const int32_t* work, int num_items,
+                       int num_seqs, int total_q, int num_heads, int num_kv_heads, int head_dim,
+                       int block_size, int num_blocks, int max_blocks_per_seq,
+                       int max_query_len, float scale, pa_dtype dtype, pa_stream_t stream) {
+  if (num_seqs > 0 && (!work || !aligned(work, 8)))
+    return pa_fail(PA_ERR_INVALID, "pa_prefill_planned: null or misaligned work list");
+  return prefill_common(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                        work, num_items, num_seqs, total_q, num_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                        max_query_len, scale, dtype, stream);
 }
 
 int pa_device_errors(pa_stream_t stream, unsigned int* flags) {

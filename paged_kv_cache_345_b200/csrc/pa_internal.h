@@ -86,6 +86,10 @@ struct PrefillShape {
   int num_seqs, total_q, num_heads, num_kv_heads, head_dim, block_size, num_blocks;
   int max_blocks_per_seq, max_query_len;
   float scale;
+  // pa_prefill_planned: the device work list (num_items items {sequence,
+  // item}) that replaces the kernel's own search; null otherwise
+  const int32_t* work;
+  int num_items;
 };
 // Causal chunked-prefill attention (pa_prefill.cu); bf16, head_dim 128.
 cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, const void* k_cache,

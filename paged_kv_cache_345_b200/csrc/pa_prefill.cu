@@ -76,6 +76,9 @@ struct PrefillParams {
   float* ws_m;
   float* ws_l;
   float* ws_acc;
+  // pa_prefill_planned: work item jw is {sequence, item} (made on the host in
+  // the order the search below would find); null: the kernel searches
+  const int32_t* work;
 };
 
 template <int G>
@@ -253,7 +256,15 @@ __global__ void __launch_bounds__(PrefillConfig<G>::kThreads, 1)
     pos_last = L - 1;
     nt = (L - key_lo + KEYN - 1) / KEYN;
   } else {
-    if (S <= kOrderMaxSeqs) {
+    if (p.work != nullptr) {
+      const int2 it = __ldg(reinterpret_cast<const int2*>(p.work) + jw);
+      s = it.x;
+      z = it.y;
+      if (static_cast<unsigned>(s) >= static_cast<unsigned>(S) || z < 0) {
+        if (threadIdx.x == 0) atomicOr(p.err, PA_DEVERR_PLAN);
+        return;
+      }
+    } else if (S <= kOrderMaxSeqs) {
       bool bad = false, found;
       if (S <= 32) found = work_item<1, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
       else if (S <= 64) found = work_item<2, CTOK, KEYN>(p, S, jw, lane, &s, &z, &bad);
@@ -710,9 +721,14 @@ cudaError_t launch_prefill(const PrefillShape& sh, void* out, const void* q, con
   p.total_q = sh.total_q;
   p.max_query_len = sh.max_query_len;
   // work indices: every sequence could have max_query_len rows; those past
-  // the last item exit at once (they are dispatched last)
+  // the last item exit at once (they are dispatched last). A planned call's
+  // list has exactly the items that hold rows.
   const int tok = 2 * (128 / (sh.num_heads / sh.num_kv_heads));  // query tokens per CTA
-  const int64_t items = static_cast<int64_t>(sh.num_seqs) * ((sh.max_query_len + tok - 1) / tok);
+  int64_t items = static_cast<int64_t>(sh.num_seqs) * ((sh.max_query_len + tok - 1) / tok);
+  if (sh.work != nullptr) {
+    p.work = sh.work;
+    items = sh.num_items;
+  }
   return dispatch_prefill<false>(p, q, k_cache, v_cache, items * sh.num_kv_heads, stream);
 }
 

@@ -223,3 +223,54 @@ def test_prefill_chunk_above_host_bound_is_flagged_and_skipped():
     assert pa.pa_device_errors() & pa.PA_DEVERR_CONTEXT
     assert bool((out[:5] == 5.0).all())          # skipped
     assert bool((out[5:] == 0.0).all())          # V = 0 everywhere -> zeros
+
+
+def _planned_case(hq, hkv, before, chunks, bs=16):
+    lens = [b + c for b, c in zip(before, chunks)]
+    nb = sum(-(-L // bs) for L in lens) + 8
+    cache = PagedKVCache(nb, bs, hkv, D, "bf16", "cuda",
+                         max_blocks_per_seq=max(1, max(-(-L // bs) for L in lens)),
+                         free_order=synth.block_permutation(nb, 3006 + bs))
+    seqs = [cache.add_sequence() for _ in lens]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", torch.bfloat16)  # noqa
+    rows = [_rows(s, L, hkv) for s, L in enumerate(lens)]
+    cache.write(seqs, lens, dev(np.concatenate([r[0] for r in rows])),
+                dev(np.concatenate([r[1] for r in rows])))
+    q = dev(np.concatenate([_queries(s, c, hq) for s, c in enumerate(chunks)]))
+    tables, ctx, _ = cache.tables(seqs)
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    return cache, q, tables, ctx, qs, np.asarray(lens, dtype=np.int32)
+
+
+@pytest.mark.parametrize("hq,hkv,before,chunks", [
+    (32, 8, [0, 0, 0, 0, 0], [129, 700, 1500, 300, 2900]),      # whole prompts, G = 4
+    (32, 8, [128, 700, 1500, 300], [512, 512, 512, 512]),       # chunks on cached contexts
+    (8, 8, [0, 50, 0, 3], [300, 7, 1000, 0]),                   # G = 1, an empty chunk
+    (32, 4, [10, 0], [600, 900]),                               # G = 8
+])
+def test_planned_prefill_equals_the_searching_kernel(hq, hkv, before, chunks):
+    """pa_prefill_planned on pa_prefill_plan's list: every row computed, bit for
+    bit what pa_prefill (each CTA finding its own item) computes."""
+    cache, q, tables, ctx, qs, lens = _planned_case(hq, hkv, before, chunks)
+    qs_d = torch.from_numpy(qs).cuda()
+    work = torch.from_numpy(np.ascontiguousarray(pa.pa_prefill_plan(qs, lens, hq, hkv))).cuda()
+    a, b = torch.full_like(q, float("nan")), torch.full_like(q, float("nan"))
+    pa.pa_prefill(a, q, cache.k_cache, cache.v_cache, tables, ctx, qs_d, max(chunks),
+                  1 / np.sqrt(D))
+    pa.pa_prefill(b, q, cache.k_cache, cache.v_cache, tables, ctx, qs_d, max(chunks),
+                  1 / np.sqrt(D), work=work)
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() == 0
+    assert not torch.isnan(b).any()
+    assert torch.equal(a, b)
+
+
+def test_planned_prefill_flags_an_item_outside_the_batch():
+    cache, q, tables, ctx, qs, lens = _planned_case(32, 8, [0, 0], [200, 300])
+    work = np.ascontiguousarray(pa.pa_prefill_plan(qs, lens, 32, 8)).copy()
+    work[0, 0] = 2                                   # no sequence 2
+    out = torch.full_like(q, float("nan"))
+    pa.pa_prefill(out, q, cache.k_cache, cache.v_cache, tables, ctx, torch.from_numpy(qs).cuda(),
+                  300, 1 / np.sqrt(D), work=torch.from_numpy(work).cuda())
+    torch.cuda.synchronize()
+    assert pa.pa_device_errors() & pa.PA_DEVERR_PLAN

@@ -1,6 +1,6 @@
-"""Host side of the planned decode: pa_decode_plan's work list and the
-argument checks of pa_decode_planned (no GPU: every rejected call fails before
-any CUDA call).
+"""Host side of the planned calls: pa_decode_plan's and pa_prefill_plan's work
+lists and the argument checks of pa_decode_planned and pa_prefill_planned (no
+GPU: every rejected call fails before any CUDA call).
 
 "Paged Attention" (klaylearn.com glossary), definition: decode reads each
 sequence's blocks through its table; the split of a context into partitions
@@ -134,3 +134,81 @@ def test_planned_decode_rejects_on_host(over, status):
 
 def test_planned_decode_zero_sequences_is_a_no_op():
     assert _planned(S=0, n=0)[0] == pa.PA_OK
+
+
+# ------------------------------------------------------------- prefill plan
+
+def _prefill_items(qs, lens, group, keyn=64):
+    """(-cost, sequence, item) of every item, from the definition: item z of a
+    chunk of n rows holds rows [first, first + rows) counted from the chunk's
+    start, first = (items - 1 - z) * ctok, and its last row sees key
+    L - n + first + rows - 1; its cost is the key tiles up to that key."""
+    ctok = 256 // group
+    out = []
+    for s in range(len(lens)):
+        n, L = int(qs[s + 1] - qs[s]), int(lens[s])
+        items = -(-n // ctok)
+        for z in range(items):
+            first = (items - 1 - z) * ctok
+            rows = min(ctok, n - first)
+            out.append((-((L - n + first + rows - 1) // keyn + 1), s, z))
+    return sorted(out)
+
+
+@pytest.mark.parametrize("seed,group", [(0, 4), (1, 1), (2, 8), (3, 2)])
+def test_prefill_plan_is_longest_first(seed, group):
+    rng = np.random.default_rng(seed)
+    S = 40
+    n = rng.integers(0, 900, size=S)
+    n[rng.integers(0, S, size=5)] = 0                       # sequences without rows
+    lens = (n + rng.integers(0, 5000, size=S)).astype(np.int32)
+    lens[rng.integers(0, S, size=5)] = 0                    # contexts of only the chunk
+    lens = np.maximum(lens, n).astype(np.int32)
+    qs = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    work = pa.pa_prefill_plan(qs, lens, 8 * group, 8)
+    want = _prefill_items(qs, lens, group)
+    assert work[:, 0].tolist() == [s for _, s, _ in want]
+    assert work[:, 1].tolist() == [z for _, _, z in want]
+
+
+def test_prefill_plan_rejects():
+    qs = np.array([0, 10, 30], dtype=np.int32)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_prefill_plan(qs, np.array([10, 19], dtype=np.int32), 32, 8)   # 20 rows over 19
+    assert e.value.status == pa.PA_ERR_INVALID
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_prefill_plan(qs, np.array([10, 30], dtype=np.int32), 24, 8)   # group 3
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+    with pytest.raises(pa.PagedAttentionError) as e:
+        pa.pa_prefill_plan(qs, np.array([10, 30], dtype=np.int32), 32, 8,
+                           out=np.zeros((1, 2), dtype=np.int32))               # capacity
+    assert e.value.status == pa.PA_ERR_INVALID
+
+
+def _prefill_planned(**over):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, qs=FAKE, work=FAKE, n=4, S=2,
+             tq=100, Hq=32, Hkv=8, D=128, bs=16, nb=64, mbps=16, mq=64, scale=0.1,
+             dt=pa.PA_BF16)
+    a.update(over)
+    st = pa._lib.pa_prefill_planned(a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["qs"],
+                                    a["work"], a["n"], a["S"], a["tq"], a["Hq"], a["Hkv"],
+                                    a["D"], a["bs"], a["nb"], a["mbps"], a["mq"], a["scale"],
+                                    a["dt"], None)
+    return st, pa._lib.pa_last_error().decode()
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(work=None), pa.PA_ERR_INVALID),
+    (dict(work=ctypes.c_void_p(0x10004)), pa.PA_ERR_INVALID),
+    (dict(n=-1), pa.PA_ERR_INVALID),
+    (dict(n=3), pa.PA_ERR_INVALID),        # more than S * ceil(64 / 64) = 2 items
+    (dict(dt=pa.PA_F32), pa.PA_ERR_UNSUPPORTED),
+    (dict(Hq=24), pa.PA_ERR_UNSUPPORTED),
+])
+def test_planned_prefill_rejects_on_host(over, status):
+    st, msg = _prefill_planned(**over)
+    assert st == status, msg
+
+
+def test_planned_prefill_without_items_is_a_no_op():
+    assert _prefill_planned(n=0)[0] == pa.PA_OK
