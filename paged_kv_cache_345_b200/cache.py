@@ -9,7 +9,9 @@ workspace. Each method marshals arguments and calls libpa.so:
       (pa_kv_append). Serves both prefill (many tokens) and decode (one token).
   prefill(q, k_rows, v_rows, seq_ids, counts)  append each sequence's chunk
       of counts[i] tokens (write), then causal attention of the chunk's query
-      rows over the whole context (pa_prefill); bf16 caches.
+      rows over the whole context (pa_prefill_planned on the work items
+      pa_prefill_plan lists from the host lengths; planned=False: pa_prefill,
+      same result); bf16 caches.
   decode(q, seq_ids)  block tables to the device, then pa_decode (bf16 and
       E4M3 caches: pa_decode_planned on the grid pa_decode_plan lists from the
       host lengths, which the block manager knows; planned=False: the plain
@@ -43,7 +45,7 @@ from . import (BlockManager, pa_copy_blocks, pa_decode, pa_decode_append, pa_dec
                pa_decode_fp8, pa_decode_partition_size, pa_decode_plan, pa_decode_planned,
                pa_decode_shared_prefix,
                pa_decode_shared_prefix_workspace_bytes, pa_decode_workspace_bytes, pa_kv_append,
-               pa_kv_append_fp8, pa_prefill)
+               pa_kv_append_fp8, pa_prefill, pa_prefill_plan)
 
 _TORCH_DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8_e4m3": torch.uint8}
 
@@ -121,18 +123,27 @@ class PagedKVCache:
 
     # -------------------------------------------------------------- prefill
     @_on_stream
-    def prefill(self, q, k_rows, v_rows, seq_ids, counts, scale: float | None = None, out=None):
+    def prefill(self, q, k_rows, v_rows, seq_ids, counts, scale: float | None = None, out=None,
+                planned: bool = True):
         """Append counts[i] tokens to seq_ids[i] and attend them causally: q, k_rows,
-        v_rows are [sum(counts), H, d] device tensors in sequence order."""
+        v_rows are [sum(counts), H, d] device tensors in sequence order. planned:
+        the work items listed on the host (pa_prefill_plan, pa_prefill_planned);
+        else each CTA finds its own (pa_prefill). Same result."""
         if self.fp8:
             raise NotImplementedError("pa_prefill reads bf16 caches")
         self.write(seq_ids, counts, k_rows, v_rows)
-        block_tables, context_lens, _ = self.tables(seq_ids)
+        mbps = max(1, max(self.bm.seq_num_blocks(s) for s in seq_ids))
+        tables, lens = self.bm.block_tables(seq_ids, mbps)
+        block_tables, context_lens = self._to_device(tables), self._to_device(lens)
         qs = np.concatenate([[0], np.cumsum(np.asarray(counts, dtype=np.int64))]).astype(np.int32)
         out = torch.empty_like(q) if out is None else out
         scale = 1.0 / float(np.sqrt(self.head_dim)) if scale is None else scale
+        work = None
+        if planned and len(seq_ids) and int(qs[-1]) > 0:
+            work = self._to_device(pa_prefill_plan(qs, lens, q.shape[1], self.num_kv_heads))
         pa_prefill(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
-                   self._to_device(qs), int(max(counts, default=0)), scale, stream=self.stream)
+                   self._to_device(qs), int(max(counts, default=0)), scale, stream=self.stream,
+                   work=work)
         return out
 
     # --------------------------------------------------------------- decode
