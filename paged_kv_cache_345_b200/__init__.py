@@ -18,6 +18,9 @@ Entry points (same names as the C ABI):
   pa_decode_plan, pa_decode_planned
                    host work list of the (sequence, partition) pairs that hold
                    tokens, and the decode (bf16 or E4M3) on that grid
+  pa_prefill_plan, pa_prefill_planned
+                   host work list of the prefill's items in the kernel's
+                   longest-first order, and the prefill on it
   BlockManager     host free list + reference counts + block tables
 """
 
